@@ -1,0 +1,545 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other
+than itself — a library E2M1 cast (ml_dtypes), exact comparisons with powers
+of two, exhaustive enumeration of the random numbers, a library Hadamard
+matrix (scipy), published hash vectors, hand-worked groups and the pages'
+worked oscillation example. CPU only.
+"""
+import math
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle as O
+from golden_io import hand_groups, load, unpack_nibbles
+
+F4 = ml_dtypes.float4_e2m1fn
+BF16 = ml_dtypes.bfloat16
+GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        v = bits.view(BF16).astype(np.float64)
+    return bits[np.isfinite(v)], v[np.isfinite(v)]
+
+
+# --------------------------------------------------------------------------
+# Random numbers
+# --------------------------------------------------------------------------
+
+def test_hash_finalizer_published_vectors():
+    for case in load("murmur3_vectors.json")["empty_key"]:
+        assert O.mix32(case["seed"]) == int(case["hash"], 16)
+
+
+def test_hash_frozen_known_answers():
+    kat = load("hash_kat.json")
+    for c in kat["rand16"]:
+        assert O.rand16(c["seed"], c["stream"], c["i"]) == c["r"]
+    for c in kat["rht_sign"]:
+        assert O.rht_sign(c["seed"], c["c"]) == c["s"]
+
+
+def test_rand16_uniform_and_paired():
+    r = O.rand16_range(1234, 0, 0, 1 << 20).astype(np.int64)
+    assert r.max() < 65536
+    # chi-square over 256 bins of the top byte; 255 dof, mean 255, sd ~22.6
+    counts = np.bincount(r >> 8, minlength=256)
+    exp = len(r) / 256
+    chi2 = ((counts - exp) ** 2 / exp).sum()
+    assert chi2 < 255 + 6 * 22.6
+    # the low byte too
+    counts = np.bincount(r & 0xFF, minlength=256)
+    assert ((counts - exp) ** 2 / exp).sum() < 255 + 6 * 22.6
+    # even and odd elements of a pair are the two halves of one 32-bit hash
+    k = O.key(1234, 0)
+    for p in (0, 1, 77, 123456):
+        h = O.counter_hash(k, p)
+        assert r[2 * p] == (h & 0xFFFF) and r[2 * p + 1] == (h >> 16)
+    # streams and seeds give unrelated sequences
+    r1 = O.rand16_range(1234, 1, 0, 4096).astype(np.float64)
+    r2 = O.rand16_range(1235, 0, 0, 4096).astype(np.float64)
+    for other in (r1, r2):
+        assert abs(np.corrcoef(r[:4096], other)[0, 1]) < 0.08
+
+
+def test_counter_hash_high_word_matters():
+    k = O.key(7, 0)
+    assert O.counter_hash(k, 5) != O.counter_hash(k, 5 + (1 << 32))
+
+
+# --------------------------------------------------------------------------
+# Scale exponent: e = floor(log2 absmax) - 2, clamped to [-127, 127]
+# --------------------------------------------------------------------------
+
+def _check_exponent(a, e):
+    if a == 0:
+        assert e == -127
+        return
+    if e > -127:
+        assert math.ldexp(1.0, e + 2) <= a < math.ldexp(1.0, e + 3), (a, e)
+    else:
+        assert a < math.ldexp(1.0, -124), (a, e)
+    assert -127 <= e <= 125
+
+
+def test_scale_exponent_exhaustive_bf16():
+    _, v = all_finite_bf16()
+    for a in np.unique(np.abs(v)):
+        _check_exponent(float(a), O.scale_exponent(float(a)))
+
+
+def test_scale_exponent_fp32_sample_and_edges():
+    g = np.random.Generator(np.random.PCG64(11))
+    bits = g.integers(0, 0x7F800000, size=20000, dtype=np.uint32)
+    vals = list(bits.view(np.float32).astype(np.float64))
+    for k in range(-149, 128):
+        p = math.ldexp(1.0, k)
+        vals += [p, float(np.nextafter(np.float32(p), np.float32(0)))]
+    vals += [float(np.finfo(np.float32).max), 0.0]
+    for a in vals:
+        _check_exponent(a, O.scale_exponent(a))
+
+
+# --------------------------------------------------------------------------
+# E2M1 encoding (Q_D) and decoding, against the ml_dtypes E2M1 cast
+# --------------------------------------------------------------------------
+
+def test_rne_exhaustive_bf16_times_every_scale_against_library():
+    """Every finite bf16 x under every reachable exponent e, through the
+    tensor quantizer: each group holds an anchor that forces e, plus 31 x.
+    Expected codes come from ml_dtypes' round-to-nearest-even E2M1 cast of
+    x * 2^-e."""
+    _, v = all_finite_bf16()
+    anchor_m = 7.96875  # largest bf16 below 8: keeps absmax * 2^-e in [4, 8)
+    groups, expect, exps = [], [], []
+    for e in range(-127, 126):
+        A = math.ldexp(anchor_m, e)
+        xs = v[np.abs(v) <= A]
+        pad = (-len(xs)) % 31
+        xs = np.concatenate([xs, np.zeros(pad)]).reshape(-1, 31)
+        grp = np.concatenate([np.full((len(xs), 1), A), xs], axis=1)
+        groups.append(grp)
+        scaled = (grp * math.ldexp(1.0, -e)).astype(np.float32)
+        expect.append(scaled.astype(F4).view(np.uint8))
+        exps.append(np.full(len(xs), e + 127))
+    x = np.concatenate(groups).astype(np.float32).astype(BF16)
+    expect = np.concatenate(expect)
+    codes, scales = O.quantize(x, O.ROWS, O.RNE)
+    assert np.array_equal(scales[:, 0], np.concatenate(exps))
+    got = unpack_nibbles(codes)
+    bad = np.nonzero(got != expect)
+    assert bad[0].size == 0, (x[bad][:8], got[bad][:8], expect[bad][:8])
+
+
+def test_rne_scalar_ties_and_saturation():
+    # Bin edges (midpoints) and their tie-to-even outcomes; saturation at 6.
+    cases = {0.25: 0, 0.75: 2, 1.25: 2, 1.75: 4, 2.5: 4, 3.5: 6, 5.0: 6,
+             6.0: 7, 7.999: 7, 0.0: 0, 0.2500001: 1, 4.999: 6, 5.0001: 7}
+    for a, m in cases.items():
+        assert O.rne_index(a) == m, a
+        lib = int(np.array([a], np.float32).astype(F4).view(np.uint8)[0])
+        assert lib == m, a
+
+
+def test_sign_of_zero_codes():
+    assert O.encode(-0.0, 0) == 8
+    assert O.encode(-0.1, 0) == 8
+    assert O.encode(0.1, 0) == 0
+
+
+def test_decode_every_code_and_scale_against_library():
+    lib_vals = np.arange(16, dtype=np.uint8).view(F4).astype(np.float64)
+    for sb in range(255):
+        for code in range(16):
+            want = math.ldexp(lib_vals[code], sb - 127)
+            got = O.decode(code, sb)
+            assert got == want and math.copysign(1, got) == math.copysign(1, want)
+    assert math.isnan(O.decode(3, 255))
+
+
+def test_hand_worked_groups():
+    for name, x, sb, codes in hand_groups():
+        c, s = O.quantize(x.reshape(1, 32), O.ROWS, O.RNE)
+        assert s[0, 0] == sb, name
+        assert np.array_equal(unpack_nibbles(c)[0], codes), name
+
+
+def test_dequantize_roundtrip_of_grid_values():
+    # x built from grid values times the group scale is reproduced exactly.
+    g = np.random.Generator(np.random.PCG64(5))
+    R, C = 64, 128
+    e = g.integers(-120, 120, size=(R, C // 32))
+    m = g.integers(0, 8, size=(R, C))
+    m[:, ::32] = 7  # every group holds +-6 * 2^e: absmax fixes e
+    sign = np.where(g.random((R, C)) < 0.5, -1.0, 1.0)
+    vals = sign * np.array(GRID)[m] * np.exp2(np.repeat(e, 32, axis=1))
+    x = vals.astype(np.float32).astype(BF16)
+    assert np.array_equal(x.astype(np.float64), vals)
+    codes, scales = O.quantize(x)
+    assert np.array_equal(scales, (e + 127).astype(np.uint8))
+    y = O.dequantize(codes, scales, R, C)
+    assert np.array_equal(y.view(np.uint16)[vals != 0], x.view(np.uint16)[vals != 0])
+    yf = O.dequantize(codes, scales, R, C, out_dtype="f32")
+    assert np.array_equal(yf.astype(np.float64), vals)
+
+
+# --------------------------------------------------------------------------
+# Stochastic rounding (Q_S)
+# --------------------------------------------------------------------------
+
+def _lo_step(a):
+    lo = max(g for g in GRID if g <= a)
+    hi = GRID[GRID.index(lo) + 1]
+    return lo, hi - lo
+
+
+def test_sr_exhaustive_over_random_numbers_is_unbiased():
+    """For every bf16 magnitude in [2^-6, 6) and every one of the 65536
+    random numbers: the result is lo or hi, and the mean over all random
+    numbers is a within 2^-17 of a step (the closed-form resolution bound)."""
+    _, v = all_finite_bf16()
+    mags = np.unique(np.abs(v[(np.abs(v) >= 2.0 ** -6) & (np.abs(v) < 6)]))
+    for a in mags:
+        a = float(a)
+        lo, step = _lo_step(a)
+        n_up = O.sr_count_up(a)
+        mean = Fraction(lo) + Fraction(step) * Fraction(n_up, 65536)
+        assert abs(mean - Fraction(a)) <= Fraction(step) / (1 << 17), a
+    for a in GRID[:7]:
+        assert O.sr_count_up(a) == 0  # grid values are fixed points
+    for a in (6.0, 6.5, 7.96875):
+        assert all(O.sr_index(a, r) == 7 for r in (0, 1, 40000, 65535))
+
+
+def test_sr_result_is_a_neighbour_and_monotone_in_r():
+    for a in (0.1, 0.3, 0.74, 1.2, 1.9, 2.7, 3.3, 4.8, 5.9):
+        lo, step = _lo_step(a)
+        idx = [O.sr_index(a, r) for r in range(0, 65536, 97)]
+        lo_i = GRID.index(lo)
+        assert set(idx) <= {lo_i, lo_i + 1}
+        assert all(x >= y for x, y in zip(idx, idx[1:]))  # up for small r
+
+
+def test_sr_end_to_end_unbiased_over_elements():
+    """Q_S through the tensor path with the counter hash: every row repeats
+    one group, so the mean over rows estimates E[Q_S(v)] (4 sigma bound)."""
+    S = 8192
+    vals = np.array([6.0, 0.3, 1.1, 2.6, 4.7, 5.2, 0.05, -3.3], np.float64)
+    row = np.zeros(32)
+    row[:8] = vals
+    x = np.tile(row, (S, 1)).astype(np.float32).astype(BF16)
+    xv = x[0].astype(np.float64)
+    codes, scales = O.quantize(x, O.ROWS, O.SR, seed=99)
+    deq = O.dequantize(codes, scales, S, 32, out_dtype="f32").astype(np.float64)
+    for j in range(1, 8):
+        a = abs(xv[j])
+        lo, step = _lo_step(a)
+        p = (a - lo) / step
+        sd = step * math.sqrt(p * (1 - p)) / math.sqrt(S)
+        mean = np.mean(np.abs(deq[:, j]))
+        assert abs(mean - a) <= 4 * sd + step / (1 << 17), (j, mean, a)
+        assert np.all(np.sign(deq[:, j]) * np.sign(xv[j]) >= 0)
+
+
+def test_sr_saturation_bias_documented():
+    # a in (6, 8) always goes to 6: Q_S is biased there under this scale rule.
+    assert O.sr_count_up(6.7) == 0 and O.sr_index(6.7, 0) == 7
+
+
+# --------------------------------------------------------------------------
+# Layouts: brute force on tiny tensors with exact rationals
+# --------------------------------------------------------------------------
+
+def _brute_group(xs):
+    """Exact brute force of one RNE group: search the exponent, then try
+    all 16 codes in the value domain."""
+    fx = [Fraction(float(t)) for t in xs]
+    amax = max(abs(t) for t in fx)
+    if amax == 0:
+        k = -200
+    else:
+        k = 0
+        while Fraction(2) ** k > amax:
+            k -= 1
+        while Fraction(2) ** (k + 1) <= amax:
+            k += 1
+    e = min(max(k - 2, -127), 127)
+    out = []
+    for t in fx:
+        best = None
+        for code in range(16):
+            val = (-1 if code & 8 else 1) * Fraction(GRID[code & 7]) * Fraction(2) ** e
+            if (code & 8) != (8 if math.copysign(1, float(t)) < 0 else 0):
+                continue
+            d = abs(t - val)
+            if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
+                best = (d, code)
+        out.append(best[1])
+    return e + 127, out
+
+
+@pytest.mark.parametrize("shape,axis", [((32, 32), O.ROWS), ((64, 96), O.ROWS),
+                                        ((32, 96), O.COLS), ((96, 40), O.COLS)])
+def test_tiny_tensors_brute_force_layout(shape, axis):
+    g = np.random.Generator(np.random.PCG64(shape[0] * 1000 + shape[1] + axis))
+    R, C = shape
+    x = (g.standard_normal(shape) * np.exp2(g.integers(-8, 8, size=shape))
+         ).astype(np.float32).astype(BF16)
+    codes, scales = O.quantize(x, axis, O.RNE)
+    got = unpack_nibbles(codes)
+    xv = x.astype(np.float64)
+    if axis == O.ROWS:
+        for r in range(R):
+            for k in range(C // 32):
+                sb, cs = _brute_group(xv[r, 32 * k:32 * k + 32])
+                assert scales[r, k] == sb
+                assert list(got[r, 32 * k:32 * k + 32]) == cs
+    else:
+        for c in range(C):
+            for k in range(R // 32):
+                sb, cs = _brute_group(xv[32 * k:32 * k + 32, c])
+                assert scales[c, k] == sb
+                assert list(got[c, 32 * k:32 * k + 32]) == cs
+
+
+def test_cols_sr_uses_input_row_major_index():
+    # SR along columns keys element (r, c) by r*cols + c: the same random
+    # numbers as the row layout of the transposed grouping.
+    g = np.random.Generator(np.random.PCG64(3))
+    R, C = 64, 32
+    x = g.standard_normal((R, C)).astype(np.float32).astype(BF16)
+    codes, scales = O.quantize(x, O.COLS, O.SR, seed=17)
+    got = unpack_nibbles(codes)
+    xv = x.astype(np.float64)
+    for c in (0, 5, 31):
+        for k in range(R // 32):
+            col = xv[32 * k:32 * k + 32, c]
+            e = int(scales[c, k]) - 127
+            for j in range(32):
+                r = 32 * k + j
+                r16 = O.rand16(17, 0, r * C + c)
+                assert got[c, r] == O.encode(col[j], e, O.SR, r16)
+
+
+# --------------------------------------------------------------------------
+# Double quantization (TetraJet rebuttal, Question 2)
+# --------------------------------------------------------------------------
+
+def test_double_quant_structure():
+    g = np.random.Generator(np.random.PCG64(21))
+    R, C = 96, 64
+    x = (g.standard_normal((R, C)) * 10.0 ** g.uniform(-1, 1, size=C)
+         ).astype(np.float32).astype(BF16)
+    rc, rs, cc, cs = O.double_quantize(x, seed=1)
+    rc2, rs2 = O.quantize(x, O.ROWS, O.RNE)
+    assert np.array_equal(rc, rc2) and np.array_equal(rs, rs2)
+    d = O.dequantize(rc, rs, R, C, out_dtype="f32").astype(np.float64)
+    # column scales follow the scale rule on Q_D(X), not on X
+    for c in range(C):
+        for k in range(R // 32):
+            amax = np.max(np.abs(d[32 * k:32 * k + 32, c]))
+            _check_exponent(float(amax), int(cs[c, k]) - 127)
+    # every column value is a grid neighbour of the exact scaled value
+    dcol = O.dequantize(cc, cs, R, C, O.COLS, out_dtype="f32").astype(np.float64)
+    for c in range(0, C, 7):
+        for r in range(R):
+            e = int(cs[c, r // 32]) - 127
+            a = abs(d[r, c]) * 2.0 ** -e
+            got = abs(dcol[c, r]) * 2.0 ** -e
+            if a >= 6:
+                assert got == 6.0
+            else:
+                lo, step = _lo_step(a)
+                assert got in (lo, lo + step)
+
+
+def test_double_quant_columns_unbiased_over_seeds():
+    g = np.random.Generator(np.random.PCG64(8))
+    R, C = 64, 32
+    x = g.standard_normal((R, C)).astype(np.float32).astype(BF16)
+    S = 400
+    acc = np.zeros((C, R))
+    for s in range(S):
+        rc, rs, cc, cs = O.double_quantize(x, seed=1000 + s)
+        acc += O.dequantize(cc, cs, R, C, O.COLS, out_dtype="f32")
+    d = O.dequantize(rc, rs, R, C, out_dtype="f32").astype(np.float64).T
+    mean = acc / S
+    scale = np.exp2(np.repeat(cs.astype(np.float64) - 127, 32, axis=1))
+    ok = np.abs(d) / scale < 6  # outside saturation Q_S is unbiased
+    step = 2.0 * scale  # the widest step, a loose sigma bound
+    bound = 4 * 0.5 * step / math.sqrt(S) + 1e-12
+    assert np.all(np.abs(mean - d)[ok] <= bound[ok])
+
+
+# --------------------------------------------------------------------------
+# Randomized Hadamard transform
+# --------------------------------------------------------------------------
+
+def test_rht_matches_scipy_hadamard():
+    g = np.random.Generator(np.random.PCG64(4))
+    R, C = 8, 96
+    x = (g.standard_t(3, size=(R, C)) * 0.02).astype(np.float32).astype(BF16)
+    y = O.rht_rotate(x, sign_seed=2)
+    H = scipy.linalg.hadamard(32).astype(np.float64)
+    s = np.array([O.rht_sign(2, c) for c in range(C)], np.float64)
+    xs = (x.astype(np.float64) * s).reshape(R, C // 32, 32)
+    ref = (xs @ H.T / math.sqrt(32)).reshape(R, C)
+    ref32 = ref.astype(np.float32)
+    ulp = np.spacing(np.abs(ref32))
+    assert np.all(np.abs(y - ref32) <= ulp)
+
+
+def test_rht_signs_balanced_and_seeded():
+    s2 = np.array([O.rht_sign(2, c) for c in range(4096)])
+    s3 = np.array([O.rht_sign(3, c) for c in range(4096)])
+    assert set(np.unique(s2)) == {-1, 1}
+    assert abs(s2.sum()) < 4 * 64  # 4 sigma of a fair +-1 sum
+    assert np.mean(s2 == s3) < 0.6
+
+
+def test_rht_orthonormal_properties():
+    g = np.random.Generator(np.random.PCG64(6))
+    x = g.standard_normal((4, 64)).astype(np.float32)
+    y = O.rht_rotate(x, sign_seed=9).astype(np.float64)
+    xg = x.astype(np.float64).reshape(-1, 32)
+    yg = y.reshape(-1, 32)
+    assert np.allclose(np.linalg.norm(yg, axis=1), np.linalg.norm(xg, axis=1),
+                       rtol=1e-6)
+    # the inverse: H is symmetric and H H = 32 I, so x = s .* (H y / sqrt 32)
+    s9 = np.array([O.rht_sign(9, c) for c in range(64)])
+    H = scipy.linalg.hadamard(32).astype(np.float64)
+    rec = (yg @ H / math.sqrt(32)).reshape(4, 64) * s9
+    assert np.allclose(rec, x, atol=1e-6)
+    # one outlier spreads over all 32 entries with magnitude |x| / sqrt(32)
+    z = np.zeros((1, 32), np.float32)
+    z[0, 13] = 8.0
+    yz = O.rht_rotate(z, sign_seed=5)
+    assert np.allclose(np.abs(yz), 8.0 / math.sqrt(32), rtol=1e-7)
+
+
+def test_rht_quantize_is_quantize_of_rotated():
+    g = np.random.Generator(np.random.PCG64(12))
+    x = g.standard_normal((32, 64)).astype(np.float32).astype(BF16)
+    codes, scales, y = O.rht_quantize(x, 2, O.SR, 2)
+    c2, s2 = O.quantize(y, O.ROWS, O.SR, seed=2)
+    assert np.array_equal(codes, c2) and np.array_equal(scales, s2)
+    assert np.array_equal(y, O.rht_rotate(x, 2))
+
+
+# --------------------------------------------------------------------------
+# Oscillation tracker (ALTO explainer: the d_Q / d_w ratio)
+# --------------------------------------------------------------------------
+
+def _one_group_state(w0):
+    """State for a single 1x32 group whose entry 0 is the anchor 3.0: the
+    scale is then 2^-1 and the bins below 1 are 0.25 apart."""
+    w = np.zeros((1, 32), np.float32)
+    w[0, 0] = 3.0
+    w[0, 1] = w0
+    return w, w.copy(), np.zeros_like(w), np.zeros_like(w)
+
+
+def _run(traj, threshold=4.0):
+    w, ws, dw, dq = _one_group_state(traj[0])
+    flagged = 0
+    for t, val in enumerate(traj[1:], start=1):
+        w[0, 1] = val
+        flagged = O.osc_step(w, ws, dw, dq, window_end=(t == len(traj) - 1),
+                             threshold=threshold)
+    return w, ws, dw, dq, flagged
+
+
+def test_osc_worked_example_from_the_page():
+    ex = load("osc_worked_example.json")
+    assert ex["bin_spacing"] == 0.25
+    P = ex["window"]
+    # oscillating: 6 edge crossings at the 0.625 edge (bins 0.5 / 0.75),
+    # then small moves that cross nothing, total travel 0.02
+    traj = [0.624]
+    for _ in range(6):
+        traj.append(0.626 if traj[-1] < 0.625 else 0.624)
+    for _ in range(4):
+        traj += [traj[-1] + 0.001, traj[-1]]
+    traj += [traj[-1]] * (P + 1 - len(traj))
+    w, ws, dw, dq, flagged = _run(np.array(traj, np.float32))
+    case = ex["cases"][0]
+    assert flagged == 1 and case["flagged"]
+    assert w[0, 1] == np.float32(0.5)  # snapped to the centre of its bin
+    # an oscillating weight whose last move crosses the edge snaps to the
+    # bin it sits in now, not the one it came from
+    traj = [0.624 if t % 2 == 0 else 0.626 for t in range(P + 1)]
+    w, ws, dw, dq, flagged = _run(np.array(traj, np.float32))
+    assert flagged == 1 and traj[-1] == 0.624 and traj[-2] == 0.626
+    assert w[0, 1] == np.float32(0.5)
+    # healthy: drift 0.30 across one edge
+    traj = np.linspace(0.40, 0.70, P + 1).astype(np.float32)
+    w, ws, dw, dq, flagged = _run(traj)
+    assert flagged == 0 and not ex["cases"][1]["flagged"]
+    assert w[0, 1] == np.float32(0.70)
+
+
+def test_osc_accumulators_before_window_end():
+    w, ws, dw, dq = _one_group_state(0.624)
+    w[0, 1] = 0.626
+    assert O.osc_step(w, ws, dw, dq) == 0
+    assert dw[0, 1] == np.float32(np.float32(0.626) - np.float32(0.624))
+    assert dq[0, 1] == 0.25  # one crossing = one bin spacing
+    assert ws[0, 1] == w[0, 1]
+    w[0, 1] = 0.6235  # a move down across the edge adds its length too
+    assert O.osc_step(w, ws, dw, dq) == 0
+    f = np.float32
+    want = f(f(f(0.626) - f(0.624)) + f(f(0.626) - f(0.6235)))
+    assert dw[0, 1] == want and dq[0, 1] == 0.5
+    ex = load("osc_worked_example.json")
+    # direct ratio check with the page's numbers on a prepared state
+    for case in ex["cases"]:
+        w, ws, dw, dq = _one_group_state(0.6)
+        dw[0, 1], dq[0, 1] = case["d_w"], case["d_q"]
+        assert O.osc_step(w, ws, dw, dq, window_end=True,
+                          threshold=ex["threshold"]) == int(case["flagged"])
+        assert dw[0, 1] == 0 and dq[0, 1] == 0
+
+
+def test_osc_snap_invariants_on_workload():
+    from mxfp4_block_quantization_quantizer_b200 import workloads as W
+    w = W.osc_w(seed=3, rows=16, cols=256)
+    ws, dw, dq = w.copy(), np.zeros_like(w), np.zeros_like(w)
+    for t in range(200):
+        O.osc_synthetic_update(w, 3, t)
+        before = w.copy()
+        n = O.osc_step(w, ws, dw, dq, window_end=(t == 199))
+    assert n > 0
+    moved = w != before
+    assert moved.sum() <= n
+    c0, s0 = O.quantize(before)
+    c1, s1 = O.quantize(w)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)  # Q(snap w) = Q(w)
+    dqv = O.dequantize(c1, s1, *w.shape, out_dtype="f32")
+    assert np.array_equal(w[moved], dqv[moved])  # snapped to the bin value
+    w2, ws2, dw2, dq2 = w.copy(), w.copy(), np.zeros_like(w), np.zeros_like(w)
+    O.osc_step(w2, ws2, dw2, dq2, window_end=True)
+    assert np.array_equal(w2, w)  # idempotent
+    assert not dw.any() and not dq.any() and np.array_equal(ws, w)
+
+
+def test_osc_synthetic_update_magnitude_and_signs():
+    g = np.random.Generator(np.random.PCG64(1))
+    w = g.normal(0, 0.02, size=(64, 64)).astype(np.float32)
+    w0 = w.copy()
+    O.osc_synthetic_update(w, 3, 7, 1e-4)
+    mag = (np.float32(1e-4) * np.abs(w0)).astype(np.float32)
+    plus = (w0 + mag).astype(np.float32)
+    minus = (w0 - mag).astype(np.float32)
+    assert np.all((w == plus) | (w == minus))
+    frac_plus = np.mean(w == plus)
+    assert 0.45 < frac_plus < 0.55
+    w1 = w0.copy()
+    O.osc_synthetic_update(w1, 3, 7, 1e-4)
+    assert np.array_equal(w1, w)
+    O.osc_synthetic_update(w1, 3, 8, 1e-4)
+    assert not np.array_equal(w1, w)
