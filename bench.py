@@ -1,0 +1,409 @@
+"""Benchmark of the MXFP4 block quantizer hot path on B200.
+
+One step = one pass of the whole hot path over the sweep workload
+(8192 x 28672 bf16, N(0,1) with 0.1% outliers x100, seed 5 + rank):
+  rows RNE quantize, columns SR quantize, fused double quantization,
+  dequantize of the row layout, Hadamard-rotate + rows SR quantize,
+plus one oscillation-tracker step (with its synthetic update) on the
+tracker workload (4096 x 4096 fp32 master weight).
+Metric: GB/s of algorithmic bytes in+out (whole job), with % of the measured
+HBM peak per kernel. Inputs are larger than L2 (470 MB and 268 MB against a
+126 MB L2), so no flush is needed between steps.
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (one 32-row band per op); it is the reported baseline.
+Multi-GPU (torchrun): every rank runs the same step on its own data
+(weak scaling, no collective on the data path); the timed region is the max
+over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+SWEEP = (8192, 28672)
+OSC = (4096, 4096)
+SEED = 5
+
+# Algorithmic bytes per element (in + out), per op.
+BYTES_PER_ELEM = {
+    "quant_rows_rne": 2 + 0.5 + 1 / 32,
+    "quant_cols_sr": 2 + 0.5 + 1 / 32,
+    "double_quant": 2 + 2 * (0.5 + 1 / 32),
+    "dequant_rows": 0.5 + 1 / 32 + 2,
+    "rht_quant_sr": 2 + 0.5 + 1 / 32,
+    "osc_update": 8,
+    "osc_step": 28,
+}
+OP_ELEMS = {k: SWEEP[0] * SWEEP[1] for k in BYTES_PER_ELEM}
+OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
+
+
+def alg_bytes(op):
+    return BYTES_PER_ELEM[op] * OP_ELEMS[op]
+
+
+STEP_BYTES = sum(alg_bytes(op) for op in BYTES_PER_ELEM)
+STEP_ELEMS = sum(OP_ELEMS.values())
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def config_block(args, world):
+    return {"workload": "sweep 8192x28672 bf16 N(0,1)+0.1% x100 outliers "
+                        "[rows RNE, cols SR, double quant, dequant rows, "
+                        "RHT+rows SR] + oscillation tracker step on 4096x4096 "
+                        "fp32 master weight",
+            "shape": list(SWEEP), "osc_shape": list(OSC), "seed": SEED,
+            "sr_seed": SEED, "rht_sign_seed": 2, "osc_threshold": 4.0,
+            "l2": "inputs larger than L2 (470 MB, 268 MB); no flush",
+            "parallelism": "replicas x%d (weak, no collective)" % world}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def cpu_sample_step(x_band, w_band, osc_state, row0):
+    """One step of the oracle on a sample: a 32-row band of the sweep for
+    each op, and a 16-row band of the tracker workload. Returns bytes."""
+    import oracle as O
+    C = x_band.shape[1]
+    n = x_band.size
+    O.quantize(x_band, O.ROWS, O.RNE, 0, row0=row0)
+    O.quantize(x_band, O.COLS, O.SR, SEED, row0=row0)
+    O.double_quantize(x_band, SEED, row0=row0)
+    c, s = O.quantize(x_band, O.ROWS, O.RNE, 0, row0=row0)
+    O.dequantize(c, s, 32, C)
+    O.rht_quantize(x_band, 2, O.SR, SEED, row0=row0)
+    w, ws, dw, dq = osc_state
+    O.osc_synthetic_update(w, SEED, 0, row0=0)
+    O.osc_step(w, ws, dw, dq)
+    nb = 0.0
+    for op in ("quant_rows_rne", "quant_cols_sr", "double_quant", "dequant_rows",
+               "rht_quant_sr"):
+        nb += BYTES_PER_ELEM[op] * n
+    nb += (BYTES_PER_ELEM["osc_update"] + BYTES_PER_ELEM["osc_step"]) * w.size
+    return nb, n * 5 + w.size * 2
+
+
+def cpu_baseline_sample(x_np, w_np, max_seconds=20.0):
+    band = np.ascontiguousarray(x_np[:32])
+    wb = np.ascontiguousarray(w_np[:16])
+    state = (wb.copy(), wb.copy(), np.zeros_like(wb), np.zeros_like(wb))
+    t0 = time.perf_counter()
+    total_b, total_e, reps = 0.0, 0, 0
+    while True:
+        b, e = cpu_sample_step(band, wb, state, 0)
+        total_b += b
+        total_e += e
+        reps += 1
+        if time.perf_counter() - t0 > max_seconds or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": total_b / dt / 1e9, "unit": "GB/s", "cores": 1,
+            "kind": "oracle",
+            "sample": "%d reps of one 32x28672 band of the sweep per op (rows RNE, "
+                      "cols SR, double quant, dequant, RHT+SR) and a 16x4096 band "
+                      "of the tracker (update + step); single thread, %.1f s"
+                      % (reps, dt),
+            "gelem_s": total_e / dt / 1e9}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from mxfp4_block_quantization_quantizer_b200 import workloads as W
+    x = W.normal_bf16(64, SWEEP[1], SEED, 0.001, 100.0)
+    w = W.osc_w(seed=3, rows=16, cols=OSC[1])
+    band = np.ascontiguousarray(x[:32])
+    state = (w.copy(), w.copy(), np.zeros_like(w), np.zeros_like(w))
+    for _ in range(args.warmup):
+        cpu_sample_step(band, w, state, 0)
+    t0 = time.perf_counter()
+    nb = ne = 0
+    for _ in range(args.steps):
+        b, e = cpu_sample_step(band, w, state, 0)
+        nb += b
+        ne += e
+    dt = time.perf_counter() - t0
+    value = nb / dt / 1e9
+    line = {"impl": "reference", "metric": "MXFP4 quantize GB/s (bytes in+out)",
+            "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": config_block(args, 1),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": "each step: one 32x28672 band of the sweep "
+                                       "per op and a 16x4096 tracker band"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gelem_s": ne / dt / 1e9}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for line in out.strip().splitlines():
+            p = [s.strip() for s in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mxfp4_block_quantization_quantizer_b200 as m
+    from mxfp4_block_quantization_quantizer_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    m.lib()
+
+    # inputs (seeded numpy), uploaded once
+    x_np = W.sweep(seed=SEED + rank)
+    w_np = W.osc_w(seed=3 + rank)
+    x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
+    w0 = torch.from_numpy(w_np).to(dev)
+    R, C = SWEEP
+    u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)  # noqa: E731
+    rows_out = (u8(R, C // 2), u8(R, C // 32))
+    cols_out = (u8(C, R // 2), u8(C, R // 32))
+    dq_out = (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32))
+    rht_out = (u8(R, C // 2), u8(R, C // 32), None)
+    y = torch.empty(R, C, dtype=torch.bfloat16, device=dev)
+    w = w0.clone()
+    ws, dwt, dqt = w.clone(), torch.zeros_like(w), torch.zeros_like(w)
+    nflag = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    ops = list(BYTES_PER_ELEM)
+    stream = torch.cuda.current_stream(dev)
+    ev = {op: [] for op in ops}
+    step_no = [0]
+
+    def step(record):
+        t = step_no[0]
+        step_no[0] += 1
+        pairs = []
+
+        def timed(op, fn):
+            if record:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                pairs.append((op, a, b))
+            else:
+                fn()
+
+        timed("quant_rows_rne", lambda: m.quantize(x, m.ROWS, m.RNE, 0, out=rows_out))
+        timed("quant_cols_sr", lambda: m.quantize(x, m.COLS, m.SR, SEED, out=cols_out))
+        timed("double_quant", lambda: m.double_quantize(x, SEED, out=dq_out))
+        timed("dequant_rows", lambda: m.dequantize(rows_out[0], rows_out[1], R, C, out=y))
+        timed("rht_quant_sr", lambda: m.rht_quantize(x, 2, m.SR, SEED, out=rht_out))
+        timed("osc_update", lambda: m.osc_synthetic_update(w, 3, t % 200))
+        timed("osc_step", lambda: m.osc_step(w, ws, dwt, dqt, window_end=(t % 200 == 199),
+                                             n_flagged=nflag))
+        return pairs
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler.start()
+    time.sleep(0.3)
+    all_pairs = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        all_pairs.extend(step(True))
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    for op, a, b in all_pairs:
+        ev[op].append(a.elapsed_time(b))
+    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+
+    # end to end: pinned host input -> device -> kernels -> host results
+    x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    w_host = torch.from_numpy(w_np).pin_memory()
+    outs = [rows_out[0], rows_out[1], cols_out[0], cols_out[1], *dq_out, y,
+            rht_out[0], rht_out[1], w, nflag]
+    host_outs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = x_host.numel() * 2 + w_host.numel() * 4
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    for _ in range(1):
+        x.copy_(x_host, non_blocking=True)
+        w.copy_(w_host, non_blocking=True)
+        step(False)
+        for h, o in zip(host_outs, outs):
+            h.copy_(o, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        w.copy_(w_host, non_blocking=True)
+        step(False)
+        for h, o in zip(host_outs, outs):
+            h.copy_(o, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_end)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(te.item())
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        per_op = {}
+        for op in ops:
+            d = statistics.mean(ev[op]) * 1e-3
+            ach = alg_bytes(op) / d / 1e9
+            per_op[op] = {"us": d * 1e6, "GB_s": ach, "frac": ach / peak,
+                          "bytes": alg_bytes(op)}
+        dom = max(per_op, key=lambda k: per_op[k]["us"])
+        step_s = elapsed_ms * 1e-3 / args.steps
+        value = world * STEP_BYTES / step_s / 1e9
+        traffic = None
+        prof = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(prof):
+            try:
+                traffic = json.load(open(prof)).get(dom)
+            except Exception:
+                traffic = None
+        line = {
+            "metric": "MXFP4 quantize GB/s (bytes in+out)",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": config_block(args, world),
+            "gelem_s": world * STEP_ELEMS / step_s / 1e9,
+            "hbm_frac": value / world / peak,
+            "roofline": {"bound": "hbm", "kernel": dom,
+                         "achieved": per_op[dom]["GB_s"], "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": per_op[dom]["frac"], "traffic": traffic},
+            "ops": per_op,
+            "e2e": {"value": world * STEP_BYTES * args.e2e_steps / (e2e_ms * 1e-3) / 1e9,
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(ops) * args.steps,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline_sample(x_np, w_np)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+"""ctypes binding of libmxfp4 (include/mxfp4.h).
+
+Argument marshalling only: tensors become device pointers and sizes, the
+current torch stream becomes the cudaStream_t, output buffers are allocated
+with torch. Every step of the computation runs in the library's kernels.
+There is no fallback: if the library is missing, or a tensor is not on a CUDA
+device, the call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmxfp4.so")
+
+F32, BF16 = 0, 1
+ROWS, COLS = 0, 1
+RNE, SR = 0, 1
+
+# Every symbol include/mxfp4.h declares.
+SYMBOLS = ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_double_quantize",
+           "mxfp4_rht_quantize", "mxfp4_osc_step",
+           "mxfp4_osc_synthetic_update", "mxfp4_status_string")
+
+
+class Mxfp4Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmxfp4 (ctypes.CDLL). Raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libmxfp4.so is not built (expected at %s); run "
+                "__graft_entry__.build() or python -m "
+                "mxfp4_block_quantization_quantizer_b200.build" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, u64, u32, i32 = (ctypes.c_void_p, ctypes.c_int64,
+                                  ctypes.c_uint64, ctypes.c_uint32,
+                                  ctypes.c_int)
+        sig = {
+            "mxfp4_quantize": [vp, i32, i64, i64, i32, i32, u64, vp, vp, vp],
+            "mxfp4_dequantize": [vp, vp, i64, i64, i32, vp, i32, vp],
+            "mxfp4_double_quantize": [vp, i32, i64, i64, u64, vp, vp, vp, vp,
+                                      vp],
+            "mxfp4_rht_quantize": [vp, i32, i64, i64, u64, i32, u64, vp, vp,
+                                   vp, vp],
+            "mxfp4_osc_step": [vp, vp, vp, vp, i64, i64, i32, ctypes.c_float,
+                               vp, vp],
+            "mxfp4_osc_synthetic_update": [vp, i64, i64, u64, u32,
+                                           ctypes.c_float, vp],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes, f.restype = args, i32
+        L.mxfp4_status_string.argtypes = [i32]
+        L.mxfp4_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().mxfp4_status_string(status).decode()
+
+
+def _check(status, what):
+    if status != 0:
+        raise Mxfp4Error(status, what)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError("expected a bfloat16 or float32 tensor, got %s" % t.dtype)
+
+
+def _cuda2d(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dim() != 2 or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous 2-D tensor" % name)
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _empty_u8(shape, device):
+    return torch.empty(shape, dtype=torch.uint8, device=device)
+
+
+def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None):
+    """mxfp4_quantize: returns (codes, scales) in the layout of `axis`:
+    ROWS -> codes [R, C/2], scales [R, C/32]; COLS -> codes [C, R/2],
+    scales [C, R/32]."""
+    _cuda2d(x, "x")
+    R, C = x.shape
+    if out is None:
+        shape_c = (R, C // 2) if axis == ROWS else (C, R // 2)
+        shape_s = (R, C // 32) if axis == ROWS else (C, R // 32)
+        out = (_empty_u8(shape_c, x.device), _empty_u8(shape_s, x.device))
+    codes, scales = out
+    _check(lib().mxfp4_quantize(_ptr(x), _dtype_code(x), R, C, axis, rounding,
+                                seed, _ptr(codes), _ptr(scales),
+                                _stream(x.device, stream)), "mxfp4_quantize")
+    return codes, scales
+
+
+def dequantize(codes, scales, rows, cols, axis=ROWS, out_dtype=torch.bfloat16,
+               out=None, stream=None):
+    """mxfp4_dequantize: values [rows, cols] (ROWS) or [cols, rows] (COLS)."""
+    if not codes.is_cuda or not scales.is_cuda:
+        raise TypeError("codes and scales must be CUDA tensors")
+    if out is None:
+        shape = (rows, cols) if axis == ROWS else (cols, rows)
+        out = torch.empty(shape, dtype=out_dtype, device=codes.device)
+    _check(lib().mxfp4_dequantize(_ptr(codes), _ptr(scales), rows, cols, axis,
+                                  _ptr(out), _dtype_code(out),
+                                  _stream(codes.device, stream)),
+           "mxfp4_dequantize")
+    return out
+
+
+def double_quantize(x, seed=0, out=None, stream=None):
+    """mxfp4_double_quantize: (row_codes, row_scales, col_codes, col_scales)."""
+    _cuda2d(x, "x")
+    R, C = x.shape
+    if out is None:
+        d = x.device
+        out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d),
+               _empty_u8((C, R // 2), d), _empty_u8((C, R // 32), d))
+    rc, rs, cc, cs = out
+    _check(lib().mxfp4_double_quantize(_ptr(x), _dtype_code(x), R, C, seed,
+                                       _ptr(rc), _ptr(rs), _ptr(cc), _ptr(cs),
+                                       _stream(x.device, stream)),
+           "mxfp4_double_quantize")
+    return out
+
+
+def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
+                 out=None, stream=None):
+    """mxfp4_rht_quantize: (codes, scales, rotated or None), ROWS layout."""
+    _cuda2d(x, "x")
+    R, C = x.shape
+    if out is None:
+        d = x.device
+        rot = torch.empty((R, C), dtype=torch.float32, device=d) if want_rotated else None
+        out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d), rot)
+    codes, scales, rot = out
+    _check(lib().mxfp4_rht_quantize(_ptr(x), _dtype_code(x), R, C, sign_seed,
+                                    rounding, sr_seed, _ptr(codes),
+                                    _ptr(scales), _ptr(rot),
+                                    _stream(x.device, stream)),
+           "mxfp4_rht_quantize")
+    return out
+
+
+def osc_step(w, w_snap, d_w, d_q, window_end=False, threshold=4.0,
+             n_flagged=None, stream=None):
+    """mxfp4_osc_step on fp32 tensors, in place. n_flagged: optional int64
+    CUDA tensor of one element to which the flag count is added."""
+    for name, t in (("w", w), ("w_snap", w_snap), ("d_w", d_w), ("d_q", d_q)):
+        _cuda2d(t, name)
+        if t.dtype != torch.float32 or t.shape != w.shape:
+            raise TypeError("%s must be float32 with the shape of w" % name)
+    if n_flagged is not None and (not n_flagged.is_cuda
+                                  or n_flagged.dtype not in (torch.int64, torch.uint64)):
+        raise TypeError("n_flagged must be a CUDA int64 tensor")
+    R, C = w.shape
+    _check(lib().mxfp4_osc_step(_ptr(w), _ptr(w_snap), _ptr(d_w), _ptr(d_q),
+                                R, C, int(bool(window_end)), threshold,
+                                _ptr(n_flagged), _stream(w.device, stream)),
+           "mxfp4_osc_step")
+
+
+def osc_synthetic_update(w, seed, step, rel_step=1e-4, stream=None):
+    """mxfp4_osc_synthetic_update on an fp32 CUDA tensor, in place."""
+    _cuda2d(w, "w")
+    if w.dtype != torch.float32:
+        raise TypeError("w must be float32")
+    R, C = w.shape
+    _check(lib().mxfp4_osc_synthetic_update(_ptr(w), R, C, seed, step,
+                                            rel_step, _stream(w.device, stream)),
+           "mxfp4_osc_synthetic_update")
+
+
+# The C names, for callers that prefer them.
+mxfp4_quantize = quantize
+mxfp4_dequantize = dequantize
+mxfp4_double_quantize = double_quantize
+mxfp4_rht_quantize = rht_quantize
+mxfp4_osc_step = osc_step
+mxfp4_osc_synthetic_update = osc_synthetic_update
+mxfp4_status_string = status_string

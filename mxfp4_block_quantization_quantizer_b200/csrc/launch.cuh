@@ -1,0 +1,48 @@
+// Kernel launchers of libmxfp4 (internal; the C ABI in capi.cu validates
+// arguments and calls these). Each returns the cudaError_t of its launch.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxfp4 {
+
+// Grid size for a grid-stride kernel: resident blocks per SM x SMs of the
+// current device, capped by the amount of work.
+int persistent_grid(const void* kernel, int threads, size_t smem,
+                    int64_t work_blocks);
+
+cudaError_t launch_quant_rows(const void* x, bool bf16, int64_t rows,
+                              int64_t cols, bool sr, uint64_t seed,
+                              uint8_t* codes, uint8_t* scales, cudaStream_t s);
+
+cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
+                              int64_t cols, bool sr, uint64_t seed,
+                              uint8_t* codes, uint8_t* scales, cudaStream_t s);
+
+// Flat decode of n_groups groups (rows of the output are contiguous runs of
+// whole groups in both layouts).
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
+                           int64_t n_groups, void* y, bool bf16_out,
+                           cudaStream_t s);
+
+cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
+                                int64_t cols, uint64_t seed,
+                                uint8_t* row_codes, uint8_t* row_scales,
+                                uint8_t* col_codes, uint8_t* col_scales,
+                                cudaStream_t s);
+
+cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
+                             int64_t cols, uint64_t sign_seed, bool sr,
+                             uint64_t sr_seed, uint8_t* codes,
+                             uint8_t* scales, float* rotated, cudaStream_t s);
+
+cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
+                            int64_t rows, int64_t cols, bool window_end,
+                            float threshold, unsigned long long* n_flagged,
+                            cudaStream_t s);
+
+cudaError_t launch_osc_update(float* w, int64_t n, uint64_t seed,
+                              uint32_t step, float rel_step, cudaStream_t s);
+
+}  // namespace mxfp4

@@ -1,0 +1,235 @@
+// Device-side building blocks of the MXFP4 block quantizer (sm_100a).
+//
+// Format (ALTO explainer, "ALTO MXFP4 training — Weight de-oscillation",
+// Jargon: MXFP4, E2M1, Bin; "Unveiling the Potential of Quantization with
+// MXFP4", abstract: power-of-two block scaling):
+//   - one E8M0 scale byte per 32-element group, byte = e + 127 with
+//     e = floor(log2(absmax)) - 2 clamped to [-127, 127]; 0 for a zero group,
+//     0xFF (codes 0) for a group holding Inf/NaN;
+//   - 4-bit E2M1 codes: sign in bit 3, magnitude index m of
+//     {0, .5, 1, 1.5, 2, 3, 4, 6} in bits 0..2; the even element of a pair
+//     in the low nibble.
+//
+// All arithmetic that decides a code is exact: scaling multiplies by a power
+// of two, rounding to nearest-even uses the hardware E2M1 conversion, and
+// stochastic rounding compares integer bit fields. The library is built
+// without fast-math and with FMA contraction off, so subnormal inputs are
+// not flushed.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mxfp4 {
+
+constexpr int kGroup = 32;
+
+// ---------------------------------------------------------------------------
+// Counter-based random numbers. mix() is the MurmurHash3 32-bit finalizer.
+// K(seed, s) = mix(lo32(seed) ^ mix(hi32(seed) + s * 0x9E3779B9));
+// pair p: h = mix(mix(K ^ hi32(p)) + lo32(p)); the element with even
+// row-major index i = 2p takes h & 0xFFFF, the odd one takes h >> 16.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint32_t mix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85EBCA6Bu;
+  h ^= h >> 13;
+  h *= 0xC2B2AE35u;
+  h ^= h >> 16;
+  return h;
+}
+
+__host__ __device__ __forceinline__ uint32_t stream_key(uint64_t seed,
+                                                        uint32_t stream) {
+  return mix32(static_cast<uint32_t>(seed) ^
+               mix32(static_cast<uint32_t>(seed >> 32) + stream * 0x9E3779B9u));
+}
+
+// Per-key constants handed to kernels: the key and mix(key ^ 0), the inner
+// hash of every counter below 2^32.
+struct RngKey {
+  uint32_t k;
+  uint32_t k0;
+};
+
+__host__ __forceinline__ RngKey make_key(uint64_t seed, uint32_t stream) {
+  RngKey r;
+  r.k = stream_key(seed, stream);
+  r.k0 = mix32(r.k ^ 0u);
+  return r;
+}
+
+// Inner hash for counters whose high word is `hi` (0 for every tensor below
+// 2^33 elements).
+__device__ __forceinline__ uint32_t inner_key(RngKey key, uint32_t hi) {
+  return hi == 0 ? key.k0 : mix32(key.k ^ hi);
+}
+
+// ---------------------------------------------------------------------------
+// Scale
+// ---------------------------------------------------------------------------
+
+// E8M0 byte from the fp32 bit pattern of |absmax| (bf16 inputs are widened
+// first: same exponent field). With E the biased exponent field,
+// floor(log2 absmax) = E - 127 for normal values, so byte = E - 2, clamped at
+// 0, which also covers zero and subnormal maxima (e clamps to -127).
+__device__ __forceinline__ uint32_t scale_byte(uint32_t abs_bits) {
+  uint32_t E = abs_bits >> 23;
+  return abs_bits >= 0x7F800000u ? 0xFFu : (E > 2u ? E - 2u : 0u);
+}
+
+// 2^-e as fp32 for byte sb = e + 127 <= 252: biased exponent 254 - sb.
+__device__ __forceinline__ float inv_scale(uint32_t sb) {
+  uint32_t b = sb > 252u ? 252u : sb;
+  return __uint_as_float((254u - b) << 23);
+}
+
+// 2^e as fp32 for byte sb (sb = 0 gives the subnormal 2^-127).
+__device__ __forceinline__ float scale_value(uint32_t sb) {
+  return __uint_as_float(sb ? (sb << 23) : 0x00400000u);
+}
+
+// ---------------------------------------------------------------------------
+// E2M1 rounding
+// ---------------------------------------------------------------------------
+
+// Round 8 scaled values to nearest-even E2M1 with saturation to +-6 (the
+// hardware conversion); element j lands in nibble j of the result.
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]),
+        "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// Stochastic E2M1 code of one scaled value v (exact) with its 16-bit random
+// number r: lo = largest grid value <= |v|, hi = the next one; the result is
+// hi iff (r + 0.5) * 2^-16 < (|v| - lo) / (hi - lo); |v| >= 6 gives 6.
+//
+// In every binade [2^k, 2^k+1) with k >= 0 the grid keeps one mantissa bit,
+// so the low 22 mantissa bits of |v| are frac * 2^22 exactly. Below 1 the
+// grid step is 0.5 throughout; 1 + |v| (rounded up) maps [0, 1) onto [1, 2)
+// with the same step and rounding up keeps the comparison exact, because the
+// threshold lies on the 2^-18 grid. The test is then frac * 2^22 > 64r + 32.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
+  float a = fabsf(v);
+  bool small = a < 1.0f;
+  float y = __fadd_ru(a, small ? 1.0f : 0.0f);
+  uint32_t yb = __float_as_uint(y);
+  int m = static_cast<int>(yb >> 22) - (small ? 254 : 252);
+  uint32_t rem = yb & 0x3FFFFFu;
+  m += rem > ((r << 6) | 32u) ? 1 : 0;
+  m = m > 7 ? 7 : m;
+  return (__float_as_uint(v) >> 28 & 8u) | static_cast<uint32_t>(m);
+}
+
+// Stochastic codes of 8 values whose random numbers come in 4 hashes (pair
+// k of the 8 values uses h[k]: low half for the even element).
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float* v,
+                                              const uint32_t* h) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t c0 = e2m1_sr(v[2 * k], h[k] & 0xFFFFu);
+    uint32_t c1 = e2m1_sr(v[2 * k + 1], h[k] >> 16);
+    out |= (c0 | (c1 << 4)) << (8 * k);
+  }
+  return out;
+}
+
+// Nearest-even E2M1 value of a scaled v (exact, no codes): with K the power
+// of two 2^(max(E,0) + 22), E the binade of |v|, the fp32 sum |v| + K has an
+// ulp equal to the E2M1 grid step at |v| (2^(E-1), or 0.5 below 1), so the
+// round-to-nearest-even addition lands on the nearest grid value with ties to
+// the even one and the subtraction is exact; values from 6 up saturate to 6.
+// The sign of v is kept (a negative value that rounds to 0 gives -0).
+__device__ __forceinline__ float e2m1_rn_value(float v) {
+  const uint32_t vb = __float_as_uint(v);
+  const uint32_t ab = vb & 0x7FFFFFFFu;
+  const uint32_t eb = ab & 0x7F800000u;
+  const float K = __uint_as_float((eb > 0x3F800000u ? eb : 0x3F800000u) + 0x0B000000u);
+  const float a = __uint_as_float(ab);
+  float q = __fsub_rn(__fadd_rn(a, K), K);
+  q = fminf(q, 6.0f);
+  return __uint_as_float(__float_as_uint(q) | (vb & 0x80000000u));
+}
+
+// ---------------------------------------------------------------------------
+// Decode
+// ---------------------------------------------------------------------------
+
+// The 8 codes of one 32-bit word as fp32 values G[m] with their signs
+// (hardware E2M1 -> f16 conversion, exact), element j from nibble j.
+// Decode only words that were loaded from memory (global or shared): feeding
+// the result of e2m1x8_rn straight into this conversion in registers produced
+// wrong values in one kernel shape on this toolchain, so no kernel does that.
+__device__ __forceinline__ void e2m1x8_decode(uint32_t w, float* out) {
+  uint32_t h0, h1, h2, h3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(w));
+  const uint32_t h[4] = {h0, h1, h2, h3};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float lo, hi;
+    asm("{\n\t.reg .f16 l, u;\n\t"
+        "mov.b32 {l, u}, %2;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, u;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(h[k]));
+    out[2 * k] = lo;
+    out[2 * k + 1] = hi;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Packed bf16 helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) {
+  return __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w) {
+  return __uint_as_float(w & 0xFFFF0000u);
+}
+
+// Per-half unsigned max of two packed 16-bit pairs.
+__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Two exact fp32 values -> packed bf16x2 (low element in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// 16-byte load of read-once data: no L1 allocation.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+constexpr uint32_t kNaNbf16x2 = 0x7FC07FC0u;
+constexpr uint32_t kNaNf32 = 0x7FC00000u;
+
+}  // namespace mxfp4

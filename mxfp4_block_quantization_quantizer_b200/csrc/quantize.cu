@@ -1,0 +1,592 @@
+// MXFP4 block quantize (1x32 row groups and 32x1 column groups) and
+// dequantize kernels for sm_100a.
+//
+// Sources: "ALTO MXFP4 training — Weight de-oscillation — What does it
+// mean?", Jargon (MXFP4, E2M1, Bin, Stochastic rounding);
+// "Oscillation-Reduced MXFP4 Training for Vision Transformers", rebuttal,
+// Question 2 (Q_D along 1x32 groups for the forward GEMM, 32x1 groups for the
+// backward GEMM).
+//
+// Row groups: a [rows, cols] tensor with cols % 32 == 0 is a flat array of
+// rows*cols/32 groups, so the row kernel is a grid-stride loop over groups.
+// Four threads share a group (8 elements, one 16-byte load per thread for
+// bf16), the absmax is reduced with two quad shuffles, and each thread
+// writes the 4 code bytes of its 8 elements; a warp covers 8 consecutive
+// groups per load, so loads and code stores are fully coalesced. U groups
+// per quad are loaded before any arithmetic to keep enough bytes in flight.
+//
+// Column groups: a CTA stages a 128-row tile (128 bf16 or 64 fp32 columns)
+// in shared memory, then each thread reduces two adjacent columns over 32
+// rows (one 32-bit shared word per row; a warp reads 32 consecutive words of
+// one row: no bank conflicts) and writes 16 code bytes per column. The four
+// row groups of a column in the tile write one contiguous 64-byte run, so
+// every DRAM sector of the transposed output is written whole.
+#include "launch.cuh"
+#include "mxfp4_device.cuh"
+
+namespace mxfp4 {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Row groups
+// ---------------------------------------------------------------------------
+
+constexpr int kRowThreads = 256;
+
+template <bool BF16, bool SR, int U>
+__global__ void __launch_bounds__(kRowThreads)
+    k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey key,
+                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const int64_t warp = (int64_t(blockIdx.x) * kRowThreads + threadIdx.x) >> 5;
+  const int64_t chunk = (int64_t(gridDim.x) * kRowThreads) >> 2;  // quads
+  const int64_t my = warp * 8 + (lane >> 2);
+
+  for (int64_t base = 0; base < n_groups; base += chunk * U) {
+    float v[U][8];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * chunk + my;
+      ok[u] = g < n_groups;
+      if (BF16) {
+        uint4 w = ok[u] ? ld_stream(static_cast<const uint16_t*>(x) + g * 32 +
+                                    sub * 8)
+                        : make_uint4(0, 0, 0, 0);
+        v[u][0] = bf16_lo(w.x), v[u][1] = bf16_hi(w.x);
+        v[u][2] = bf16_lo(w.y), v[u][3] = bf16_hi(w.y);
+        v[u][4] = bf16_lo(w.z), v[u][5] = bf16_hi(w.z);
+        v[u][6] = bf16_lo(w.w), v[u][7] = bf16_hi(w.w);
+      } else {
+        const float* p = static_cast<const float*>(x) + g * 32 + sub * 8;
+        uint4 a = ok[u] ? ld_stream(p) : make_uint4(0, 0, 0, 0);
+        uint4 b = ok[u] ? ld_stream(p + 4) : make_uint4(0, 0, 0, 0);
+        v[u][0] = __uint_as_float(a.x), v[u][1] = __uint_as_float(a.y);
+        v[u][2] = __uint_as_float(a.z), v[u][3] = __uint_as_float(a.w);
+        v[u][4] = __uint_as_float(b.x), v[u][5] = __uint_as_float(b.y);
+        v[u][6] = __uint_as_float(b.z), v[u][7] = __uint_as_float(b.w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * chunk + my;
+      uint32_t amax = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        amax = max(amax, __float_as_uint(v[u][j]) & 0x7FFFFFFFu);
+      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      const uint32_t sb = scale_byte(amax);
+      const float mul = inv_scale(sb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[u][j] *= mul;
+      uint32_t word;
+      if (SR) {
+        const uint64_t p0 = uint64_t(g) * 16 + uint64_t(sub) * 4;
+        const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) h[k] = mix32(kh + uint32_t(p0) + k);
+        word = e2m1x8_sr(v[u], h);
+      } else {
+        word = e2m1x8_rn(v[u]);
+      }
+      if (sb == 0xFFu) word = 0;
+      if (ok[u]) {
+        reinterpret_cast<uint32_t*>(codes)[g * 4 + sub] = word;
+        if (sub == 0) scales[g] = static_cast<uint8_t>(sb);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Column groups
+// ---------------------------------------------------------------------------
+
+constexpr int kTileRows = 128;
+
+template <bool BF16>
+struct ColTile {
+  static constexpr int kCols = BF16 ? 128 : 64;           // tile columns
+  static constexpr int kThreads = (kCols / 2) * (kTileRows / 32);
+  static constexpr int kElemBytes = BF16 ? 2 : 4;
+  static constexpr int kChunkElems = 16 / kElemBytes;     // per 16-byte load
+  static constexpr int kChunksPerRow = kCols / kChunkElems;
+};
+
+// Quantize the two adjacent columns c0, c0+1 of a staged tile over the 32
+// rows starting at tile row tr (global row r0). x2 receives the 32 element
+// pairs; the column group codes go to codes (COLS layout) and scales.
+template <bool SR>
+__device__ __forceinline__ void column_pair_groups(
+    const float (&a)[32], const float (&b)[32], int64_t r0, int64_t c0,
+    int64_t rows, int64_t cols, RngKey key, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  uint32_t ma = 0, mb = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    ma = max(ma, __float_as_uint(a[j]) & 0x7FFFFFFFu);
+    mb = max(mb, __float_as_uint(b[j]) & 0x7FFFFFFFu);
+  }
+  const uint32_t sa = scale_byte(ma), sbb = scale_byte(mb);
+  const float mula = inv_scale(sa), mulb = inv_scale(sbb);
+  uint32_t wa[4], wb[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float va[8], vb[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      va[j] = a[8 * q + j] * mula;
+      vb[j] = b[8 * q + j] * mulb;
+    }
+    if (SR) {
+      // Element (r, c) has random-number index i = r*cols + c. c0 is even;
+      // when i is even, (r, c0) and (r, c0+1) are the two halves of pair
+      // i/2; when cols is odd and r is odd, they belong to adjacent pairs.
+      uint32_t ha[4], hb[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t r_a[2], r_b[2];
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const int64_t r = r0 + 8 * q + 2 * k + t;
+          const uint64_t i = uint64_t(r) * uint64_t(cols) + uint64_t(c0);
+          const uint64_t p = i >> 1;
+          const uint32_t h = mix32(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
+          if ((i & 1) == 0) {
+            r_a[t] = h & 0xFFFFu;
+            r_b[t] = h >> 16;
+          } else {
+            const uint64_t p2 = p + 1;
+            const uint32_t h2 =
+                mix32(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
+            r_a[t] = h >> 16;
+            r_b[t] = h2 & 0xFFFFu;
+          }
+        }
+        ha[k] = r_a[0] | (r_a[1] << 16);
+        hb[k] = r_b[0] | (r_b[1] << 16);
+      }
+      wa[q] = e2m1x8_sr(va, ha);
+      wb[q] = e2m1x8_sr(vb, hb);
+    } else {
+      wa[q] = e2m1x8_rn(va);
+      wb[q] = e2m1x8_rn(vb);
+    }
+  }
+  if (sa == 0xFFu) wa[0] = wa[1] = wa[2] = wa[3] = 0;
+  if (sbb == 0xFFu) wb[0] = wb[1] = wb[2] = wb[3] = 0;
+  const int64_t half_rows = rows / 2;
+  if (c0 < cols) {
+    *reinterpret_cast<uint4*>(codes + c0 * half_rows + r0 / 2) =
+        make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    scales[c0 * (rows / 32) + r0 / 32] = static_cast<uint8_t>(sa);
+  }
+  if (c0 + 1 < cols) {
+    *reinterpret_cast<uint4*>(codes + (c0 + 1) * half_rows + r0 / 2) =
+        make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    scales[(c0 + 1) * (rows / 32) + r0 / 32] = static_cast<uint8_t>(sbb);
+  }
+}
+
+// Load one [128 x kCols] tile into shared memory (zero outside the tensor).
+// VEC: every row starts 16-byte aligned and cols is a multiple of the
+// 16-byte chunk, so chunks are either wholly inside or wholly outside.
+template <bool BF16, bool VEC>
+__device__ __forceinline__ void load_tile(const void* __restrict__ x,
+                                          int64_t rows, int64_t cols,
+                                          int64_t tile_r, int64_t tile_c,
+                                          uint4* tile) {
+  using T = ColTile<BF16>;
+  constexpr int kChunks = kTileRows * T::kChunksPerRow;
+  constexpr int kPer = kChunks / T::kThreads;
+  uint4 buf[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = k * T::kThreads + threadIdx.x;
+    const int r = idx / T::kChunksPerRow, ch = idx % T::kChunksPerRow;
+    const int64_t gr = tile_r + r, gc = tile_c + int64_t(ch) * T::kChunkElems;
+    if (VEC) {
+      buf[k] = (gr < rows && gc < cols)
+                   ? ld_stream(static_cast<const char*>(x) +
+                               (gr * cols + gc) * T::kElemBytes)
+                   : make_uint4(0, 0, 0, 0);
+    } else {
+      uint32_t e[4] = {0, 0, 0, 0};
+      if (BF16) {
+        const uint16_t* p = static_cast<const uint16_t*>(x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (gr < rows && gc + j < cols)
+            e[j / 2] |= uint32_t(p[gr * cols + gc + j]) << (16 * (j & 1));
+      } else {
+        const uint32_t* p = static_cast<const uint32_t*>(x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (gr < rows && gc + j < cols) e[j] = p[gr * cols + gc + j];
+      }
+      buf[k] = make_uint4(e[0], e[1], e[2], e[3]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) tile[k * T::kThreads + threadIdx.x] = buf[k];
+}
+
+template <bool BF16, bool SR, bool VEC>
+__global__ void __launch_bounds__(ColTile<BF16>::kThreads)
+    k_quant_cols(const void* __restrict__ x, int64_t rows, int64_t cols,
+                 RngKey key, uint8_t* __restrict__ codes,
+                 uint8_t* __restrict__ scales) {
+  using T = ColTile<BF16>;
+  __shared__ uint4 tile[kTileRows * T::kChunksPerRow];
+  const int64_t tiles_c = (cols + T::kCols - 1) / T::kCols;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
+  const int cp = threadIdx.x % (T::kCols / 2);
+  const int rg = threadIdx.x / (T::kCols / 2);
+  for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int64_t tile_r = (t / tiles_c) * kTileRows;
+    const int64_t tile_c = (t % tiles_c) * T::kCols;
+    load_tile<BF16, VEC>(x, rows, cols, tile_r, tile_c, tile);
+    __syncthreads();
+    const int64_t r0 = tile_r + 32 * rg;
+    if (r0 < rows) {
+      float a[32], b[32];
+      if (BF16) {
+        const uint32_t* s = reinterpret_cast<const uint32_t*>(tile);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t w = s[(32 * rg + j) * (T::kCols / 2) + cp];
+          a[j] = bf16_lo(w);
+          b[j] = bf16_hi(w);
+        }
+      } else {
+        const float2* s = reinterpret_cast<const float2*>(tile);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float2 w = s[(32 * rg + j) * (T::kCols / 2) + cp];
+          a[j] = w.x;
+          b[j] = w.y;
+        }
+      }
+      column_pair_groups<SR>(a, b, r0, tile_c + 2 * cp, rows, cols, key,
+                             codes, scales);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dequantize (flat groups; both layouts)
+// ---------------------------------------------------------------------------
+
+template <bool BF16OUT, int U>
+__global__ void __launch_bounds__(kRowThreads)
+    k_dequant(const uint8_t* __restrict__ codes,
+              const uint8_t* __restrict__ scales, int64_t n_groups,
+              void* __restrict__ y) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const int64_t warp = (int64_t(blockIdx.x) * kRowThreads + threadIdx.x) >> 5;
+  const int64_t chunk = (int64_t(gridDim.x) * kRowThreads) >> 2;
+  const int64_t my = warp * 8 + (lane >> 2);
+  for (int64_t base = 0; base < n_groups; base += chunk * U) {
+    uint32_t w[U], sb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * chunk + my;
+      const bool ok = g < n_groups;
+      w[u] = ok ? __ldcs(reinterpret_cast<const uint32_t*>(codes) + g * 4 + sub)
+                : 0u;
+      sb[u] = ok ? __ldcs(scales + g) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * chunk + my;
+      if (g >= n_groups) continue;
+      float f[8];
+      e2m1x8_decode(w[u], f);
+      const float s = scale_value(sb[u]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] *= s;
+      if (BF16OUT) {
+        uint4 o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                             pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        if (sb[u] == 0xFFu) o = make_uint4(kNaNbf16x2, kNaNbf16x2, kNaNbf16x2,
+                                           kNaNbf16x2);
+        __stcs(reinterpret_cast<uint4*>(static_cast<uint16_t*>(y) + g * 32 +
+                                        sub * 8),
+               o);
+      } else {
+        float4 o0 = make_float4(f[0], f[1], f[2], f[3]);
+        float4 o1 = make_float4(f[4], f[5], f[6], f[7]);
+        if (sb[u] == 0xFFu) {
+          const float n = __uint_as_float(kNaNf32);
+          o0 = o1 = make_float4(n, n, n, n);
+        }
+        float4* p = reinterpret_cast<float4*>(static_cast<float*>(y) + g * 32 +
+                                              sub * 8);
+        __stcs(p, o0);
+        __stcs(p + 1, o1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused double quantization (TetraJet rebuttal, Question 2): one pass over a
+// 128x128 tile computes the row layout of Q_D(1x32)(X) (RNE) in registers and
+// writes it; the same codes and row scales are staged in shared memory (4.5
+// bits per element), and the column pass decodes them, exactly, back to the
+// values of Q_D(X) and quantizes those along 32x1 columns with stochastic
+// rounding. X is read once; no transpose pass, no intermediate in global
+// memory.
+// ---------------------------------------------------------------------------
+
+constexpr int kDqThreads = 256;
+constexpr int kDqCols = 128;
+
+template <bool BF16>
+__global__ void __launch_bounds__(kDqThreads)
+    k_double_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
+                   RngKey key, uint8_t* __restrict__ row_codes,
+                   uint8_t* __restrict__ row_scales,
+                   uint8_t* __restrict__ col_codes,
+                   uint8_t* __restrict__ col_scales) {
+  // Q_D(X) of the tile: codes [128 rows][64 bytes] and the scale byte of
+  // every 1x32 row group [128 rows][4].
+  __shared__ uint32_t s_codes[kTileRows * (kDqCols / 8)];
+  __shared__ uint8_t s_scales[kTileRows * (kDqCols / 32)];
+  const int64_t tiles_c = (cols + kDqCols - 1) / kDqCols;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
+  const int ch = threadIdx.x & 15;   // 8-column chunk of a tile row
+  const int rr = threadIdx.x >> 4;   // tile row, plus 16 per pass
+  const int cp = threadIdx.x & 63;   // column pair of the column pass
+  const int rg = threadIdx.x >> 6;   // 32-row group of the column pass
+  constexpr int kPasses = kTileRows / 16;
+  for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const int64_t tile_r = (t / tiles_c) * kTileRows;
+    const int64_t tile_c = (t % tiles_c) * kDqCols;
+    const int64_t gc = tile_c + 8 * ch;
+    // Row pass: all loads first, then quad-reduced 1x32 groups.
+    uint4 raw[kPasses][BF16 ? 1 : 2];
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+      const int64_t gr = tile_r + rr + 16 * k;
+      const bool ok = gr < rows && gc < cols;
+      if (BF16) {
+        raw[k][0] = ok ? ld_stream(static_cast<const uint16_t*>(x) + gr * cols + gc)
+                       : make_uint4(0, 0, 0, 0);
+      } else {
+        const float* p = static_cast<const float*>(x) + gr * cols + gc;
+        raw[k][0] = ok ? ld_stream(p) : make_uint4(0, 0, 0, 0);
+        raw[k][BF16 ? 0 : 1] = ok ? ld_stream(p + 4) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+      const int64_t gr = tile_r + rr + 16 * k;
+      const bool ok = gr < rows && gc < cols;
+      float v[8];
+      if (BF16) {
+        const uint4 w = raw[k][0];
+        v[0] = bf16_lo(w.x), v[1] = bf16_hi(w.x), v[2] = bf16_lo(w.y);
+        v[3] = bf16_hi(w.y), v[4] = bf16_lo(w.z), v[5] = bf16_hi(w.z);
+        v[6] = bf16_lo(w.w), v[7] = bf16_hi(w.w);
+      } else {
+        const uint4 a = raw[k][0], b = raw[k][BF16 ? 0 : 1];
+        v[0] = __uint_as_float(a.x), v[1] = __uint_as_float(a.y);
+        v[2] = __uint_as_float(a.z), v[3] = __uint_as_float(a.w);
+        v[4] = __uint_as_float(b.x), v[5] = __uint_as_float(b.y);
+        v[6] = __uint_as_float(b.z), v[7] = __uint_as_float(b.w);
+      }
+      uint32_t amax = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        amax = max(amax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+      const uint32_t sb = scale_byte(amax);
+      const float mul = inv_scale(sb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] *= mul;
+      uint32_t word = e2m1x8_rn(v);
+      if (sb == 0xFFu) word = 0;
+      if (ok) {
+        *reinterpret_cast<uint32_t*>(row_codes + gr * (cols / 2) + gc / 2) = word;
+        if ((ch & 3) == 0) row_scales[gr * (cols / 32) + gc / 32] = uint8_t(sb);
+      }
+      s_codes[(rr + 16 * k) * (kDqCols / 8) + ch] = word;
+      if ((ch & 3) == 0) s_scales[(rr + 16 * k) * (kDqCols / 32) + ch / 4] = uint8_t(sb);
+    }
+    __syncthreads();
+    // Column pass: decode Q_D(X) for columns 2cp, 2cp+1 over 32 rows (one
+    // shared byte per row holds both codes), then stochastic rounding along
+    // the 32x1 groups. A row group of scale 0xFF decodes to NaN (0 x inf).
+    const int64_t r0 = tile_r + 32 * rg;
+    if (r0 < rows) {
+      const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
+      float a[32], b[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t w4 = 0;
+        float sv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 32 * rg + 4 * q + i;
+          w4 |= uint32_t(sc[r * (kDqCols / 2) + cp]) << (8 * i);
+          sv[i] = scale_value(s_scales[r * (kDqCols / 32) + cp / 16]);
+        }
+        float f[8];
+        e2m1x8_decode(w4, f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[4 * q + i] = f[2 * i] * sv[i];
+          b[4 * q + i] = f[2 * i + 1] * sv[i];
+        }
+      }
+      column_pair_groups<true>(a, b, r0, tile_c + 2 * cp, rows, cols, key,
+                               col_codes, col_scales);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Launchers
+// ---------------------------------------------------------------------------
+
+int persistent_grid(const void* kernel, int threads, size_t smem,
+                    int64_t work_blocks) {
+  int dev = 0, sms = 148, per_sm = 1;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads,
+                                                    smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  int64_t g = int64_t(sms) * per_sm;
+  if (work_blocks < g) g = work_blocks;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+template <bool BF16, bool SR>
+static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
+                                   RngKey key, uint8_t* codes,
+                                   uint8_t* scales, cudaStream_t s) {
+  constexpr int U = BF16 ? 4 : 2;
+  auto kern = k_quant_rows<BF16, SR, U>;
+  const int64_t groups_per_block = (kRowThreads / 4) * U;
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                   kRowThreads, 0,
+                                   (n_groups + groups_per_block - 1) /
+                                       groups_per_block);
+  kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rows(const void* x, bool bf16, int64_t rows,
+                              int64_t cols, bool sr, uint64_t seed,
+                              uint8_t* codes, uint8_t* scales,
+                              cudaStream_t s) {
+  const int64_t n_groups = rows * cols / kGroup;
+  const RngKey key = make_key(seed, 0);
+  if (bf16)
+    return sr ? quant_rows_impl<true, true>(x, n_groups, key, codes, scales, s)
+              : quant_rows_impl<true, false>(x, n_groups, key, codes, scales, s);
+  return sr ? quant_rows_impl<false, true>(x, n_groups, key, codes, scales, s)
+            : quant_rows_impl<false, false>(x, n_groups, key, codes, scales, s);
+}
+
+template <bool BF16, bool SR, bool VEC>
+static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
+                                   RngKey key, uint8_t* codes,
+                                   uint8_t* scales, cudaStream_t s) {
+  using T = ColTile<BF16>;
+  auto kern = k_quant_cols<BF16, SR, VEC>;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
+                          ((cols + T::kCols - 1) / T::kCols);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                   T::kThreads, 0, n_tiles);
+  kern<<<grid, T::kThreads, 0, s>>>(x, rows, cols, key, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
+                              int64_t cols, bool sr, uint64_t seed,
+                              uint8_t* codes, uint8_t* scales,
+                              cudaStream_t s) {
+  const RngKey key = make_key(seed, 0);
+  const bool vec = cols % (bf16 ? 8 : 4) == 0;
+#define MXFP4_COLS(B, S, V) \
+  return quant_cols_impl<B, S, V>(x, rows, cols, key, codes, scales, s)
+  if (bf16) {
+    if (sr) {
+      if (vec) MXFP4_COLS(true, true, true);
+      MXFP4_COLS(true, true, false);
+    }
+    if (vec) MXFP4_COLS(true, false, true);
+    MXFP4_COLS(true, false, false);
+  }
+  if (sr) {
+    if (vec) MXFP4_COLS(false, true, true);
+    MXFP4_COLS(false, true, false);
+  }
+  if (vec) MXFP4_COLS(false, false, true);
+  MXFP4_COLS(false, false, false);
+#undef MXFP4_COLS
+}
+
+cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
+                           int64_t n_groups, void* y, bool bf16_out,
+                           cudaStream_t s) {
+  constexpr int U = 4;
+  const int64_t groups_per_block = (kRowThreads / 4) * U;
+  const int64_t blocks = (n_groups + groups_per_block - 1) / groups_per_block;
+  if (bf16_out) {
+    auto kern = k_dequant<true, U>;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kRowThreads, 0, blocks);
+    kern<<<grid, kRowThreads, 0, s>>>(codes, scales, n_groups, y);
+  } else {
+    auto kern = k_dequant<false, U>;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kRowThreads, 0, blocks);
+    kern<<<grid, kRowThreads, 0, s>>>(codes, scales, n_groups, y);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mxfp4
+
+namespace mxfp4 {
+
+cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
+                                int64_t cols, uint64_t seed,
+                                uint8_t* row_codes, uint8_t* row_scales,
+                                uint8_t* col_codes, uint8_t* col_scales,
+                                cudaStream_t s) {
+  const RngKey key = make_key(seed, 0);
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
+                          ((cols + kDqCols - 1) / kDqCols);
+  if (bf16) {
+    auto kern = k_double_quant<true>;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kDqThreads, 0, n_tiles);
+    kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes,
+                                     row_scales, col_codes, col_scales);
+  } else {
+    auto kern = k_double_quant<false>;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kDqThreads, 0, n_tiles);
+    kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes,
+                                     row_scales, col_codes, col_scales);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace mxfp4

@@ -63,16 +63,17 @@ def _declare(L):
         "orc_encode": ([dbl, i32, i32, u32], i32),
         "orc_decode": ([i32, i32], dbl),
         "orc_rht_sign": ([u64, u32], i32),
-        "orc_quantize": ([vp, i32, i64, i64, i32, i32, u64, _u8p, _u8p], i32),
+        "orc_quantize": ([vp, i32, i64, i64, i64, i32, i32, u64, _u8p, _u8p],
+                         i32),
         "orc_dequantize": ([_u8p, _u8p, i64, i64, i32, vp, i32], i32),
-        "orc_double_quantize": ([vp, i32, i64, i64, u64, _u8p, _u8p, _u8p,
-                                 _u8p], i32),
+        "orc_double_quantize": ([vp, i32, i64, i64, i64, u64, _u8p, _u8p,
+                                 _u8p, _u8p], i32),
         "orc_rht_rotate": ([vp, i32, i64, i64, u64, _fp], i32),
-        "orc_rht_quantize": ([vp, i32, i64, i64, u64, i32, u64, _u8p, _u8p,
-                              _fp], i32),
+        "orc_rht_quantize": ([vp, i32, i64, i64, i64, u64, i32, u64, _u8p,
+                              _u8p, _fp], i32),
         "orc_osc_step": ([_fp, _fp, _fp, _fp, i64, i64, i32, ctypes.c_float],
                          i64),
-        "orc_osc_synthetic_update": ([_fp, i64, i64, u64, u32,
+        "orc_osc_synthetic_update": ([_fp, i64, i64, i64, u64, u32,
                                       ctypes.c_float], i32),
     }
     for name, (args, res) in sig.items():
@@ -131,14 +132,16 @@ class Oracle:
         return self.L.orc_rht_sign(sign_seed, c)
 
     # --- tensor entry points ---------------------------------------------
-    def quantize(self, x, axis=ROWS, rounding=RNE, seed=0):
-        """Block quantize x [R, C]; returns (codes, scales), axis layout."""
+    def quantize(self, x, axis=ROWS, rounding=RNE, seed=0, row0=0):
+        """Block quantize x [R, C]; returns (codes, scales), axis layout.
+        x may be rows row0.. of a larger tensor (random numbers are keyed by
+        the index in that tensor)."""
         x, dt = _as_input(x)
         R, C = x.shape
         codes = np.zeros(R * C // 2, np.uint8)
         scales = np.zeros(R * C // 32, np.uint8)
-        rc = self.L.orc_quantize(x.ctypes.data, dt, R, C, axis, rounding,
-                                 seed, _u8(codes), _u8(scales))
+        rc = self.L.orc_quantize(x.ctypes.data, dt, R, C, row0, axis,
+                                 rounding, seed, _u8(codes), _u8(scales))
         if rc != 0:
             raise ValueError("bad shape for the oracle quantizer: %s" % (x.shape,))
         if axis == ROWS:
@@ -159,14 +162,14 @@ class Oracle:
                               y.ctypes.data, dt)
         return y.view(ml_dtypes.bfloat16) if dt == DT_BF16 else y
 
-    def double_quantize(self, x, seed):
+    def double_quantize(self, x, seed, row0=0):
         """Q_S(32x1)(Q_D(1x32)(x)): (row codes, row scales, col codes,
         col scales)."""
         x, dt = _as_input(x)
         R, C = x.shape
         out = [np.zeros(R * C // 2, np.uint8), np.zeros(R * C // 32, np.uint8),
                np.zeros(R * C // 2, np.uint8), np.zeros(R * C // 32, np.uint8)]
-        rc = self.L.orc_double_quantize(x.ctypes.data, dt, R, C, seed,
+        rc = self.L.orc_double_quantize(x.ctypes.data, dt, R, C, row0, seed,
                                         *[_u8(a) for a in out])
         if rc != 0:
             raise ValueError("bad shape for the oracle double quantizer")
@@ -181,7 +184,7 @@ class Oracle:
             raise ValueError("bad shape for the oracle rotation")
         return y
 
-    def rht_quantize(self, x, sign_seed, rounding, sr_seed):
+    def rht_quantize(self, x, sign_seed, rounding, sr_seed, row0=0):
         """Rotate each 1x32 row group, quantize along rows: (codes, scales,
         rotated fp32)."""
         x, dt = _as_input(x)
@@ -189,7 +192,7 @@ class Oracle:
         codes = np.zeros(R * C // 2, np.uint8)
         scales = np.zeros(R * C // 32, np.uint8)
         y = np.zeros((R, C), np.float32)
-        if self.L.orc_rht_quantize(x.ctypes.data, dt, R, C, sign_seed,
+        if self.L.orc_rht_quantize(x.ctypes.data, dt, R, C, row0, sign_seed,
                                    rounding, sr_seed, _u8(codes),
                                    _u8(scales), _f32(y)):
             raise ValueError("bad shape for the oracle rotation")
@@ -207,11 +210,12 @@ class Oracle:
             raise ValueError("bad shape for the oracle tracker")
         return int(n)
 
-    def osc_synthetic_update(self, w, seed, step, rel_step=1e-4):
+    def osc_synthetic_update(self, w, seed, step, rel_step=1e-4, row0=0):
         if w.dtype != np.float32 or not w.flags.c_contiguous:
             raise TypeError("w must be contiguous float32")
         R, C = w.shape
-        self.L.orc_osc_synthetic_update(_f32(w), R, C, seed, step, rel_step)
+        self.L.orc_osc_synthetic_update(_f32(w), R, C, row0, seed, step,
+                                        rel_step)
 
 
 _default = None

@@ -208,10 +208,12 @@ static void put_nibble(uint8_t* codes, int64_t byte, int high, int code) {
     codes[byte] = (uint8_t)((codes[byte] & 0xF0) | code);
 }
 
-/* Quantize values xv[rows*cols] (row-major doubles). */
+/* Quantize values xv[rows*cols] (row-major doubles). The tensor is rows
+ * row0 .. row0+rows-1 of a larger one with the same cols: random numbers
+ * are keyed by the element's index in that larger tensor. */
 static void quantize_values(const double* xv, int64_t rows, int64_t cols,
-                            int axis, int rounding, uint64_t seed,
-                            uint8_t* codes, uint8_t* scales) {
+                            int64_t row0, int axis, int rounding,
+                            uint64_t seed, uint8_t* codes, uint8_t* scales) {
   double g[32];
   uint64_t idx[32];
   int cq[32];
@@ -220,7 +222,7 @@ static void quantize_values(const double* xv, int64_t rows, int64_t cols,
       for (int64_t k = 0; k < cols / 32; ++k) {
         for (int j = 0; j < 32; ++j) {
           int64_t c = 32 * k + j;
-          idx[j] = (uint64_t)(r * cols + c);
+          idx[j] = (uint64_t)((row0 + r) * cols + c);
           g[j] = xv[r * cols + c];
         }
         scales[r * (cols / 32) + k] =
@@ -235,7 +237,7 @@ static void quantize_values(const double* xv, int64_t rows, int64_t cols,
       for (int64_t k = 0; k < rows / 32; ++k) {
         for (int j = 0; j < 32; ++j) {
           int64_t r = 32 * k + j;
-          idx[j] = (uint64_t)(r * cols + c);
+          idx[j] = (uint64_t)((row0 + r) * cols + c);
           g[j] = xv[r * cols + c];
         }
         scales[c * (rows / 32) + k] =
@@ -258,14 +260,15 @@ static double* load_all(const void* x, int dtype, int64_t n) {
 /* Public oracle entry points                                           */
 /* ------------------------------------------------------------------ */
 
-/* Block quantize x[rows][cols] along axis. Returns 0, or -1 on bad shape. */
+/* Block quantize x[rows][cols] along axis (rows row0.. of a larger tensor,
+ * see quantize_values). Returns 0, or -1 on bad shape. */
 int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
-                 int axis, int rounding, uint64_t seed, uint8_t* codes,
-                 uint8_t* scales) {
+                 int64_t row0, int axis, int rounding, uint64_t seed,
+                 uint8_t* codes, uint8_t* scales) {
   if (rows <= 0 || cols <= 0) return -1;
   if ((axis == AX_ROWS ? cols : rows) % 32 != 0) return -1;
   double* xv = load_all(x, dtype, rows * cols);
-  quantize_values(xv, rows, cols, axis, rounding, seed, codes, scales);
+  quantize_values(xv, rows, cols, row0, axis, rounding, seed, codes, scales);
   free(xv);
   return 0;
 }
@@ -314,16 +317,17 @@ int orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
 
 /* [TJ] Question 2: Q_S along 32x1 groups of the dequantized Q_D(1x32)(X). */
 int orc_double_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
-                        uint64_t seed, uint8_t* row_codes,
+                        int64_t row0, uint64_t seed, uint8_t* row_codes,
                         uint8_t* row_scales, uint8_t* col_codes,
                         uint8_t* col_scales) {
   if (rows <= 0 || cols <= 0 || rows % 32 || cols % 32) return -1;
   int64_t n = rows * cols;
   double* xv = load_all(x, dtype, n);
-  quantize_values(xv, rows, cols, AX_ROWS, RND_RNE, 0, row_codes, row_scales);
+  quantize_values(xv, rows, cols, row0, AX_ROWS, RND_RNE, 0, row_codes,
+                  row_scales);
   double* d = (double*)malloc((size_t)n * sizeof(double));
   dequantize_values(row_codes, row_scales, rows, cols, AX_ROWS, d);
-  quantize_values(d, rows, cols, AX_COLS, RND_SR, seed, col_codes,
+  quantize_values(d, rows, cols, row0, AX_COLS, RND_SR, seed, col_codes,
                   col_scales);
   free(d);
   free(xv);
@@ -369,13 +373,14 @@ int orc_rht_rotate(const void* x, int dtype, int64_t rows, int64_t cols,
 /* Rotate, then quantize the fp32 rotated values along rows. `rotated`
  * receives y when not NULL. */
 int orc_rht_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
-                     uint64_t sign_seed, int rounding, uint64_t sr_seed,
-                     uint8_t* codes, uint8_t* scales, float* rotated) {
+                     int64_t row0, uint64_t sign_seed, int rounding,
+                     uint64_t sr_seed, uint8_t* codes, uint8_t* scales,
+                     float* rotated) {
   if (rows <= 0 || cols <= 0 || cols % 32) return -1;
   float* y = rotated ? rotated : (float*)malloc((size_t)(rows * cols) * 4);
   orc_rht_rotate(x, dtype, rows, cols, sign_seed, y);
-  orc_quantize(y, DT_F32, rows, cols, AX_ROWS, rounding, sr_seed, codes,
-               scales);
+  orc_quantize(y, DT_F32, rows, cols, row0, AX_ROWS, rounding, sr_seed,
+               codes, scales);
   if (!rotated) free(y);
   return 0;
 }
@@ -439,13 +444,16 @@ int64_t orc_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
 
 /* Synthetic update driving the tracker: w += s * (rel_step * |w|), as an
  * fp32 multiply then an fp32 add; s from stream 2 keyed by
- * seed + (step << 32), one hash per element index. */
+ * seed + (step << 32), one hash per element index (rows row0.. of a larger
+ * tensor with the same cols). */
 int orc_osc_synthetic_update(float* w, int64_t rows, int64_t cols,
-                             uint64_t seed, uint32_t step, float rel_step) {
+                             int64_t row0, uint64_t seed, uint32_t step,
+                             float rel_step) {
   if (rows <= 0 || cols <= 0) return -1;
   uint32_t k = orc_key(seed + ((uint64_t)step << 32), 2);
   for (int64_t i = 0; i < rows * cols; ++i) {
-    double s = (orc_counter_hash(k, (uint64_t)i) >> 31) ? -1.0 : 1.0;
+    uint64_t gi = (uint64_t)(row0 * cols + i);
+    double s = (orc_counter_hash(k, gi) >> 31) ? -1.0 : 1.0;
     float mag = (float)((double)rel_step * fabs((double)w[i]));
     w[i] = (float)((double)w[i] + s * (double)mag);
   }

@@ -38,8 +38,9 @@ MUTANTS = [
      "double frac = (a - GRID[lo]) / (GRID[lo + 1] - GRID[lo]);",
      "double frac = (a - GRID[lo]) / 0.5;",
      ["test_sr_exhaustive_over_random_numbers_is_unbiased"]),
-    ("column rng index transposed", "idx[j] = (uint64_t)(r * cols + c);\n          g[j] = xv[r * cols + c];\n        }\n        scales[c",
-     "idx[j] = (uint64_t)(c * rows + r);\n          g[j] = xv[r * cols + c];\n        }\n        scales[c",
+    ("column rng index transposed",
+     "int64_t r = 32 * k + j;\n          idx[j] = (uint64_t)((row0 + r) * cols + c);",
+     "int64_t r = 32 * k + j;\n          idx[j] = (uint64_t)(c * rows + r);",
      ["test_cols_sr_uses_input_row_major_index"]),
     ("column codes in row layout",
      "put_nibble(codes, c * (rows / 2) + r / 2, (int)(r & 1), cq[j]);",
@@ -60,8 +61,9 @@ MUTANTS = [
      "orc_key(sign_seed, 0)", ["test_hash_frozen_known_answers"]),
     ("decode drops the sign", "return (code & 8) ? -v : v;", "return v;",
      ["test_decode_every_code_and_scale_against_library"]),
-    ("double quant columns from X", "quantize_values(d, rows, cols, AX_COLS",
-     "quantize_values(xv, rows, cols, AX_COLS", ["test_double_quant_structure"]),
+    ("double quant columns from X", "quantize_values(d, rows, cols, row0, AX_COLS",
+     "quantize_values(xv, rows, cols, row0, AX_COLS",
+     ["test_double_quant_structure"]),
     ("tracker without abs",
      "float dist_w = (float)fabs((double)w[i] - (double)w_snap[i]);",
      "float dist_w = (float)((double)w[i] - (double)w_snap[i]);",
@@ -72,8 +74,8 @@ MUTANTS = [
      ["test_osc_worked_example_from_the_page"]),
     ("no reset at window end", "      d_w[i] = 0.0f;\n", "",
      ["test_osc_accumulators_before_window_end"]),
-    ("update sign bit", "(orc_counter_hash(k, (uint64_t)i) >> 31)",
-     "(orc_counter_hash(k, (uint64_t)i) >> 30)",
+    ("update sign bit", "(orc_counter_hash(k, gi) >> 31)",
+     "(orc_counter_hash(k, gi) >> 30)",
      ["test_osc_synthetic_update_magnitude_and_signs"]),
 ]
 
