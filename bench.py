@@ -72,6 +72,11 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", default="",
+                    help="comma-separated ops to run (profiling); default all")
+    ap.add_argument("--rows", type=int, default=SWEEP[0],
+                    help="rows of the sweep workload (profiling a smaller case)")
     return ap.parse_args()
 
 
@@ -246,11 +251,11 @@ def run_ours(args):
     m.lib()
 
     # inputs (seeded numpy), uploaded once
-    x_np = W.sweep(seed=SEED + rank)
+    R, C = args.rows, SWEEP[1]
+    x_np = W.sweep(seed=SEED + rank, rows=R)
     w_np = W.osc_w(seed=3 + rank)
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     w0 = torch.from_numpy(w_np).to(dev)
-    R, C = SWEEP
     u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)  # noqa: E731
     rows_out = (u8(R, C // 2), u8(R, C // 32))
     cols_out = (u8(C, R // 2), u8(C, R // 32))
@@ -261,7 +266,11 @@ def run_ours(args):
     ws, dwt, dqt = w.clone(), torch.zeros_like(w), torch.zeros_like(w)
     nflag = torch.zeros(1, dtype=torch.int64, device=dev)
 
-    ops = list(BYTES_PER_ELEM)
+    ops = [o for o in BYTES_PER_ELEM if not args.only or o in args.only.split(",")]
+    if (R, C) != SWEEP:
+        for o in ops:
+            if o not in ("osc_update", "osc_step"):
+                OP_ELEMS[o] = R * C
     stream = torch.cuda.current_stream(dev)
     ev = {op: [] for op in ops}
     step_no = [0]
@@ -272,6 +281,8 @@ def run_ours(args):
         pairs = []
 
         def timed(op, fn):
+            if op not in ops:
+                return
             if record:
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
@@ -319,6 +330,13 @@ def run_ours(args):
     elapsed_ms = float(t_max.item())
 
     # end to end: pinned host input -> device -> kernels -> host results
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ops": ops,
+                              "ms": elapsed_ms / args.steps}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     w_host = torch.from_numpy(w_np).pin_memory()
     outs = [rows_out[0], rows_out[1], cols_out[0], cols_out[1], *dq_out, y,

@@ -59,10 +59,23 @@ __host__ __forceinline__ RngKey make_key(uint64_t seed, uint32_t stream) {
   return r;
 }
 
+// mix32 on the device. The right shifts are written as high halves of
+// multiplies by powers of two (h >> k == umulhi(h, 2^(32-k))), which issue
+// on the multiply-add pipe and leave the integer logic pipe, the limit of the
+// stochastic-rounding kernels, to the XORs.
+__device__ __forceinline__ uint32_t mix32_d(uint32_t h) {
+  h ^= __umulhi(h, 1u << 16);
+  h *= 0x85EBCA6Bu;
+  h ^= __umulhi(h, 1u << 19);
+  h *= 0xC2B2AE35u;
+  h ^= __umulhi(h, 1u << 16);
+  return h;
+}
+
 // Inner hash for counters whose high word is `hi` (0 for every tensor below
 // 2^33 elements).
 __device__ __forceinline__ uint32_t inner_key(RngKey key, uint32_t hi) {
-  return hi == 0 ? key.k0 : mix32(key.k ^ hi);
+  return hi == 0 ? key.k0 : mix32_d(key.k ^ hi);
 }
 
 // ---------------------------------------------------------------------------
@@ -109,37 +122,46 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
   return out;
 }
 
-// Stochastic E2M1 code of one scaled value v (exact) with its 16-bit random
-// number r: lo = largest grid value <= |v|, hi = the next one; the result is
-// hi iff (r + 0.5) * 2^-16 < (|v| - lo) / (hi - lo); |v| >= 6 gives 6.
+// Stochastic E2M1 code of one scaled value v (exact): lo = largest grid
+// value <= |v|, hi = the next one; the result is hi iff
+// (r + 0.5) * 2^-16 < (|v| - lo) / (hi - lo), r the element's 16-bit random
+// number; |v| >= 6 gives 6.
 //
 // In every binade [2^k, 2^k+1) with k >= 0 the grid keeps one mantissa bit,
-// so the low 22 mantissa bits of |v| are frac * 2^22 exactly. Below 1 the
-// grid step is 0.5 throughout; 1 + |v| (rounded up) maps [0, 1) onto [1, 2)
-// with the same step and rounding up keeps the comparison exact, because the
-// threshold lies on the 2^-18 grid. The test is then frac * 2^22 > 64r + 32.
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
-  float a = fabsf(v);
-  bool small = a < 1.0f;
-  float y = __fadd_ru(a, small ? 1.0f : 0.0f);
-  uint32_t yb = __float_as_uint(y);
-  int m = static_cast<int>(yb >> 22) - (small ? 254 : 252);
-  uint32_t rem = yb & 0x3FFFFFu;
-  m += rem > ((r << 6) | 32u) ? 1 : 0;
-  m = m > 7 ? 7 : m;
-  return (__float_as_uint(v) >> 28 & 8u) | static_cast<uint32_t>(m);
+// so the low 22 mantissa bits of |v| are frac * 2^22 exactly, and the code is
+// the top bits of |v| minus those of 0.5. Below 1 the grid step is 0.5
+// throughout; (1 + |v|) / 2 rounded up maps [0, 1) onto [0.5, 1] with the
+// same structure (and is the smaller of the two for |v| >= 1, the larger
+// below), and rounding up keeps the test exact because the threshold lies on
+// the 2^-18 grid. The test frac * 2^22 > 64r + 32 is an addition: with
+// noise = 2^22 - 33 - 64r, the mantissa field plus noise carries into bit 22
+// exactly when the value goes up (the carry may run on into the exponent:
+// 1.5 -> 2, 3 -> 4). The bias 0.5 = 0x3F000000 is folded into the noise.
+__device__ __forceinline__ uint32_t sr_noise_lo(uint32_t h) {  // r = h & 0xFFFF
+  return (~(h * 64u) & 0x3FFFC0u) | 0xC100001Fu;
+}
+__device__ __forceinline__ uint32_t sr_noise_hi(uint32_t h) {  // r = h >> 16
+  return (~__umulhi(h, 1u << 22) & 0x3FFFC0u) | 0xC100001Fu;
 }
 
-// Stochastic codes of 8 values whose random numbers come in 4 hashes (pair
-// k of the 8 values uses h[k]: low half for the even element).
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
+  const float a = fabsf(v);
+  const uint32_t half1p = __float_as_uint(__fmaf_ru(a, 0.5f, 0.5f));
+  uint32_t y = max(__float_as_uint(a), half1p);
+  y = min(y, 0x40C00000u);  // |v| >= 6 saturates to 6
+  const uint32_t m = (y + noise) >> 22;
+  return m + (__float_as_uint(v) >> 31) * 8u;
+}
+
+// Stochastic codes of 8 values; pair k of the 8 values takes its two random
+// numbers from h[k] (low half for the even element).
 __device__ __forceinline__ uint32_t e2m1x8_sr(const float* v,
                                               const uint32_t* h) {
   uint32_t out = 0;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    uint32_t c0 = e2m1_sr(v[2 * k], h[k] & 0xFFFFu);
-    uint32_t c1 = e2m1_sr(v[2 * k + 1], h[k] >> 16);
-    out |= (c0 | (c1 << 4)) << (8 * k);
+    out += e2m1_sr(v[2 * k], sr_noise_lo(h[k])) * (1u << (8 * k));
+    out += e2m1_sr(v[2 * k + 1], sr_noise_hi(h[k])) * (1u << (8 * k + 4));
   }
   return out;
 }
@@ -200,7 +222,7 @@ __device__ __forceinline__ void e2m1x8_decode(uint32_t w, float* out) {
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) {
-  return __uint_as_float(w << 16);
+  return __uint_as_float(w * 65536u);
 }
 __device__ __forceinline__ float bf16_hi(uint32_t w) {
   return __uint_as_float(w & 0xFFFF0000u);

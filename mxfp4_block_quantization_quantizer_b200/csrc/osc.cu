@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kOscThreads)
     const uint32_t kh = inner_key(key, uint32_t(i0 >> 32));
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t h = mix32(kh + uint32_t(i0) + j);
+      const uint32_t h = mix32_d(kh + uint32_t(i0) + j);
       const float mag = __fmul_rn(rel_step, fabsf(f[j]));
       f[j] = __fadd_rn(f[j], (h >> 31) ? -mag : mag);
     }
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kOscThreads)
   }
   if (blockIdx.x == 0 && threadIdx.x < n - n4 * 4) {
     const uint64_t i = uint64_t(n4) * 4 + threadIdx.x;
-    const uint32_t h = mix32(inner_key(key, uint32_t(i >> 32)) + uint32_t(i));
+    const uint32_t h = mix32_d(inner_key(key, uint32_t(i >> 32)) + uint32_t(i));
     const float mag = __fmul_rn(rel_step, fabsf(w[i]));
     w[i] = __fadd_rn(w[i], (h >> 31) ? -mag : mag);
   }

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kRowThreads)
         const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
         uint32_t h[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) h[k] = mix32(kh + uint32_t(p0) + k);
+        for (int k = 0; k < 4; ++k) h[k] = mix32_d(kh + uint32_t(p0) + k);
         word = e2m1x8_sr(v[u], h);
       } else {
         word = e2m1x8_rn(v[u]);
@@ -118,61 +118,60 @@ struct ColTile {
 };
 
 // Quantize the two adjacent columns c0, c0+1 of a staged tile over the 32
-// rows starting at tile row tr (global row r0). x2 receives the 32 element
-// pairs; the column group codes go to codes (COLS layout) and scales.
-template <bool SR>
+// rows r0 .. r0+31: a[] and b[] hold the values, ma and mb the fp32 bit
+// patterns of their absolute maxima. Codes go to the COLS layout.
+//
+// Random numbers: element (r, c) has index i = r*cols + c and c0 is even.
+// EVEN (cols even): i is even, so (r, c0) and (r, c0+1) are the two halves
+// of pair i/2, and the pair index of row r0+j is p0 + j*cols/2. Otherwise
+// odd rows split the two columns over adjacent pairs. BIG: the tensor has
+// 2^33 elements or more, so the high word of a pair index can be nonzero.
+template <bool SR, bool EVEN, bool BIG>
 __device__ __forceinline__ void column_pair_groups(
-    const float (&a)[32], const float (&b)[32], int64_t r0, int64_t c0,
-    int64_t rows, int64_t cols, RngKey key, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales) {
-  uint32_t ma = 0, mb = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    ma = max(ma, __float_as_uint(a[j]) & 0x7FFFFFFFu);
-    mb = max(mb, __float_as_uint(b[j]) & 0x7FFFFFFFu);
-  }
+    const float (&a)[32], const float (&b)[32], uint32_t ma, uint32_t mb,
+    int64_t r0, int64_t c0, int64_t rows, int64_t cols, RngKey key,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const uint32_t sa = scale_byte(ma), sbb = scale_byte(mb);
   const float mula = inv_scale(sa), mulb = inv_scale(sbb);
-  uint32_t wa[4], wb[4];
+  uint32_t wa[4] = {0, 0, 0, 0}, wb[4] = {0, 0, 0, 0};
+  if (SR) {
+    const uint64_t i0 = uint64_t(r0) * uint64_t(cols) + uint64_t(c0);
+    const uint32_t p0_lo = uint32_t(i0 >> 1);
+    const uint32_t half_lo = uint32_t(uint64_t(cols) >> 1);
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float va[8], vb[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      va[j] = a[8 * q + j] * mula;
-      vb[j] = b[8 * q + j] * mulb;
-    }
-    if (SR) {
-      // Element (r, c) has random-number index i = r*cols + c. c0 is even;
-      // when i is even, (r, c0) and (r, c0+1) are the two halves of pair
-      // i/2; when cols is odd and r is odd, they belong to adjacent pairs.
-      uint32_t ha[4], hb[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t r_a[2], r_b[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int64_t r = r0 + 8 * q + 2 * k + t;
-          const uint64_t i = uint64_t(r) * uint64_t(cols) + uint64_t(c0);
-          const uint64_t p = i >> 1;
-          const uint32_t h = mix32(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
-          if ((i & 1) == 0) {
-            r_a[t] = h & 0xFFFFu;
-            r_b[t] = h >> 16;
-          } else {
-            const uint64_t p2 = p + 1;
-            const uint32_t h2 =
-                mix32(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
-            r_a[t] = h >> 16;
-            r_b[t] = h2 & 0xFFFFu;
-          }
+    for (int j = 0; j < 32; ++j) {
+      uint32_t na, nb;
+      if (EVEN && !BIG) {
+        const uint32_t h = mix32_d(key.k0 + p0_lo + uint32_t(j) * half_lo);
+        na = sr_noise_lo(h);
+        nb = sr_noise_hi(h);
+      } else {
+        const uint64_t i = i0 + uint64_t(j) * uint64_t(cols);
+        const uint64_t p = i >> 1;
+        const uint32_t h = mix32_d(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
+        if ((i & 1) == 0) {
+          na = sr_noise_lo(h);
+          nb = sr_noise_hi(h);
+        } else {
+          const uint64_t p2 = p + 1;
+          const uint32_t h2 =
+              mix32_d(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
+          na = sr_noise_hi(h);
+          nb = sr_noise_lo(h2);
         }
-        ha[k] = r_a[0] | (r_a[1] << 16);
-        hb[k] = r_b[0] | (r_b[1] << 16);
       }
-      wa[q] = e2m1x8_sr(va, ha);
-      wb[q] = e2m1x8_sr(vb, hb);
-    } else {
+      wa[j >> 3] += e2m1_sr(a[j] * mula, na) * (1u << (4 * (j & 7)));
+      wb[j >> 3] += e2m1_sr(b[j] * mulb, nb) * (1u << (4 * (j & 7)));
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float va[8], vb[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        va[j] = a[8 * q + j] * mula;
+        vb[j] = b[8 * q + j] * mulb;
+      }
       wa[q] = e2m1x8_rn(va);
       wb[q] = e2m1x8_rn(vb);
     }
@@ -190,6 +189,17 @@ __device__ __forceinline__ void column_pair_groups(
         make_uint4(wb[0], wb[1], wb[2], wb[3]);
     scales[(c0 + 1) * (rows / 32) + r0 / 32] = static_cast<uint8_t>(sbb);
   }
+}
+
+// Absolute maxima (fp32 bit patterns) of the two bf16 columns packed in the
+// 32 words w (low half: column c0, high half: column c0+1).
+__device__ __forceinline__ void packed_col_max(const uint32_t (&w)[32],
+                                               uint32_t& ma, uint32_t& mb) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) m = umax16x2(m, w[j] & 0x7FFF7FFFu);
+  ma = m << 16;
+  mb = m & 0xFFFF0000u;
 }
 
 // Load one [128 x kCols] tile into shared memory (zero outside the tensor).
@@ -235,7 +245,7 @@ __device__ __forceinline__ void load_tile(const void* __restrict__ x,
   for (int k = 0; k < kPer; ++k) tile[k * T::kThreads + threadIdx.x] = buf[k];
 }
 
-template <bool BF16, bool SR, bool VEC>
+template <bool BF16, bool SR, bool VEC, bool EVEN, bool BIG>
 __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     k_quant_cols(const void* __restrict__ x, int64_t rows, int64_t cols,
                  RngKey key, uint8_t* __restrict__ codes,
@@ -254,13 +264,17 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     const int64_t r0 = tile_r + 32 * rg;
     if (r0 < rows) {
       float a[32], b[32];
+      uint32_t ma = 0, mb = 0;
       if (BF16) {
         const uint32_t* s = reinterpret_cast<const uint32_t*>(tile);
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = s[(32 * rg + j) * (T::kCols / 2) + cp];
+        packed_col_max(w, ma, mb);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const uint32_t w = s[(32 * rg + j) * (T::kCols / 2) + cp];
-          a[j] = bf16_lo(w);
-          b[j] = bf16_hi(w);
+          a[j] = bf16_lo(w[j]);
+          b[j] = bf16_hi(w[j]);
         }
       } else {
         const float2* s = reinterpret_cast<const float2*>(tile);
@@ -269,10 +283,12 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
           const float2 w = s[(32 * rg + j) * (T::kCols / 2) + cp];
           a[j] = w.x;
           b[j] = w.y;
+          ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
+          mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
         }
       }
-      column_pair_groups<SR>(a, b, r0, tile_c + 2 * cp, rows, cols, key,
-                             codes, scales);
+      column_pair_groups<SR, EVEN, BIG>(a, b, ma, mb, r0, tile_c + 2 * cp,
+                                        rows, cols, key, codes, scales);
     }
     __syncthreads();
   }
@@ -348,7 +364,7 @@ __global__ void __launch_bounds__(kRowThreads)
 constexpr int kDqThreads = 256;
 constexpr int kDqCols = 128;
 
-template <bool BF16>
+template <bool BF16, bool BIG>
 __global__ void __launch_bounds__(kDqThreads)
     k_double_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
                    RngKey key, uint8_t* __restrict__ row_codes,
@@ -429,6 +445,7 @@ __global__ void __launch_bounds__(kDqThreads)
     if (r0 < rows) {
       const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
       float a[32], b[32];
+      uint32_t ma = 0, mb = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         uint32_t w4 = 0;
@@ -445,10 +462,14 @@ __global__ void __launch_bounds__(kDqThreads)
         for (int i = 0; i < 4; ++i) {
           a[4 * q + i] = f[2 * i] * sv[i];
           b[4 * q + i] = f[2 * i + 1] * sv[i];
+          ma = max(ma, __float_as_uint(a[4 * q + i]) & 0x7FFFFFFFu);
+          mb = max(mb, __float_as_uint(b[4 * q + i]) & 0x7FFFFFFFu);
         }
       }
-      column_pair_groups<true>(a, b, r0, tile_c + 2 * cp, rows, cols, key,
-                               col_codes, col_scales);
+      // cols is a multiple of 32 here, so every pair index is even-aligned
+      column_pair_groups<true, true, BIG>(a, b, ma, mb, r0, tile_c + 2 * cp,
+                                          rows, cols, key, col_codes,
+                                          col_scales);
     }
     __syncthreads();
   }
@@ -502,12 +523,12 @@ cudaError_t launch_quant_rows(const void* x, bool bf16, int64_t rows,
             : quant_rows_impl<false, false>(x, n_groups, key, codes, scales, s);
 }
 
-template <bool BF16, bool SR, bool VEC>
+template <bool BF16, bool SR, bool VEC, bool EVEN, bool BIG>
 static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
   using T = ColTile<BF16>;
-  auto kern = k_quant_cols<BF16, SR, VEC>;
+  auto kern = k_quant_cols<BF16, SR, VEC, EVEN, BIG>;
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + T::kCols - 1) / T::kCols);
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
@@ -516,29 +537,36 @@ static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
   return cudaGetLastError();
 }
 
+// 2^33 elements or more: pair indices reach 2^32.
+static bool big_tensor(int64_t rows, int64_t cols) {
+  return rows * cols >= (int64_t(1) << 33);
+}
+
+template <bool BF16>
+static cudaError_t quant_cols_dispatch(const void* x, int64_t rows,
+                                       int64_t cols, bool sr, RngKey key,
+                                       uint8_t* codes, uint8_t* scales,
+                                       cudaStream_t s) {
+  const bool vec = cols % (BF16 ? 8 : 4) == 0;
+  if (!sr)
+    return vec ? quant_cols_impl<BF16, false, true, true, false>(x, rows, cols, key, codes, scales, s)
+               : quant_cols_impl<BF16, false, false, true, false>(x, rows, cols, key, codes, scales, s);
+  if (cols % 2 != 0)  // odd rows split column pairs over two hashes
+    return quant_cols_impl<BF16, true, false, false, true>(x, rows, cols, key, codes, scales, s);
+  if (big_tensor(rows, cols))
+    return vec ? quant_cols_impl<BF16, true, true, true, true>(x, rows, cols, key, codes, scales, s)
+               : quant_cols_impl<BF16, true, false, true, true>(x, rows, cols, key, codes, scales, s);
+  return vec ? quant_cols_impl<BF16, true, true, true, false>(x, rows, cols, key, codes, scales, s)
+             : quant_cols_impl<BF16, true, false, true, false>(x, rows, cols, key, codes, scales, s);
+}
+
 cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
                               int64_t cols, bool sr, uint64_t seed,
                               uint8_t* codes, uint8_t* scales,
                               cudaStream_t s) {
   const RngKey key = make_key(seed, 0);
-  const bool vec = cols % (bf16 ? 8 : 4) == 0;
-#define MXFP4_COLS(B, S, V) \
-  return quant_cols_impl<B, S, V>(x, rows, cols, key, codes, scales, s)
-  if (bf16) {
-    if (sr) {
-      if (vec) MXFP4_COLS(true, true, true);
-      MXFP4_COLS(true, true, false);
-    }
-    if (vec) MXFP4_COLS(true, false, true);
-    MXFP4_COLS(true, false, false);
-  }
-  if (sr) {
-    if (vec) MXFP4_COLS(false, true, true);
-    MXFP4_COLS(false, true, false);
-  }
-  if (vec) MXFP4_COLS(false, false, true);
-  MXFP4_COLS(false, false, false);
-#undef MXFP4_COLS
+  return bf16 ? quant_cols_dispatch<true>(x, rows, cols, sr, key, codes, scales, s)
+              : quant_cols_dispatch<false>(x, rows, cols, sr, key, codes, scales, s);
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
@@ -573,19 +601,13 @@ cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
   const RngKey key = make_key(seed, 0);
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + kDqCols - 1) / kDqCols);
-  if (bf16) {
-    auto kern = k_double_quant<true>;
-    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
-                                     kDqThreads, 0, n_tiles);
-    kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes,
-                                     row_scales, col_codes, col_scales);
-  } else {
-    auto kern = k_double_quant<false>;
-    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
-                                     kDqThreads, 0, n_tiles);
-    kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes,
-                                     row_scales, col_codes, col_scales);
-  }
+  const bool big = big_tensor(rows, cols);
+  auto kern = bf16 ? (big ? k_double_quant<true, true> : k_double_quant<true, false>)
+                   : (big ? k_double_quant<false, true> : k_double_quant<false, false>);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                   kDqThreads, 0, n_tiles);
+  kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes, row_scales,
+                                   col_codes, col_scales);
   return cudaGetLastError();
 }
 

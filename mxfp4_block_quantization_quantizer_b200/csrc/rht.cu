@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(kRhtThreads)
     // warp w hashes the 32 column signs of column group blockIdx.x*8 + w
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t c = uint32_t((int64_t(blockIdx.x) * kRhtGroupsX + w) * 32 + lane);
-    const unsigned neg = __ballot_sync(0xFFFFFFFFu, (mix32(sign_key + c) >> 31) != 0);
+    const unsigned neg = __ballot_sync(0xFFFFFFFFu, (mix32_d(sign_key + c) >> 31) != 0);
     if (lane == 0) sign_bits[w] = neg;
   }
   __syncthreads();
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kRhtThreads)
         const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
         uint32_t h[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) h[t] = mix32(kh + uint32_t(p0) + t);
+        for (int t = 0; t < 4; ++t) h[t] = mix32_d(kh + uint32_t(p0) + t);
         wq[q] = e2m1x8_sr(v, h);
       } else {
         wq[q] = e2m1x8_rn(v);
