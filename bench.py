@@ -55,6 +55,53 @@ STEP_BYTES = sum(alg_bytes(op) for op in BYTES_PER_ELEM)
 STEP_ELEMS = sum(OP_ELEMS.values())
 
 
+def rank_seed(rank):
+    """Each rank quantizes its own seeded sweep (replicas, weak scaling)."""
+    return SEED + rank
+
+
+def reduce_max(value, world, device=None):
+    """Max over ranks of a float (the timed region's duration)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_step, steps, elapsed_ms_max):
+    """Whole-job GB/s: all ranks' algorithmic bytes over the slowest rank."""
+    return world * bytes_per_step * steps / (elapsed_ms_max * 1e-3) / 1e9
+
+
+def kernel_source_digest():
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "mxfp4_block_quantization_quantizer_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(op):
+    """ncu dram read+write bytes per full launch of op, from
+    profiles/dram_traffic.txt, or None when the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    digest = kernel_source_digest()
+    for line in lines:
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == op and parts[2] == "src=" + digest:
+            return float(parts[1])
+    return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -252,7 +299,7 @@ def run_ours(args):
 
     # inputs (seeded numpy), uploaded once
     R, C = args.rows, SWEEP[1]
-    x_np = W.sweep(seed=SEED + rank, rows=R)
+    x_np = W.sweep(seed=rank_seed(rank), rows=R)
     w_np = W.osc_w(seed=3 + rank)
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     w0 = torch.from_numpy(w_np).to(dev)
@@ -324,10 +371,7 @@ def run_ours(args):
     elapsed_ms = start.elapsed_time(end)
     for op, a, b in all_pairs:
         ev[op].append(a.elapsed_time(b))
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = reduce_max(elapsed_ms, world, dev)
 
     # end to end: pinned host input -> device -> kernels -> host results
     if args.no_e2e:
@@ -364,11 +408,9 @@ def run_ours(args):
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_end)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    e2e_ms = reduce_max(e2e_ms, world, dev)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_ms = float(te.item())
 
     if rank == 0:
         peak, peak_kind = measured_peaks()
@@ -380,14 +422,8 @@ def run_ours(args):
                           "bytes": alg_bytes(op)}
         dom = max(per_op, key=lambda k: per_op[k]["us"])
         step_s = elapsed_ms * 1e-3 / args.steps
-        value = world * STEP_BYTES / step_s / 1e9
-        traffic = None
-        prof = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(prof):
-            try:
-                traffic = json.load(open(prof)).get(dom)
-            except Exception:
-                traffic = None
+        value = job_gbs(world, STEP_BYTES, args.steps, elapsed_ms)
+        traffic = measured_traffic(dom)
         line = {
             "metric": "MXFP4 quantize GB/s (bytes in+out)",
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -402,7 +438,7 @@ def run_ours(args):
                          "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": per_op[dom]["frac"], "traffic": traffic},
             "ops": per_op,
-            "e2e": {"value": world * STEP_BYTES * args.e2e_steps / (e2e_ms * 1e-3) / 1e9,
+            "e2e": {"value": job_gbs(world, STEP_BYTES, args.e2e_steps, e2e_ms),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": len(ops) * args.steps,

@@ -137,20 +137,22 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 // noise = 2^22 - 33 - 64r, the mantissa field plus noise carries into bit 22
 // exactly when the value goes up (the carry may run on into the exponent:
 // 1.5 -> 2, 3 -> 4). The bias 0.5 = 0x3F000000 is folded into the noise.
+__device__ __forceinline__ uint32_t sr_noise(uint32_t r) {
+  return r * 0xFFFFFFC0u + 0xC13FFFDFu;  // (2^22 - 33 - 64r) - 0x3F000000
+}
 __device__ __forceinline__ uint32_t sr_noise_lo(uint32_t h) {  // r = h & 0xFFFF
-  return (~(h * 64u) & 0x3FFFC0u) | 0xC100001Fu;
+  return sr_noise(h & 0xFFFFu);
 }
 __device__ __forceinline__ uint32_t sr_noise_hi(uint32_t h) {  // r = h >> 16
-  return (~__umulhi(h, 1u << 22) & 0x3FFFC0u) | 0xC100001Fu;
+  return sr_noise(__umulhi(h, 1u << 16));
 }
 
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
   const float a = fabsf(v);
-  const uint32_t half1p = __float_as_uint(__fmaf_ru(a, 0.5f, 0.5f));
-  uint32_t y = max(__float_as_uint(a), half1p);
-  y = min(y, 0x40C00000u);  // |v| >= 6 saturates to 6
-  const uint32_t m = (y + noise) >> 22;
-  return m + (__float_as_uint(v) >> 31) * 8u;
+  float y = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
+  y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
+  const uint32_t m = __umulhi(__float_as_uint(y) + noise, 1u << 10);  // >> 22
+  return m + __umulhi(__float_as_uint(v), 2u) * 8u;                  // sign
 }
 
 // Stochastic codes of 8 values; pair k of the 8 values takes its two random
@@ -249,6 +251,25 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
       : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
       : "l"(p));
   return r;
+}
+
+// Asynchronous 16-byte global -> shared copy (bypassing L1). When !valid
+// nothing is read and the 16 shared bytes are zero-filled; src must still be
+// a mapped global address.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* src,
+                                           bool valid) {
+  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst),
+               "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+// Wait until at most N committed groups of this thread are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
 constexpr uint32_t kNaNbf16x2 = 0x7FC07FC0u;

@@ -117,51 +117,58 @@ struct ColTile {
   static constexpr int kChunksPerRow = kCols / kChunkElems;
 };
 
-// Quantize the two adjacent columns c0, c0+1 of a staged tile over the 32
-// rows r0 .. r0+31: a[] and b[] hold the values, ma and mb the fp32 bit
-// patterns of their absolute maxima. Codes go to the COLS layout.
-//
-// Random numbers: element (r, c) has index i = r*cols + c and c0 is even.
-// EVEN (cols even): i is even, so (r, c0) and (r, c0+1) are the two halves
-// of pair i/2, and the pair index of row r0+j is p0 + j*cols/2. Otherwise
-// odd rows split the two columns over adjacent pairs. BIG: the tensor has
-// 2^33 elements or more, so the high word of a pair index can be nonzero.
-template <bool SR, bool EVEN, bool BIG>
-__device__ __forceinline__ void column_pair_groups(
-    const float (&a)[32], const float (&b)[32], uint32_t ma, uint32_t mb,
-    int64_t r0, int64_t c0, int64_t rows, int64_t cols, RngKey key,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+// Random-number noise of the two adjacent elements (r0+j, c0), (r0+j, c0+1)
+// of a column pass. Element (r, c) has index i = r*cols + c; c0 is even.
+// EVEN (cols even): i is even, so both elements are the halves of pair
+// i/2, and the pair index of row r0+j is p0 + j*cols/2. Otherwise odd rows
+// split the two elements over adjacent pairs. BIG: the tensor has 2^33
+// elements or more, so the high word of a pair index can be nonzero.
+template <bool EVEN, bool BIG>
+__device__ __forceinline__ void column_noise(RngKey key, uint64_t i0,
+                                             int64_t cols, int j, uint32_t& na,
+                                             uint32_t& nb) {
+  if (EVEN && !BIG) {
+    const uint32_t h = mix32_d(key.k0 + uint32_t(i0 >> 1) +
+                               uint32_t(j) * uint32_t(uint64_t(cols) >> 1));
+    na = sr_noise_lo(h);
+    nb = sr_noise_hi(h);
+  } else {
+    const uint64_t i = i0 + uint64_t(j) * uint64_t(cols);
+    const uint64_t p = i >> 1;
+    const uint32_t h = mix32_d(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
+    if ((i & 1) == 0) {
+      na = sr_noise_lo(h);
+      nb = sr_noise_hi(h);
+    } else {
+      const uint64_t p2 = p + 1;
+      const uint32_t h2 = mix32_d(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
+      na = sr_noise_hi(h);
+      nb = sr_noise_lo(h2);
+    }
+  }
+}
+
+// Quantize the two adjacent columns c0, c0+1 over the 32 rows r0 .. r0+31.
+// get(j) returns the values of row r0+j (x: column c0, y: column c0+1); ma
+// and mb are the fp32 bit patterns of the two columns' absolute maxima.
+// Codes go to the COLS layout.
+template <bool SR, bool EVEN, bool BIG, typename Get>
+__device__ __forceinline__ void column_pair_quant(
+    Get get, uint32_t ma, uint32_t mb, int64_t r0, int64_t c0, int64_t rows,
+    int64_t cols, RngKey key, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
   const uint32_t sa = scale_byte(ma), sbb = scale_byte(mb);
   const float mula = inv_scale(sa), mulb = inv_scale(sbb);
   uint32_t wa[4] = {0, 0, 0, 0}, wb[4] = {0, 0, 0, 0};
   if (SR) {
     const uint64_t i0 = uint64_t(r0) * uint64_t(cols) + uint64_t(c0);
-    const uint32_t p0_lo = uint32_t(i0 >> 1);
-    const uint32_t half_lo = uint32_t(uint64_t(cols) >> 1);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       uint32_t na, nb;
-      if (EVEN && !BIG) {
-        const uint32_t h = mix32_d(key.k0 + p0_lo + uint32_t(j) * half_lo);
-        na = sr_noise_lo(h);
-        nb = sr_noise_hi(h);
-      } else {
-        const uint64_t i = i0 + uint64_t(j) * uint64_t(cols);
-        const uint64_t p = i >> 1;
-        const uint32_t h = mix32_d(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
-        if ((i & 1) == 0) {
-          na = sr_noise_lo(h);
-          nb = sr_noise_hi(h);
-        } else {
-          const uint64_t p2 = p + 1;
-          const uint32_t h2 =
-              mix32_d(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
-          na = sr_noise_hi(h);
-          nb = sr_noise_lo(h2);
-        }
-      }
-      wa[j >> 3] += e2m1_sr(a[j] * mula, na) * (1u << (4 * (j & 7)));
-      wb[j >> 3] += e2m1_sr(b[j] * mulb, nb) * (1u << (4 * (j & 7)));
+      column_noise<EVEN, BIG>(key, i0, cols, j, na, nb);
+      const float2 v = get(j);
+      wa[j >> 3] += e2m1_sr(v.x * mula, na) * (1u << (4 * (j & 7)));
+      wb[j >> 3] += e2m1_sr(v.y * mulb, nb) * (1u << (4 * (j & 7)));
     }
   } else {
 #pragma unroll
@@ -169,8 +176,9 @@ __device__ __forceinline__ void column_pair_groups(
       float va[8], vb[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        va[j] = a[8 * q + j] * mula;
-        vb[j] = b[8 * q + j] * mulb;
+        const float2 v = get(8 * q + j);
+        va[j] = v.x * mula;
+        vb[j] = v.y * mulb;
       }
       wa[q] = e2m1x8_rn(va);
       wb[q] = e2m1x8_rn(vb);
@@ -191,15 +199,43 @@ __device__ __forceinline__ void column_pair_groups(
   }
 }
 
-// Absolute maxima (fp32 bit patterns) of the two bf16 columns packed in the
-// 32 words w (low half: column c0, high half: column c0+1).
-__device__ __forceinline__ void packed_col_max(const uint32_t (&w)[32],
-                                               uint32_t& ma, uint32_t& mb) {
-  uint32_t m = 0;
+// Column pass over a staged tile: thread (rg, cp) quantizes the columns
+// 2cp, 2cp+1 over tile rows 32rg .. 32rg+31. The tile is read twice (maxima,
+// then codes) rather than held in registers. A warp reads 32 consecutive
+// 32-bit words (bf16) or 64-bit words (fp32) of one row: no bank conflicts.
+template <bool BF16, bool SR, bool EVEN, bool BIG>
+__device__ __forceinline__ void column_tile_pass(
+    const uint4* tile, int kcols, int rg, int cp, int64_t tile_r,
+    int64_t tile_c, int64_t rows, int64_t cols, RngKey key,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  const int64_t r0 = tile_r + 32 * rg;
+  if (r0 >= rows) return;
+  uint32_t ma = 0, mb = 0;
+  if (BF16) {
+    const uint32_t* s = reinterpret_cast<const uint32_t*>(tile) + 32 * rg * (kcols / 2) + cp;
+    uint32_t m = 0;
 #pragma unroll
-  for (int j = 0; j < 32; ++j) m = umax16x2(m, w[j] & 0x7FFF7FFFu);
-  ma = m << 16;
-  mb = m & 0xFFFF0000u;
+    for (int j = 0; j < 32; ++j) m = umax16x2(m, s[j * (kcols / 2)] & 0x7FFF7FFFu);
+    ma = m << 16;
+    mb = m & 0xFFFF0000u;
+    column_pair_quant<SR, EVEN, BIG>(
+        [&](int j) {
+          const uint32_t w = s[j * (kcols / 2)];
+          return make_float2(bf16_lo(w), bf16_hi(w));
+        },
+        ma, mb, r0, tile_c + 2 * cp, rows, cols, key, codes, scales);
+  } else {
+    const float2* s = reinterpret_cast<const float2*>(tile) + 32 * rg * (kcols / 2) + cp;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float2 w = s[j * (kcols / 2)];
+      ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
+      mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
+    }
+    column_pair_quant<SR, EVEN, BIG>([&](int j) { return s[j * (kcols / 2)]; },
+                                     ma, mb, r0, tile_c + 2 * cp, rows, cols,
+                                     key, codes, scales);
+  }
 }
 
 // Load one [128 x kCols] tile into shared memory (zero outside the tensor).
@@ -245,7 +281,31 @@ __device__ __forceinline__ void load_tile(const void* __restrict__ x,
   for (int k = 0; k < kPer; ++k) tile[k * T::kThreads + threadIdx.x] = buf[k];
 }
 
-template <bool BF16, bool SR, bool VEC, bool EVEN, bool BIG>
+// Stage one [128 x kCols] tile of a tensor whose rows are 16-byte aligned
+// and whose cols are a whole number of 16-byte chunks, with asynchronous
+// copies (zero-filled outside the tensor), and commit them as one group.
+template <bool BF16>
+__device__ __forceinline__ void stage_tile_async(const void* __restrict__ x,
+                                                 int64_t rows, int64_t cols,
+                                                 int64_t tile_r, int64_t tile_c,
+                                                 uint4* tile) {
+  using T = ColTile<BF16>;
+  constexpr int kPer = kTileRows * T::kChunksPerRow / T::kThreads;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = k * T::kThreads + threadIdx.x;
+    const int r = idx / T::kChunksPerRow, ch = idx % T::kChunksPerRow;
+    const int64_t gr = tile_r + r, gc = tile_c + int64_t(ch) * T::kChunkElems;
+    const bool ok = gr < rows && gc < cols;
+    const char* src = static_cast<const char*>(x) +
+                      (ok ? (gr * cols + gc) * T::kElemBytes : 0);
+    cp_async16(tile + idx, src, ok);
+  }
+  cp_async_commit();
+}
+
+// Column groups, general shapes: one staged tile at a time, plain loads.
+template <bool BF16, bool SR, bool EVEN, bool BIG>
 __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     k_quant_cols(const void* __restrict__ x, int64_t rows, int64_t cols,
                  RngKey key, uint8_t* __restrict__ codes,
@@ -259,39 +319,49 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
   for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
     const int64_t tile_r = (t / tiles_c) * kTileRows;
     const int64_t tile_c = (t % tiles_c) * T::kCols;
-    load_tile<BF16, VEC>(x, rows, cols, tile_r, tile_c, tile);
+    load_tile<BF16, false>(x, rows, cols, tile_r, tile_c, tile);
     __syncthreads();
-    const int64_t r0 = tile_r + 32 * rg;
-    if (r0 < rows) {
-      float a[32], b[32];
-      uint32_t ma = 0, mb = 0;
-      if (BF16) {
-        const uint32_t* s = reinterpret_cast<const uint32_t*>(tile);
-        uint32_t w[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) w[j] = s[(32 * rg + j) * (T::kCols / 2) + cp];
-        packed_col_max(w, ma, mb);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          a[j] = bf16_lo(w[j]);
-          b[j] = bf16_hi(w[j]);
-        }
-      } else {
-        const float2* s = reinterpret_cast<const float2*>(tile);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float2 w = s[(32 * rg + j) * (T::kCols / 2) + cp];
-          a[j] = w.x;
-          b[j] = w.y;
-          ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
-          mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
-        }
-      }
-      column_pair_groups<SR, EVEN, BIG>(a, b, ma, mb, r0, tile_c + 2 * cp,
-                                        rows, cols, key, codes, scales);
-    }
+    column_tile_pass<BF16, SR, EVEN, BIG>(tile, T::kCols, rg, cp, tile_r,
+                                          tile_c, rows, cols, key, codes,
+                                          scales);
     __syncthreads();
   }
+}
+
+// Column groups, 16-byte aligned rows: double-buffered. The copies of the
+// CTA's next tile are in flight while the current tile is quantized.
+template <bool BF16, bool SR, bool EVEN, bool BIG>
+__global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
+    k_quant_cols_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
+                      RngKey key, uint8_t* __restrict__ codes,
+                      uint8_t* __restrict__ scales) {
+  using T = ColTile<BF16>;
+  constexpr int kChunks = kTileRows * T::kChunksPerRow;
+  extern __shared__ uint4 smem[];  // two tiles
+  const int64_t tiles_c = (cols + T::kCols - 1) / T::kCols;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
+  const int cp = threadIdx.x % (T::kCols / 2);
+  const int rg = threadIdx.x / (T::kCols / 2);
+  int64_t t = blockIdx.x;
+  if (t >= n_tiles) return;
+  stage_tile_async<BF16>(x, rows, cols, (t / tiles_c) * kTileRows,
+                         (t % tiles_c) * T::kCols, smem);
+  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+    const int64_t tn = t + gridDim.x;
+    if (tn < n_tiles)
+      stage_tile_async<BF16>(x, rows, cols, (tn / tiles_c) * kTileRows,
+                             (tn % tiles_c) * T::kCols, smem + (buf ^ 1) * kChunks);
+    else
+      cp_async_commit();  // keep one group per iteration
+    cp_async_wait<1>();   // this tile's copies (the older group) are done
+    __syncthreads();
+    column_tile_pass<BF16, SR, EVEN, BIG>(smem + buf * kChunks, T::kCols, rg,
+                                          cp, (t / tiles_c) * kTileRows,
+                                          (t % tiles_c) * T::kCols, rows, cols,
+                                          key, codes, scales);
+    __syncthreads();  // the next iteration's copies overwrite this buffer
+  }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -467,12 +537,132 @@ __global__ void __launch_bounds__(kDqThreads)
         }
       }
       // cols is a multiple of 32 here, so every pair index is even-aligned
-      column_pair_groups<true, true, BIG>(a, b, ma, mb, r0, tile_c + 2 * cp,
-                                          rows, cols, key, col_codes,
-                                          col_scales);
+      column_pair_quant<true, true, BIG>(
+          [&](int j) { return make_float2(a[j], b[j]); }, ma, mb, r0,
+          tile_c + 2 * cp, rows, cols, key, col_codes, col_scales);
     }
     __syncthreads();
   }
+}
+
+// Row pass of one 1x32 group quarter (8 values of tile row tr, chunk ch):
+// returns the 4 code bytes; writes the row codes and scale to global memory
+// (when in range) and stages them in shared memory for the column pass.
+__device__ __forceinline__ void dq_row_chunk(float (&v)[8], bool ok, int64_t gr,
+                                             int64_t gc, int64_t cols, int tr,
+                                             int ch, uint8_t* __restrict__ row_codes,
+                                             uint8_t* __restrict__ row_scales,
+                                             uint32_t* s_codes, uint8_t* s_scales) {
+  uint32_t amax = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) amax = max(amax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+  amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  const uint32_t sb = scale_byte(amax);
+  const float mul = inv_scale(sb);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] *= mul;
+  uint32_t word = e2m1x8_rn(v);
+  if (sb == 0xFFu) word = 0;
+  if (ok) {
+    *reinterpret_cast<uint32_t*>(row_codes + gr * (cols / 2) + gc / 2) = word;
+    if ((ch & 3) == 0) row_scales[gr * (cols / 32) + gc / 32] = uint8_t(sb);
+  }
+  s_codes[tr * (kDqCols / 8) + ch] = word;
+  if ((ch & 3) == 0) s_scales[tr * (kDqCols / 32) + ch / 4] = uint8_t(sb);
+}
+
+// Column pass of the double quantizer over the staged Q_D(X) codes: decode
+// columns 2cp, 2cp+1 of rows 32rg.. (one shared byte per row holds both
+// codes; a row group of scale 0xFF decodes to NaN as 0 x inf), then
+// stochastic rounding along the 32x1 groups.
+template <bool BIG>
+__device__ __forceinline__ void dq_column_pass(
+    const uint32_t* s_codes, const uint8_t* s_scales, int rg, int cp,
+    int64_t tile_r, int64_t tile_c, int64_t rows, int64_t cols, RngKey key,
+    uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_scales) {
+  const int64_t r0 = tile_r + 32 * rg;
+  if (r0 >= rows) return;
+  const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
+  float a[32], b[32];
+  uint32_t ma = 0, mb = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t w4 = 0;
+    float sv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = 32 * rg + 4 * q + i;
+      w4 |= uint32_t(sc[r * (kDqCols / 2) + cp]) << (8 * i);
+      sv[i] = scale_value(s_scales[r * (kDqCols / 32) + cp / 16]);
+    }
+    float f[8];
+    e2m1x8_decode(w4, f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[4 * q + i] = f[2 * i] * sv[i];
+      b[4 * q + i] = f[2 * i + 1] * sv[i];
+      ma = max(ma, __float_as_uint(a[4 * q + i]) & 0x7FFFFFFFu);
+      mb = max(mb, __float_as_uint(b[4 * q + i]) & 0x7FFFFFFFu);
+    }
+  }
+  // cols is a multiple of 32 here, so every pair index is even-aligned
+  column_pair_quant<true, true, BIG>(
+      [&](int j) { return make_float2(a[j], b[j]); }, ma, mb, r0,
+      tile_c + 2 * cp, rows, cols, key, col_codes, col_scales);
+}
+
+// Fused double quantization of bf16 X, double-buffered: the raw tiles are
+// staged with asynchronous copies, so the next tile streams in while the
+// current one is quantized along rows and then along columns.
+template <bool BIG>
+__global__ void __launch_bounds__(kDqThreads, 2)
+    k_double_quant_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
+                        RngKey key, uint8_t* __restrict__ row_codes,
+                        uint8_t* __restrict__ row_scales,
+                        uint8_t* __restrict__ col_codes,
+                        uint8_t* __restrict__ col_scales) {
+  constexpr int kChunks = kTileRows * (kDqCols / 8);
+  extern __shared__ uint4 smem[];  // two raw tiles, then the staged Q_D(X)
+  uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + 2 * kChunks);
+  uint8_t* s_scales = reinterpret_cast<uint8_t*>(s_codes + kTileRows * (kDqCols / 8));
+  const int64_t tiles_c = (cols + kDqCols - 1) / kDqCols;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
+  const int ch = threadIdx.x & 15, rr = threadIdx.x >> 4;
+  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  int64_t t = blockIdx.x;
+  if (t >= n_tiles) return;
+  stage_tile_async<true>(x, rows, cols, (t / tiles_c) * kTileRows,
+                         (t % tiles_c) * kDqCols, smem);
+  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+    const int64_t tn = t + gridDim.x;
+    if (tn < n_tiles)
+      stage_tile_async<true>(x, rows, cols, (tn / tiles_c) * kTileRows,
+                             (tn % tiles_c) * kDqCols, smem + (buf ^ 1) * kChunks);
+    else
+      cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const int64_t tile_r = (t / tiles_c) * kTileRows;
+    const int64_t tile_c = (t % tiles_c) * kDqCols;
+    const int64_t gc = tile_c + 8 * ch;
+    const uint4* raw = smem + buf * kChunks;
+#pragma unroll 2
+    for (int k = 0; k < kTileRows / 16; ++k) {
+      const int tr = rr + 16 * k;
+      const int64_t gr = tile_r + tr;
+      const uint4 w = raw[tr * (kDqCols / 8) + ch];
+      float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                    bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+      dq_row_chunk(v, gr < rows && gc < cols, gr, gc, cols, tr, ch, row_codes,
+                   row_scales, s_codes, s_scales);
+    }
+    __syncthreads();
+    dq_column_pass<BIG>(s_codes, s_scales, rg, cp, tile_r, tile_c, rows, cols,
+                        key, col_codes, col_scales);
+    __syncthreads();
+  }
+  cp_async_wait<0>();
 }
 
 }  // namespace
@@ -528,12 +718,24 @@ static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
   using T = ColTile<BF16>;
-  auto kern = k_quant_cols<BF16, SR, VEC, EVEN, BIG>;
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + T::kCols - 1) / T::kCols);
-  const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
-                                   T::kThreads, 0, n_tiles);
-  kern<<<grid, T::kThreads, 0, s>>>(x, rows, cols, key, codes, scales);
+  if (VEC) {
+    auto kern = k_quant_cols_pipe<BF16, SR, EVEN, BIG>;
+    constexpr size_t smem = 2 * kTileRows * T::kChunksPerRow * sizeof(uint4);
+    cudaError_t e = cudaFuncSetAttribute(
+        reinterpret_cast<const void*>(kern),
+        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     T::kThreads, smem, n_tiles);
+    kern<<<grid, T::kThreads, smem, s>>>(x, rows, cols, key, codes, scales);
+  } else {
+    auto kern = k_quant_cols<BF16, SR, EVEN, BIG>;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     T::kThreads, 0, n_tiles);
+    kern<<<grid, T::kThreads, 0, s>>>(x, rows, cols, key, codes, scales);
+  }
   return cudaGetLastError();
 }
 
@@ -602,8 +804,21 @@ cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + kDqCols - 1) / kDqCols);
   const bool big = big_tensor(rows, cols);
-  auto kern = bf16 ? (big ? k_double_quant<true, true> : k_double_quant<true, false>)
-                   : (big ? k_double_quant<false, true> : k_double_quant<false, false>);
+  if (bf16) {
+    auto kern = big ? k_double_quant_pipe<true> : k_double_quant_pipe<false>;
+    constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) +
+                            kTileRows * (kDqCols / 8) * 4 + kTileRows * (kDqCols / 32);
+    cudaError_t e = cudaFuncSetAttribute(
+        reinterpret_cast<const void*>(kern),
+        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kDqThreads, smem, n_tiles);
+    kern<<<grid, kDqThreads, smem, s>>>(x, rows, cols, key, row_codes,
+                                        row_scales, col_codes, col_scales);
+    return cudaGetLastError();
+  }
+  auto kern = big ? k_double_quant<false, true> : k_double_quant<false, false>;
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
                                    kDqThreads, 0, n_tiles);
   kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes, row_scales,
