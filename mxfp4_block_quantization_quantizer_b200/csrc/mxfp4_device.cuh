@@ -237,6 +237,16 @@ __device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
+// fp32 bit pattern of the largest |value| among 8 packed bf16 values: the
+// absolute bit patterns of finite and non-finite values order like their
+// magnitudes, so a per-half integer max finds the group maximum (and any
+// Inf/NaN, whose pattern is at least 0x7F80).
+__device__ __forceinline__ uint32_t bf16x8_absmax(uint4 w) {
+  const uint32_t m = umax16x2(umax16x2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
+                              umax16x2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+  return max(m << 16, m & 0xFFFF0000u);
+}
+
 // Two exact fp32 values -> packed bf16x2 (low element in the low half).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t d;

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kRowThreads)
 
   for (int64_t base = 0; base < n_groups; base += chunk * U) {
     float v[U][8];
+    uint32_t pmax[U];
     bool ok[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(kRowThreads)
         uint4 w = ok[u] ? ld_stream(static_cast<const uint16_t*>(x) + g * 32 +
                                     sub * 8)
                         : make_uint4(0, 0, 0, 0);
+        pmax[u] = bf16x8_absmax(w);
         v[u][0] = bf16_lo(w.x), v[u][1] = bf16_hi(w.x);
         v[u][2] = bf16_lo(w.y), v[u][3] = bf16_hi(w.y);
         v[u][4] = bf16_lo(w.z), v[u][5] = bf16_hi(w.z);
@@ -73,9 +75,13 @@ __global__ void __launch_bounds__(kRowThreads)
     for (int u = 0; u < U; ++u) {
       const int64_t g = base + u * chunk + my;
       uint32_t amax = 0;
+      if (BF16) {
+        amax = pmax[u];
+      } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        amax = max(amax, __float_as_uint(v[u][j]) & 0x7FFFFFFFu);
+        for (int j = 0; j < 8; ++j)
+          amax = max(amax, __float_as_uint(v[u][j]) & 0x7FFFFFFFu);
+      }
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
       const uint32_t sb = scale_byte(amax);
@@ -548,14 +554,12 @@ __global__ void __launch_bounds__(kDqThreads)
 // Row pass of one 1x32 group quarter (8 values of tile row tr, chunk ch):
 // returns the 4 code bytes; writes the row codes and scale to global memory
 // (when in range) and stages them in shared memory for the column pass.
-__device__ __forceinline__ void dq_row_chunk(float (&v)[8], bool ok, int64_t gr,
-                                             int64_t gc, int64_t cols, int tr,
-                                             int ch, uint8_t* __restrict__ row_codes,
+__device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool ok,
+                                             int64_t gr, int64_t gc, int64_t cols,
+                                             int tr, int ch,
+                                             uint8_t* __restrict__ row_codes,
                                              uint8_t* __restrict__ row_scales,
                                              uint32_t* s_codes, uint8_t* s_scales) {
-  uint32_t amax = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) amax = max(amax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   const uint32_t sb = scale_byte(amax);
@@ -616,7 +620,7 @@ __device__ __forceinline__ void dq_column_pass(
 // staged with asynchronous copies, so the next tile streams in while the
 // current one is quantized along rows and then along columns.
 template <bool BIG>
-__global__ void __launch_bounds__(kDqThreads, 2)
+__global__ void __launch_bounds__(kDqThreads, 3)
     k_double_quant_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
                         RngKey key, uint8_t* __restrict__ row_codes,
                         uint8_t* __restrict__ row_scales,
@@ -654,8 +658,8 @@ __global__ void __launch_bounds__(kDqThreads, 2)
       const uint4 w = raw[tr * (kDqCols / 8) + ch];
       float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
                     bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-      dq_row_chunk(v, gr < rows && gc < cols, gr, gc, cols, tr, ch, row_codes,
-                   row_scales, s_codes, s_scales);
+      dq_row_chunk(v, bf16x8_absmax(w), gr < rows && gc < cols, gr, gc, cols,
+                   tr, ch, row_codes, row_scales, s_codes, s_scales);
     }
     __syncthreads();
     dq_column_pass<BIG>(s_codes, s_scales, rg, cp, tile_r, tile_c, rows, cols,

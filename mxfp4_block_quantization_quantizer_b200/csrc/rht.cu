@@ -32,7 +32,7 @@ constexpr int kRhtRowsY = 32;   // rows per CTA step
 constexpr float kInvSqrt32 = 0.17677669529663687f;
 
 template <bool BF16, bool SR, bool ROT>
-__global__ void __launch_bounds__(kRhtThreads)
+__global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
     k_rht_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
                 uint32_t sign_key, RngKey key, uint8_t* __restrict__ codes,
                 uint8_t* __restrict__ scales, float* __restrict__ rotated) {
