@@ -47,6 +47,10 @@ OP_ELEMS = {k: SWEEP[0] * SWEEP[1] for k in BYTES_PER_ELEM}
 OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
 
 
+# Rows of SURVEY §8(f) built beyond the step, timed on their own.
+NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336))}
+
+
 def alg_bytes(op):
     return BYTES_PER_ELEM[op] * OP_ELEMS[op]
 
@@ -373,6 +377,31 @@ def run_ours(args):
         ev[op].append(a.elapsed_time(b))
     elapsed_ms = reduce_max(elapsed_ms, world, dev)
 
+    # next rows: Q-EMA on an fp32 master weight, timed alone
+    next_ops = {}
+    if not args.only:
+        qR, qC = NEXT_OPS["qema_quant"][1]
+        qw = torch.from_numpy(W.master_w(seed=7 + rank, rows=qR, cols=qC)).to(dev)
+        qe = torch.from_numpy(W.master_w(seed=8 + rank, rows=qR, cols=qC)).to(dev)
+        qout = (u8(qR, qC // 2), u8(qR, qC // 32))
+        for _ in range(args.warmup):
+            m.qema_quantize(qw, qe, 0.998, out=qout)
+        qev = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            m.qema_quantize(qw, qe, 0.998, out=qout)
+            b.record(stream)
+            qev.append((a, b))
+        torch.cuda.synchronize(dev)
+        d = statistics.mean(a.elapsed_time(b) for a, b in qev) * 1e-3
+        d = reduce_max(d, world, dev)
+        nbytes = NEXT_OPS["qema_quant"][0] * qR * qC
+        next_ops["qema_quant"] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9,
+                                  "bytes": nbytes, "shape": [qR, qC],
+                                  "launches": args.steps}
+        del qw, qe, qout
+
     # end to end: pinned host input -> device -> kernels -> host results
     if args.no_e2e:
         if rank == 0:
@@ -441,6 +470,7 @@ def run_ours(args):
             "e2e": {"value": job_gbs(world, STEP_BYTES, args.e2e_steps, e2e_ms),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
+            "next_ops": {k: dict(v, frac=v["GB_s"] / peak) for k, v in next_ops.items()},
             "gpu_launches": len(ops) * args.steps,
             "clocks": clocks,
         }

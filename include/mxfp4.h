@@ -179,6 +179,25 @@ mxfp4_status mxfp4_osc_synthetic_update(float* w, int64_t rows, int64_t cols,
                                         uint64_t seed, uint32_t step,
                                         float rel_step, void* stream);
 
+/*
+ * Q-EMA step fused with the forward quantization of the averaged weight:
+ * per element, in fp32 with no fused multiply-add,
+ *   w_ema = beta * w_ema + (1 - beta) * w        ((1 - beta) rounded first)
+ * then the new w_ema is block quantized along 1x32 row groups with RNE, as
+ * mxfp4_quantize(w_ema, F32, rows, cols, ROWS, RNE, ...).
+ * Source: "Oscillation-Reduced MXFP4 Training for Vision Transformers"
+ * rebuttal, Question 4 (an extra EMA weight per linear layer, quantized in
+ * the forward pass) and the hyper-parameter answers (beta in
+ * [0.997, 0.999], default 0.998).
+ *   w       device fp32 [rows][cols], the master weight, read only
+ *   w_ema   device fp32 [rows][cols], read and written
+ *   codes, scales  device, ROWS layout of the updated w_ema
+ * cols must be a multiple of 32.
+ */
+mxfp4_status mxfp4_qema_quantize(const float* w, float* w_ema, int64_t rows,
+                                 int64_t cols, float beta, uint8_t* codes,
+                                 uint8_t* scales, void* stream);
+
 /* Static text for a status code; never NULL. */
 const char* mxfp4_status_string(int status);
 

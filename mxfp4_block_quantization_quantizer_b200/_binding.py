@@ -21,7 +21,8 @@ RNE, SR = 0, 1
 # Every symbol include/mxfp4.h declares.
 SYMBOLS = ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_double_quantize",
            "mxfp4_rht_quantize", "mxfp4_osc_step",
-           "mxfp4_osc_synthetic_update", "mxfp4_status_string")
+           "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
+           "mxfp4_status_string")
 
 
 class Mxfp4Error(RuntimeError):
@@ -57,6 +58,8 @@ def lib():
                                vp, vp],
             "mxfp4_osc_synthetic_update": [vp, i64, i64, u64, u32,
                                            ctypes.c_float, vp],
+            "mxfp4_qema_quantize": [vp, vp, i64, i64, ctypes.c_float, vp, vp,
+                                    vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -200,6 +203,24 @@ def osc_synthetic_update(w, seed, step, rel_step=1e-4, stream=None):
            "mxfp4_osc_synthetic_update")
 
 
+def qema_quantize(w, w_ema, beta=0.998, out=None, stream=None):
+    """mxfp4_qema_quantize: update w_ema in place (fp32 CUDA tensors) and
+    return the ROWS-layout (codes, scales) of the new w_ema."""
+    for name, t in (("w", w), ("w_ema", w_ema)):
+        _cuda2d(t, name)
+        if t.dtype != torch.float32 or t.shape != w.shape:
+            raise TypeError("%s must be float32 with the shape of w" % name)
+    R, C = w.shape
+    if out is None:
+        out = (_empty_u8((R, C // 2), w.device), _empty_u8((R, C // 32), w.device))
+    codes, scales = out
+    _check(lib().mxfp4_qema_quantize(_ptr(w), _ptr(w_ema), R, C, beta,
+                                     _ptr(codes), _ptr(scales),
+                                     _stream(w.device, stream)),
+           "mxfp4_qema_quantize")
+    return codes, scales
+
+
 # The C names, for callers that prefer them.
 mxfp4_quantize = quantize
 mxfp4_dequantize = dequantize
@@ -207,4 +228,5 @@ mxfp4_double_quantize = double_quantize
 mxfp4_rht_quantize = rht_quantize
 mxfp4_osc_step = osc_step
 mxfp4_osc_synthetic_update = osc_synthetic_update
+mxfp4_qema_quantize = qema_quantize
 mxfp4_status_string = status_string

@@ -121,6 +121,17 @@ mxfp4_status mxfp4_osc_synthetic_update(float* w, int64_t rows, int64_t cols,
                                             rel_step, as_stream(stream)));
 }
 
+mxfp4_status mxfp4_qema_quantize(const float* w, float* w_ema, int64_t rows,
+                                 int64_t cols, float beta, uint8_t* codes,
+                                 uint8_t* scales, void* stream) {
+  if (!w || !w_ema || !codes || !scales) return MXFP4_ERR_NULL;
+  if (!dims_ok(rows, cols) || cols % 32) return MXFP4_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(w_ema) || !aligned16(codes))
+    return MXFP4_ERR_ALIGN;
+  return from_cuda(mxfp4::launch_qema_quant(w, w_ema, rows, cols, beta,
+                                            codes, scales, as_stream(stream)));
+}
+
 const char* mxfp4_status_string(int status) {
   switch (status) {
     case MXFP4_OK: return "ok";

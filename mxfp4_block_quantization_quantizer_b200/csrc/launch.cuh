@@ -42,6 +42,10 @@ cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                             float threshold, unsigned long long* n_flagged,
                             cudaStream_t s);
 
+cudaError_t launch_qema_quant(const float* w, float* w_ema, int64_t rows,
+                              int64_t cols, float beta, uint8_t* codes,
+                              uint8_t* scales, cudaStream_t s);
+
 cudaError_t launch_osc_update(float* w, int64_t n, uint64_t seed,
                               uint32_t step, float rel_step, cudaStream_t s);
 

@@ -15,6 +15,7 @@ Workloads (rows x cols):
             1x32 group has a known largest magnitude in [2^-4, 2^-3) and 25%
             of the other entries sit within 1e-3 relative of a rounding edge.
   sweep     8192 x 28672 bf16: N(0,1) with 0.1% of entries x100.
+  master_w  4096 x 14336 fp32 LLM master weight N(0, 0.02) (Q-EMA).
 """
 import numpy as np
 import ml_dtypes
@@ -28,6 +29,7 @@ SHAPES = {
     "llm_w": (4096, 14336),
     "osc_w": (4096, 4096),
     "sweep": (8192, 28672),
+    "master_w": (4096, 14336),
 }
 
 
@@ -111,6 +113,13 @@ def osc_w(seed=3, rows=4096, cols=4096, edge_frac=0.25, rel=1e-3):
     return w.astype(np.float32).reshape(rows, cols)
 
 
+def master_w(seed=7, rows=4096, cols=14336):
+    """fp32 master weight of an LLM linear layer: N(0, 0.02) (the Q-EMA
+    workload pairs it with an EMA state drawn the same way, seed + 1)."""
+    g = _rng(seed)
+    return g.normal(0.0, 0.02, size=(rows, cols)).astype(np.float32)
+
+
 def sweep(seed=5, rows=8192, cols=28672):
     return normal_bf16(rows, cols, seed, 0.001, 100.0)
 
@@ -118,5 +127,5 @@ def sweep(seed=5, rows=8192, cols=28672):
 def tensor(name, seed=None):
     """The named workload tensor (numpy, bf16 or fp32)."""
     fn = {"small": small, "deit_act": deit_act, "llm_w": llm_w,
-          "osc_w": osc_w, "sweep": sweep}[name]
+          "osc_w": osc_w, "sweep": sweep, "master_w": master_w}[name]
     return fn() if seed is None else fn(seed)

@@ -75,6 +75,8 @@ def _declare(L):
                          i64),
         "orc_osc_synthetic_update": ([_fp, i64, i64, i64, u64, u32,
                                       ctypes.c_float], i32),
+        "orc_qema_quantize": ([_fp, _fp, i64, i64, ctypes.c_float, _u8p,
+                               _u8p], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -216,6 +218,20 @@ class Oracle:
         R, C = w.shape
         self.L.orc_osc_synthetic_update(_f32(w), R, C, row0, seed, step,
                                         rel_step)
+
+
+    def qema_quantize(self, w, w_ema, beta=0.998):
+        """Q-EMA: update w_ema in place, return its 1x32 RNE (codes, scales)."""
+        for a in (w, w_ema):
+            if a.dtype != np.float32 or not a.flags.c_contiguous:
+                raise TypeError("Q-EMA arrays must be contiguous float32")
+        R, C = w.shape
+        codes = np.zeros(R * C // 2, np.uint8)
+        scales = np.zeros(R * C // 32, np.uint8)
+        if self.L.orc_qema_quantize(_f32(w), _f32(w_ema), R, C, beta,
+                                    _u8(codes), _u8(scales)):
+            raise ValueError("bad shape for the oracle Q-EMA")
+        return codes.reshape(R, C // 2), scales.reshape(R, C // 32)
 
 
 _default = None

@@ -482,3 +482,25 @@ void orc_rand16_range(uint64_t seed, uint32_t stream, uint64_t first,
   for (int64_t k = 0; k < n; ++k)
     out[k] = orc_rand16(seed, stream, first + (uint64_t)k);
 }
+
+/* ------------------------------------------------------------------ */
+/* Q-EMA ([TJ] rebuttal, Question 4 and the hyper-parameter answers:   */
+/* the forward pass quantizes an exponential moving average of the     */
+/* weight, updated whenever the parameters are; beta around 0.998)     */
+/* ------------------------------------------------------------------ */
+
+/* w_ema = beta * w_ema + (1 - beta) * w per element, each product and the
+ * sum rounded to fp32 (no fused multiply-add; 1 - beta itself rounded to
+ * fp32 first), then the 1x32 RNE quantization of the new w_ema. */
+int orc_qema_quantize(const float* w, float* w_ema, int64_t rows, int64_t cols,
+                      float beta, uint8_t* codes, uint8_t* scales) {
+  if (rows <= 0 || cols <= 0 || cols % 32) return -1;
+  const float omb = (float)(1.0 - (double)beta);
+  for (int64_t i = 0; i < rows * cols; ++i) {
+    float keep = (float)((double)beta * (double)w_ema[i]);
+    float take = (float)((double)omb * (double)w[i]);
+    w_ema[i] = (float)((double)keep + (double)take);
+  }
+  return orc_quantize(w_ema, DT_F32, rows, cols, 0, AX_ROWS, RND_RNE, 0,
+                      codes, scales);
+}

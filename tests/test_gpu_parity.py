@@ -430,3 +430,35 @@ def test_c_abi_statuses_on_device_pointers():
     assert L.mxfp4_quantize(p(x, 2), 1, 64, 64, 0, 0, 0, p(c), p(s), None) == 3
     assert L.mxfp4_quantize(p(x), 1, 64, 64, 0, 0, 0, p(c, 4), p(s), None) == 3
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------------------
+# Q-EMA: EMA update fused with 1x32 RNE quantization
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(1, 32), (37, 96), (256, 512)])
+@pytest.mark.parametrize("beta", [0.998, 0.9, 0.0, 1.0])
+def test_qema_steps(shape, beta):
+    g = np.random.Generator(np.random.PCG64(shape[0] + 7))
+    w_np = g.normal(0, 0.02, size=shape).astype(np.float32)
+    e_np = g.normal(0, 0.02, size=shape).astype(np.float32)
+    w, e = to_dev(w_np), to_dev(e_np)
+    for step in range(5):
+        c, s = m.qema_quantize(w, e, beta)
+        oc, os_ = O.qema_quantize(w_np, e_np, beta)
+        assert_bits_equal(to_np(e), e_np, "ema step %d" % step)
+        assert_bits_equal(to_np(c), oc, "codes step %d" % step)
+        assert_bits_equal(to_np(s), os_, "scales step %d" % step)
+        w_np = (w_np * np.float32(1.01)).astype(np.float32)
+        w = to_dev(w_np)
+
+
+def test_qema_edge_groups():
+    x = edge_tensor("f32")
+    e = np.zeros_like(x)
+    got_e = to_dev(e)
+    c, s = m.qema_quantize(to_dev(x), got_e, 0.5)
+    oc, os_ = O.qema_quantize(x, e, 0.5)
+    assert_f32_equal_or_both_nan(to_np(got_e), e, "ema")
+    assert_bits_equal(to_np(c), oc, "codes")
+    assert_bits_equal(to_np(s), os_, "scales")

@@ -170,3 +170,19 @@ def test_beyond_2_pow_33_elements():
         del out
     del xd
     torch.cuda.empty_cache()
+
+
+def test_master_weight_qema_sampled_bands():
+    w_np = W.master_w(seed=7)                 # 4096 x 14336 fp32
+    e_np = W.master_w(seed=8)
+    w, e = to_dev(w_np), to_dev(e_np)
+    for _ in range(3):
+        c, s = m.qema_quantize(w, e, 0.998)
+    c, s, e_got = to_np(c), to_np(s), to_np(e)
+    for r0 in (0, 2048, 4064):
+        band_w, band_e = w_np[r0:r0 + 32].copy(), e_np[r0:r0 + 32].copy()
+        for _ in range(3):
+            oc, os_ = O.qema_quantize(band_w, band_e, 0.998)
+        assert_bits_equal(e_got[r0:r0 + 32], band_e, "ema band %d" % r0)
+        assert_bits_equal(c[r0:r0 + 32], oc, "codes band %d" % r0)
+        assert_bits_equal(s[r0:r0 + 32], os_, "scales band %d" % r0)

@@ -74,13 +74,17 @@ MUTANTS = [
      ["test_osc_worked_example_from_the_page"]),
     ("no reset at window end", "      d_w[i] = 0.0f;\n", "",
      ["test_osc_accumulators_before_window_end"]),
+    ("EMA weights swapped", "float keep = (float)((double)beta * (double)w_ema[i]);",
+     "float keep = (float)((double)omb * (double)w_ema[i]);",
+     ["test_qema_matches_the_geometric_closed_form"]),
     ("update sign bit", "(orc_counter_hash(k, gi) >> 31)",
      "(orc_counter_hash(k, gi) >> 30)",
      ["test_osc_synthetic_update_magnitude_and_signs"]),
 ]
 
 PARAMS = {"test_tiny_tensors_brute_force_layout": [((32, 96), O.COLS),
-                                                   ((64, 96), O.ROWS)]}
+                                                   ((64, 96), O.ROWS)],
+          "test_qema_matches_the_geometric_closed_form": [(0.9, 200, 40)]}
 
 
 def _build(tmp_path, name, src_text):

@@ -543,3 +543,45 @@ def test_osc_synthetic_update_magnitude_and_signs():
     assert np.array_equal(w1, w)
     O.osc_synthetic_update(w1, 3, 8, 1e-4)
     assert not np.array_equal(w1, w)
+
+
+# --------------------------------------------------------------------------
+# Q-EMA (TetraJet rebuttal, Question 4: quantize an EMA of the weight)
+# --------------------------------------------------------------------------
+
+def test_qema_special_betas():
+    g = np.random.Generator(np.random.PCG64(31))
+    w = g.normal(0, 0.02, size=(8, 64)).astype(np.float32)
+    ema0 = g.normal(0, 0.02, size=(8, 64)).astype(np.float32)
+    e = ema0.copy()
+    O.qema_quantize(w, e, 0.0)
+    assert np.array_equal(e, w)  # beta 0: the EMA is the weight
+    e = ema0.copy()
+    O.qema_quantize(w, e, 1.0)
+    assert np.array_equal(e, ema0)  # beta 1: the EMA never moves
+
+
+@pytest.mark.parametrize("beta,steps,ulps", [(0.9, 200, 40), (0.998, 600, 2500)])
+def test_qema_matches_the_geometric_closed_form(beta, steps, ulps):
+    """A constant weight w: ema_n = w + (ema_0 - w) * beta^n exactly; the
+    fp32 recurrence stays within a bound of accumulated roundings
+    (each step adds at most ~1.5 ulp, damped by beta)."""
+    g = np.random.Generator(np.random.PCG64(32))
+    w = g.normal(0, 0.02, size=(4, 32)).astype(np.float32)
+    e = g.normal(0, 0.02, size=(4, 32)).astype(np.float32)
+    e0 = e.astype(np.float64)
+    for _ in range(steps):
+        O.qema_quantize(w, e, beta)
+    b = float(np.float32(beta))
+    want = w.astype(np.float64) + (e0 - w) * b ** steps
+    scale = np.maximum(np.abs(w), np.abs(e0)).astype(np.float32)
+    assert np.all(np.abs(e - want) <= ulps * np.spacing(scale))
+
+
+def test_qema_codes_are_the_quantized_ema():
+    g = np.random.Generator(np.random.PCG64(33))
+    w = g.normal(0, 0.02, size=(16, 96)).astype(np.float32)
+    e = g.normal(0, 0.02, size=(16, 96)).astype(np.float32)
+    c, s = O.qema_quantize(w, e, 0.998)
+    c2, s2 = O.quantize(e, O.ROWS, O.RNE)
+    assert np.array_equal(c, c2) and np.array_equal(s, s2)
