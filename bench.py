@@ -121,7 +121,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default="",
@@ -305,17 +305,28 @@ def run_ours(args):
     R, C = args.rows, SWEEP[1]
     x_np = W.sweep(seed=rank_seed(rank), rows=R)
     w_np = W.osc_w(seed=3 + rank)
-    x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
-    w0 = torch.from_numpy(w_np).to(dev)
     u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)  # noqa: E731
-    rows_out = (u8(R, C // 2), u8(R, C // 32))
-    cols_out = (u8(C, R // 2), u8(C, R // 32))
-    dq_out = (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32))
-    rht_out = (u8(R, C // 2), u8(R, C // 32), None)
-    y = torch.empty(R, C, dtype=torch.bfloat16, device=dev)
-    w = w0.clone()
-    ws, dwt, dqt = w.clone(), torch.zeros_like(w), torch.zeros_like(w)
-    nflag = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    def buffers():
+        """Device inputs and outputs of one step (the e2e loop uses two)."""
+        return {
+            "x": torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev),
+            "w": torch.from_numpy(w_np).to(dev),
+            "rows": (u8(R, C // 2), u8(R, C // 32)),
+            "cols": (u8(C, R // 2), u8(C, R // 32)),
+            "dq": (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32)),
+            "rht": (u8(R, C // 2), u8(R, C // 32), None),
+            "y": torch.empty(R, C, dtype=torch.bfloat16, device=dev),
+            "nflag": torch.zeros(1, dtype=torch.int64, device=dev),
+        }
+
+    def outputs(b):
+        return [*b["rows"], *b["cols"], *b["dq"], b["y"], b["rht"][0],
+                b["rht"][1], b["w"], b["nflag"]]
+
+    buf0 = buffers()
+    # tracker state (stays on the device across steps)
+    ws, dwt, dqt = buf0["w"].clone(), torch.zeros_like(buf0["w"]), torch.zeros_like(buf0["w"])
 
     ops = [o for o in BYTES_PER_ELEM if not args.only or o in args.only.split(",")]
     if (R, C) != SWEEP:
@@ -326,31 +337,33 @@ def run_ours(args):
     ev = {op: [] for op in ops}
     step_no = [0]
 
-    def step(record):
+    def step(record, b=buf0):
         t = step_no[0]
         step_no[0] += 1
         pairs = []
+        cur = torch.cuda.current_stream(dev)
 
         def timed(op, fn):
             if op not in ops:
                 return
             if record:
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(cur)
                 fn()
-                b.record(stream)
-                pairs.append((op, a, b))
+                e1.record(cur)
+                pairs.append((op, e0, e1))
             else:
                 fn()
 
-        timed("quant_rows_rne", lambda: m.quantize(x, m.ROWS, m.RNE, 0, out=rows_out))
-        timed("quant_cols_sr", lambda: m.quantize(x, m.COLS, m.SR, SEED, out=cols_out))
-        timed("double_quant", lambda: m.double_quantize(x, SEED, out=dq_out))
-        timed("dequant_rows", lambda: m.dequantize(rows_out[0], rows_out[1], R, C, out=y))
-        timed("rht_quant_sr", lambda: m.rht_quantize(x, 2, m.SR, SEED, out=rht_out))
+        x, w = b["x"], b["w"]
+        timed("quant_rows_rne", lambda: m.quantize(x, m.ROWS, m.RNE, 0, out=b["rows"]))
+        timed("quant_cols_sr", lambda: m.quantize(x, m.COLS, m.SR, SEED, out=b["cols"]))
+        timed("double_quant", lambda: m.double_quantize(x, SEED, out=b["dq"]))
+        timed("dequant_rows", lambda: m.dequantize(b["rows"][0], b["rows"][1], R, C, out=b["y"]))
+        timed("rht_quant_sr", lambda: m.rht_quantize(x, 2, m.SR, SEED, out=b["rht"]))
         timed("osc_update", lambda: m.osc_synthetic_update(w, 3, t % 200))
         timed("osc_step", lambda: m.osc_step(w, ws, dwt, dqt, window_end=(t % 200 == 199),
-                                             n_flagged=nflag))
+                                             n_flagged=b["nflag"]))
         return pairs
 
     for _ in range(args.warmup):
@@ -410,31 +423,53 @@ def run_ours(args):
         if world > 1:
             dist.destroy_process_group()
         return
+    # Double-buffered: step t's uploads, kernels and downloads run on three
+    # streams, so the uploads of step t+1 and the downloads of step t-1
+    # overlap step t (PCIe moves both directions at once).
     x_host = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     w_host = torch.from_numpy(w_np).pin_memory()
-    outs = [rows_out[0], rows_out[1], cols_out[0], cols_out[1], *dq_out, y,
-            rht_out[0], rht_out[1], w, nflag]
-    host_outs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    bufs = [buf0, buffers()]
+    host_outs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outputs(buf0)]
     h2d = x_host.numel() * 2 + w_host.numel() * 4
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    for _ in range(1):
-        x.copy_(x_host, non_blocking=True)
-        w.copy_(w_host, non_blocking=True)
-        step(False)
-        for h, o in zip(host_outs, outs):
-            h.copy_(o, non_blocking=True)
+    d2h = sum(o.numel() * o.element_size() for o in outputs(buf0))
+    s_up, s_run, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_run = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
+    for e in ev_run + ev_down:
+        e.record(stream)
+
+    def e2e_step(t):
+        k = t % 2
+        b = bufs[k]
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(ev_run[k])    # step t-2 finished reading x
+            s_up.wait_event(ev_down[k])   # and its w went out
+            b["x"].copy_(x_host, non_blocking=True)
+            b["w"].copy_(w_host, non_blocking=True)
+            ev_up[k].record(s_up)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev_up[k])
+            s_run.wait_event(ev_down[k])  # step t-2's outputs are out
+            step(False, b)
+            ev_run[k].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev_run[k])
+            for h, o in zip(host_outs, outputs(b)):
+                h.copy_(o, non_blocking=True)
+            ev_down[k].record(s_down)
+
+    for t in range(2):
+        e2e_step(t)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(args.e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        w.copy_(w_host, non_blocking=True)
-        step(False)
-        for h, o in zip(host_outs, outs):
-            h.copy_(o, non_blocking=True)
-    e_end.record(stream)
+    e_start.record(s_up)
+    for t in range(args.e2e_steps):
+        e2e_step(t)
+    s_up.wait_stream(s_down)
+    e_end.record(s_up)
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_end)
     e2e_ms = reduce_max(e2e_ms, world, dev)
