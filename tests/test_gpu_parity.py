@@ -462,3 +462,56 @@ def test_qema_edge_groups():
     assert_f32_equal_or_both_nan(to_np(got_e), e, "ema")
     assert_bits_equal(to_np(c), oc, "codes")
     assert_bits_equal(to_np(s), os_, "scales")
+
+
+# ---------------------------------------------------------------------------
+# Graph capture and concurrent streams
+# ---------------------------------------------------------------------------
+
+def test_calls_replay_from_a_cuda_graph():
+    """The entry points allocate nothing and only launch kernels on the
+    caller's stream, so a captured sequence replays to the same results."""
+    x_np = rand_tensor((256, 512), "bf16", 41)
+    x = to_dev(x_np)
+    R, C = x.shape
+    u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device="cuda")  # noqa: E731
+    rows = (u8(R, C // 2), u8(R, C // 32))
+    dq = (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32))
+    y = torch.empty(R, C, dtype=torch.bfloat16, device="cuda")
+    # warm up outside capture (first calls set kernel attributes)
+    m.quantize(x, m.ROWS, m.SR, 3, out=rows)
+    m.double_quantize(x, 4, out=dq)
+    m.dequantize(rows[0], rows[1], R, C, out=y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.quantize(x, m.ROWS, m.SR, 3, out=rows)
+        m.double_quantize(x, 4, out=dq)
+        m.dequantize(rows[0], rows[1], R, C, out=y)
+    for t in rows + dq:
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    oc, os_ = O.quantize(x_np, O.ROWS, O.SR, 3)
+    assert_bits_equal(to_np(rows[0]), oc, "graph row codes")
+    for got, want in zip(dq, O.double_quantize(x_np, 4)):
+        assert_bits_equal(to_np(got), want, "graph double quantization")
+    assert_bits_equal(to_np(y), O.dequantize(oc, os_, R, C), "graph dequantize")
+
+
+def test_two_streams_at_once():
+    a_np = rand_tensor((512, 1024), "bf16", 42)
+    b_np = rand_tensor((512, 1024), "bf16", 43)
+    a, b = to_dev(a_np), to_dev(b_np)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    s1.wait_stream(torch.cuda.current_stream())
+    s2.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s1):
+        ra = m.double_quantize(a, seed=9)
+    with torch.cuda.stream(s2):
+        rb = m.double_quantize(b, seed=9)
+    torch.cuda.synchronize()
+    for got, want in zip(ra, O.double_quantize(a_np, 9)):
+        assert_bits_equal(to_np(got), want, "stream 1")
+    for got, want in zip(rb, O.double_quantize(b_np, 9)):
+        assert_bits_equal(to_np(got), want, "stream 2")
