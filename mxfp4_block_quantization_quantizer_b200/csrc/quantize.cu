@@ -693,7 +693,7 @@ template <bool BF16, bool SR>
 static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
-  constexpr int U = BF16 ? 4 : 2;
+  constexpr int U = BF16 ? 4 : 2;  // 8 lowers occupancy and runs slower
   auto kern = k_quant_rows<BF16, SR, U>;
   const int64_t groups_per_block = (kRowThreads / 4) * U;
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
@@ -778,7 +778,7 @@ cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
                            int64_t n_groups, void* y, bool bf16_out,
                            cudaStream_t s) {
-  constexpr int U = 4;
+  constexpr int U = 8;
   const int64_t groups_per_block = (kRowThreads / 4) * U;
   const int64_t blocks = (n_groups + groups_per_block - 1) / groups_per_block;
   if (bf16_out) {
