@@ -47,7 +47,7 @@ OP_ELEMS = {k: SWEEP[0] * SWEEP[1] for k in BYTES_PER_ELEM}
 OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
 
 
-# Rows of SURVEY §8(f) built beyond the step, timed on their own.
+# Further operations built beyond the step (Q-EMA), timed on their own.
 NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336))}
 
 
@@ -190,6 +190,45 @@ def cpu_baseline_sample(x_np, w_np, max_seconds=20.0):
                       "of the tracker (update + step); single thread, %.1f s"
                       % (reps, dt),
             "gelem_s": total_e / dt / 1e9}
+
+
+def _oracle_band_worker(args):
+    """One process's share of the all-cores baseline: the sample step on its
+    own 32-row band, repeated `reps` times. Returns (bytes, elements, s)."""
+    x_band, w_band, reps = args
+    state = (w_band.copy(), w_band.copy(), np.zeros_like(w_band),
+             np.zeros_like(w_band))
+    t0 = time.perf_counter()
+    nb = ne = 0
+    for _ in range(reps):
+        b, e = cpu_sample_step(x_band, w_band, state, 0)
+        nb += b
+        ne += e
+    return nb, ne, time.perf_counter() - t0
+
+
+def cpu_baseline_all_cores(x_np, w_np, reps=8):
+    """The same oracle, row-block parallel over every host core (spawned
+    processes, one 32-row band each): whole-job bytes over wall time."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    cores = os.cpu_count() or 1
+    bands = [(np.ascontiguousarray(x_np[32 * (i % (x_np.shape[0] // 32)):][:32]),
+              np.ascontiguousarray(w_np[:16]), reps) for i in range(cores)]
+    warm = [(b[0], b[1], 1) for b in bands]
+    # spawn (never fork after CUDA); a dead worker raises instead of hanging
+    with ProcessPoolExecutor(cores, mp_context=mp.get_context("spawn")) as ex:
+        list(ex.map(_oracle_band_worker, warm, timeout=300))  # start-up
+        t0 = time.perf_counter()
+        res = list(ex.map(_oracle_band_worker, bands, timeout=600))
+        dt = time.perf_counter() - t0
+    nb = sum(r[0] for r in res)
+    ne = sum(r[1] for r in res)
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": "%d processes x %d reps of the one-band sample step "
+                      "(each its own 32x28672 band), %.1f s wall" % (cores, reps, dt),
+            "gelem_s": ne / dt / 1e9}
 
 
 def run_reference(args):
@@ -390,7 +429,7 @@ def run_ours(args):
         ev[op].append(a.elapsed_time(b))
     elapsed_ms = reduce_max(elapsed_ms, world, dev)
 
-    # next rows: Q-EMA on an fp32 master weight, timed alone
+    # further operations: Q-EMA on an fp32 master weight, timed alone
     next_ops = {}
     if not args.only:
         qR, qC = NEXT_OPS["qema_quant"][1]
@@ -511,6 +550,7 @@ def run_ours(args):
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline_sample(x_np, w_np)
+            line["cpu_baseline_all_cores"] = cpu_baseline_all_cores(x_np, w_np)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
