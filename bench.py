@@ -458,7 +458,10 @@ def run_ours(args):
     if args.no_e2e:
         if rank == 0:
             print(json.dumps({"profile_run": True, "ops": ops,
-                              "ms": elapsed_ms / args.steps}), flush=True)
+                              "ms": elapsed_ms / args.steps,
+                              "ops_us": {op: 1e3 * statistics.mean(ev[op])
+                                         for op in ops},
+                              "next_ops": next_ops}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return

@@ -282,6 +282,17 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// 16-byte read-only load that allocates in L1: for threads that read 32 or
+// more contiguous bytes in 16-byte steps, where one warp instruction covers
+// only half of each 32-byte sector and the next instruction the other half.
+__device__ __forceinline__ uint4 ld_l1(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
 constexpr uint32_t kNaNbf16x2 = 0x7FC07FC0u;
 constexpr uint32_t kNaNf32 = 0x7FC00000u;
 

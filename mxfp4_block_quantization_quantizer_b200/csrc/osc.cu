@@ -26,7 +26,7 @@ namespace {
 constexpr int kOscThreads = 256;
 
 __device__ __forceinline__ void load8(const float* p, float* v) {
-  const uint4 a = ld_stream(p), b = ld_stream(p + 4);
+  const uint4 a = ld_l1(p), b = ld_l1(p + 4);
   v[0] = __uint_as_float(a.x), v[1] = __uint_as_float(a.y);
   v[2] = __uint_as_float(a.z), v[3] = __uint_as_float(a.w);
   v[4] = __uint_as_float(b.x), v[5] = __uint_as_float(b.y);

@@ -35,8 +35,8 @@ __global__ void __launch_bounds__(kQemaThreads)
     const int64_t g = base + my;
     const bool ok = g < n_groups;
     const int64_t e = (ok ? g : 0) * 32 + sub * 8;
-    const uint4 w0 = ld_stream(w + e), w1 = ld_stream(w + e + 4);
-    const uint4 m0 = ld_stream(w_ema + e), m1 = ld_stream(w_ema + e + 4);
+    const uint4 w0 = ld_l1(w + e), w1 = ld_l1(w + e + 4);
+    const uint4 m0 = ld_l1(w_ema + e), m1 = ld_l1(w_ema + e + 4);
     const uint32_t wb[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
     const uint32_t mb[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
     float v[8];

@@ -154,18 +154,27 @@ __device__ __forceinline__ void column_noise(RngKey key, uint64_t i0,
   }
 }
 
+// Codes and scale bytes of two adjacent columns over one 32-row group: wa/wb
+// hold the 32 codes of each column (row r0+j in nibble j%8 of word j/8).
+struct ColPair {
+  uint32_t wa[4], wb[4];
+  uint32_t sa, sb;
+};
+
 // Quantize the two adjacent columns c0, c0+1 over the 32 rows r0 .. r0+31.
 // get(j) returns the values of row r0+j (x: column c0, y: column c0+1); ma
 // and mb are the fp32 bit patterns of the two columns' absolute maxima.
-// Codes go to the COLS layout.
 template <bool SR, bool EVEN, bool BIG, typename Get>
-__device__ __forceinline__ void column_pair_quant(
-    Get get, uint32_t ma, uint32_t mb, int64_t r0, int64_t c0, int64_t rows,
-    int64_t cols, RngKey key, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales) {
-  const uint32_t sa = scale_byte(ma), sbb = scale_byte(mb);
-  const float mula = inv_scale(sa), mulb = inv_scale(sbb);
-  uint32_t wa[4] = {0, 0, 0, 0}, wb[4] = {0, 0, 0, 0};
+__device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
+                                                     uint32_t mb, int64_t r0,
+                                                     int64_t c0, int64_t cols,
+                                                     RngKey key) {
+  ColPair o;
+  o.sa = scale_byte(ma);
+  o.sb = scale_byte(mb);
+  const float mula = inv_scale(o.sa), mulb = inv_scale(o.sb);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) o.wa[q] = o.wb[q] = 0;
   if (SR) {
     const uint64_t i0 = uint64_t(r0) * uint64_t(cols) + uint64_t(c0);
 #pragma unroll
@@ -173,8 +182,8 @@ __device__ __forceinline__ void column_pair_quant(
       uint32_t na, nb;
       column_noise<EVEN, BIG>(key, i0, cols, j, na, nb);
       const float2 v = get(j);
-      wa[j >> 3] += e2m1_sr(v.x * mula, na) * (1u << (4 * (j & 7)));
-      wb[j >> 3] += e2m1_sr(v.y * mulb, nb) * (1u << (4 * (j & 7)));
+      o.wa[j >> 3] += e2m1_sr(v.x * mula, na) * (1u << (4 * (j & 7)));
+      o.wb[j >> 3] += e2m1_sr(v.y * mulb, nb) * (1u << (4 * (j & 7)));
     }
   } else {
 #pragma unroll
@@ -186,36 +195,98 @@ __device__ __forceinline__ void column_pair_quant(
         va[j] = v.x * mula;
         vb[j] = v.y * mulb;
       }
-      wa[q] = e2m1x8_rn(va);
-      wb[q] = e2m1x8_rn(vb);
+      o.wa[q] = e2m1x8_rn(va);
+      o.wb[q] = e2m1x8_rn(vb);
     }
   }
-  if (sa == 0xFFu) wa[0] = wa[1] = wa[2] = wa[3] = 0;
-  if (sbb == 0xFFu) wb[0] = wb[1] = wb[2] = wb[3] = 0;
+  if (o.sa == 0xFFu) o.wa[0] = o.wa[1] = o.wa[2] = o.wa[3] = 0;
+  if (o.sb == 0xFFu) o.wb[0] = o.wb[1] = o.wb[2] = o.wb[3] = 0;
+  return o;
+}
+
+// Store a column pair straight to the COLS layout (16 bytes per column).
+__device__ __forceinline__ void store_column_pair(
+    const ColPair& o, int64_t r0, int64_t c0, int64_t rows, int64_t cols,
+    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int64_t half_rows = rows / 2;
   if (c0 < cols) {
     *reinterpret_cast<uint4*>(codes + c0 * half_rows + r0 / 2) =
-        make_uint4(wa[0], wa[1], wa[2], wa[3]);
-    scales[c0 * (rows / 32) + r0 / 32] = static_cast<uint8_t>(sa);
+        make_uint4(o.wa[0], o.wa[1], o.wa[2], o.wa[3]);
+    scales[c0 * (rows / 32) + r0 / 32] = static_cast<uint8_t>(o.sa);
   }
   if (c0 + 1 < cols) {
     *reinterpret_cast<uint4*>(codes + (c0 + 1) * half_rows + r0 / 2) =
-        make_uint4(wb[0], wb[1], wb[2], wb[3]);
-    scales[(c0 + 1) * (rows / 32) + r0 / 32] = static_cast<uint8_t>(sbb);
+        make_uint4(o.wb[0], o.wb[1], o.wb[2], o.wb[3]);
+    scales[(c0 + 1) * (rows / 32) + r0 / 32] = static_cast<uint8_t>(o.sb);
+  }
+}
+
+// Column outputs of one 128-row tile, staged in shared memory so that each
+// column's 64-byte run of codes leaves in one piece: the 16-byte chunk of
+// column pair cp, side s (0: even column), row group rg sits at uint4 index
+// 9cp + 4s + rg (the ninth chunk of each pair is padding, so the stores of
+// consecutive cp fall in distinct bank groups); scale bytes at 4c + rg for
+// tile column c.
+template <int kCols>
+struct ColStage {
+  static constexpr int kChunks = (kCols / 2) * 9;
+  static constexpr int kBytes = kChunks * 16 + kCols * 4;
+};
+
+__device__ __forceinline__ void stage_column_pair(const ColPair& o, int cp,
+                                                  int rg, uint4* s_col,
+                                                  uint8_t* s_sc) {
+  s_col[9 * cp + rg] = make_uint4(o.wa[0], o.wa[1], o.wa[2], o.wa[3]);
+  s_col[9 * cp + 4 + rg] = make_uint4(o.wb[0], o.wb[1], o.wb[2], o.wb[3]);
+  s_sc[8 * cp + rg] = static_cast<uint8_t>(o.sa);
+  s_sc[8 * cp + 4 + rg] = static_cast<uint8_t>(o.sb);
+}
+
+// Write a staged tile to the COLS layout: four consecutive threads write one
+// column's 64 contiguous code bytes, and one thread its 4 scale bytes (one
+// 32-bit store when rows is a multiple of 128, which also aligns it).
+template <int kCols, int kThreads>
+__device__ __forceinline__ void store_staged_columns(
+    const uint4* s_col, const uint8_t* s_sc, int64_t tile_r, int64_t tile_c,
+    int64_t rows, int64_t cols, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales) {
+  static_assert(kCols * 4 % kThreads == 0 && kCols <= kThreads, "stage shape");
+  const int64_t half_rows = rows / 2, groups = rows / 32;
+#pragma unroll
+  for (int i = 0; i < kCols * 4 / kThreads; ++i) {
+    const int k = i * kThreads + threadIdx.x;
+    const int cp = k >> 3, side = (k >> 2) & 1, part = k & 3;
+    const int64_t c = tile_c + 2 * cp + side, r = tile_r + 32 * part;
+    if (c < cols && r < rows)
+      *reinterpret_cast<uint4*>(codes + c * half_rows + r / 2) =
+          s_col[9 * cp + 4 * side + part];
+  }
+  const int k = threadIdx.x;
+  const int64_t c = tile_c + k;
+  if (k < kCols && c < cols) {
+    uint8_t* dst = scales + c * groups + tile_r / 32;
+    if (rows % kTileRows == 0) {
+      *reinterpret_cast<uint32_t*>(dst) = reinterpret_cast<const uint32_t*>(s_sc)[k];
+    } else {
+#pragma unroll
+      for (int part = 0; part < 4; ++part)
+        if (tile_r + 32 * part < rows) dst[part] = s_sc[4 * k + part];
+    }
   }
 }
 
 // Column pass over a staged tile: thread (rg, cp) quantizes the columns
-// 2cp, 2cp+1 over tile rows 32rg .. 32rg+31. The tile is read twice (maxima,
+// 2cp, 2cp+1 over tile rows 32rg .. 32rg+31 (rows below the tensor's end:
+// the caller checks tile_r + 32rg < rows). The tile is read twice (maxima,
 // then codes) rather than held in registers. A warp reads 32 consecutive
 // 32-bit words (bf16) or 64-bit words (fp32) of one row: no bank conflicts.
 template <bool BF16, bool SR, bool EVEN, bool BIG>
-__device__ __forceinline__ void column_tile_pass(
-    const uint4* tile, int kcols, int rg, int cp, int64_t tile_r,
-    int64_t tile_c, int64_t rows, int64_t cols, RngKey key,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+__device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
+                                                    int kcols, int rg, int cp,
+                                                    int64_t tile_r,
+                                                    int64_t tile_c,
+                                                    int64_t cols, RngKey key) {
   const int64_t r0 = tile_r + 32 * rg;
-  if (r0 >= rows) return;
   uint32_t ma = 0, mb = 0;
   if (BF16) {
     const uint32_t* s = reinterpret_cast<const uint32_t*>(tile) + 32 * rg * (kcols / 2) + cp;
@@ -224,24 +295,22 @@ __device__ __forceinline__ void column_tile_pass(
     for (int j = 0; j < 32; ++j) m = umax16x2(m, s[j * (kcols / 2)] & 0x7FFF7FFFu);
     ma = m << 16;
     mb = m & 0xFFFF0000u;
-    column_pair_quant<SR, EVEN, BIG>(
+    return column_pair_codes<SR, EVEN, BIG>(
         [&](int j) {
           const uint32_t w = s[j * (kcols / 2)];
           return make_float2(bf16_lo(w), bf16_hi(w));
         },
-        ma, mb, r0, tile_c + 2 * cp, rows, cols, key, codes, scales);
-  } else {
-    const float2* s = reinterpret_cast<const float2*>(tile) + 32 * rg * (kcols / 2) + cp;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float2 w = s[j * (kcols / 2)];
-      ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
-      mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
-    }
-    column_pair_quant<SR, EVEN, BIG>([&](int j) { return s[j * (kcols / 2)]; },
-                                     ma, mb, r0, tile_c + 2 * cp, rows, cols,
-                                     key, codes, scales);
+        ma, mb, r0, tile_c + 2 * cp, cols, key);
   }
+  const float2* s = reinterpret_cast<const float2*>(tile) + 32 * rg * (kcols / 2) + cp;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float2 w = s[j * (kcols / 2)];
+    ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
+    mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
+  }
+  return column_pair_codes<SR, EVEN, BIG>([&](int j) { return s[j * (kcols / 2)]; },
+                                          ma, mb, r0, tile_c + 2 * cp, cols, key);
 }
 
 // Load one [128 x kCols] tile into shared memory (zero outside the tensor).
@@ -327,23 +396,29 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     const int64_t tile_c = (t % tiles_c) * T::kCols;
     load_tile<BF16, false>(x, rows, cols, tile_r, tile_c, tile);
     __syncthreads();
-    column_tile_pass<BF16, SR, EVEN, BIG>(tile, T::kCols, rg, cp, tile_r,
-                                          tile_c, rows, cols, key, codes,
-                                          scales);
+    const int64_t r0 = tile_r + 32 * rg;
+    if (r0 < rows)
+      store_column_pair(column_tile_pass<BF16, SR, EVEN, BIG>(
+                            tile, T::kCols, rg, cp, tile_r, tile_c, cols, key),
+                        r0, tile_c + 2 * cp, rows, cols, codes, scales);
     __syncthreads();
   }
 }
 
 // Column groups, 16-byte aligned rows: double-buffered. The copies of the
-// CTA's next tile are in flight while the current tile is quantized.
+// CTA's next tile are in flight while the current tile is quantized; the
+// tile's column codes are staged and leave as whole 64-byte runs.
 template <bool BF16, bool SR, bool EVEN, bool BIG>
 __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
     k_quant_cols_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
                       RngKey key, uint8_t* __restrict__ codes,
                       uint8_t* __restrict__ scales) {
   using T = ColTile<BF16>;
+  using S = ColStage<T::kCols>;
   constexpr int kChunks = kTileRows * T::kChunksPerRow;
-  extern __shared__ uint4 smem[];  // two tiles
+  extern __shared__ uint4 smem[];  // two tiles, then the column stage
+  uint4* s_col = smem + 2 * kChunks;
+  uint8_t* s_sc = reinterpret_cast<uint8_t*>(s_col + S::kChunks);
   const int64_t tiles_c = (cols + T::kCols - 1) / T::kCols;
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
   const int cp = threadIdx.x % (T::kCols / 2);
@@ -361,11 +436,17 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
       cp_async_commit();  // keep one group per iteration
     cp_async_wait<1>();   // this tile's copies (the older group) are done
     __syncthreads();
-    column_tile_pass<BF16, SR, EVEN, BIG>(smem + buf * kChunks, T::kCols, rg,
-                                          cp, (t / tiles_c) * kTileRows,
-                                          (t % tiles_c) * T::kCols, rows, cols,
-                                          key, codes, scales);
-    __syncthreads();  // the next iteration's copies overwrite this buffer
+    const int64_t tile_r = (t / tiles_c) * kTileRows;
+    const int64_t tile_c = (t % tiles_c) * T::kCols;
+    if (tile_r + 32 * rg < rows)
+      stage_column_pair(column_tile_pass<BF16, SR, EVEN, BIG>(
+                            smem + buf * kChunks, T::kCols, rg, cp, tile_r,
+                            tile_c, cols, key),
+                        cp, rg, s_col, s_sc);
+    __syncthreads();
+    store_staged_columns<T::kCols, T::kThreads>(s_col, s_sc, tile_r, tile_c,
+                                                rows, cols, codes, scales);
+    __syncthreads();  // the next copies and stage writes reuse the buffers
   }
   cp_async_wait<0>();
 }
@@ -543,9 +624,10 @@ __global__ void __launch_bounds__(kDqThreads)
         }
       }
       // cols is a multiple of 32 here, so every pair index is even-aligned
-      column_pair_quant<true, true, BIG>(
-          [&](int j) { return make_float2(a[j], b[j]); }, ma, mb, r0,
-          tile_c + 2 * cp, rows, cols, key, col_codes, col_scales);
+      store_column_pair(column_pair_codes<true, true, BIG>(
+                            [&](int j) { return make_float2(a[j], b[j]); }, ma,
+                            mb, r0, tile_c + 2 * cp, cols, key),
+                        r0, tile_c + 2 * cp, rows, cols, col_codes, col_scales);
     }
     __syncthreads();
   }
@@ -579,14 +661,13 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
 // Column pass of the double quantizer over the staged Q_D(X) codes: decode
 // columns 2cp, 2cp+1 of rows 32rg.. (one shared byte per row holds both
 // codes; a row group of scale 0xFF decodes to NaN as 0 x inf), then
-// stochastic rounding along the 32x1 groups.
+// stochastic rounding along the 32x1 groups. The caller checks that the row
+// group lies inside the tensor.
 template <bool BIG>
-__device__ __forceinline__ void dq_column_pass(
+__device__ __forceinline__ ColPair dq_column_pass(
     const uint32_t* s_codes, const uint8_t* s_scales, int rg, int cp,
-    int64_t tile_r, int64_t tile_c, int64_t rows, int64_t cols, RngKey key,
-    uint8_t* __restrict__ col_codes, uint8_t* __restrict__ col_scales) {
+    int64_t tile_r, int64_t tile_c, int64_t cols, RngKey key) {
   const int64_t r0 = tile_r + 32 * rg;
-  if (r0 >= rows) return;
   const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
   float a[32], b[32];
   uint32_t ma = 0, mb = 0;
@@ -611,14 +692,15 @@ __device__ __forceinline__ void dq_column_pass(
     }
   }
   // cols is a multiple of 32 here, so every pair index is even-aligned
-  column_pair_quant<true, true, BIG>(
+  return column_pair_codes<true, true, BIG>(
       [&](int j) { return make_float2(a[j], b[j]); }, ma, mb, r0,
-      tile_c + 2 * cp, rows, cols, key, col_codes, col_scales);
+      tile_c + 2 * cp, cols, key);
 }
 
 // Fused double quantization of bf16 X, double-buffered: the raw tiles are
 // staged with asynchronous copies, so the next tile streams in while the
-// current one is quantized along rows and then along columns.
+// current one is quantized along rows and then along columns. Once the row
+// pass is done the current raw tile is free and holds the column stage.
 template <bool BIG>
 __global__ void __launch_bounds__(kDqThreads, 3)
     k_double_quant_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
@@ -662,9 +744,17 @@ __global__ void __launch_bounds__(kDqThreads, 3)
                    tr, ch, row_codes, row_scales, s_codes, s_scales);
     }
     __syncthreads();
-    dq_column_pass<BIG>(s_codes, s_scales, rg, cp, tile_r, tile_c, rows, cols,
-                        key, col_codes, col_scales);
+    static_assert(ColStage<kDqCols>::kBytes <= kChunks * 16, "stage fits a tile");
+    uint4* s_col = smem + buf * kChunks;
+    uint8_t* s_sc = reinterpret_cast<uint8_t*>(s_col + ColStage<kDqCols>::kChunks);
+    if (tile_r + 32 * rg < rows)
+      stage_column_pair(dq_column_pass<BIG>(s_codes, s_scales, rg, cp, tile_r,
+                                            tile_c, cols, key),
+                        cp, rg, s_col, s_sc);
     __syncthreads();
+    store_staged_columns<kDqCols, kDqThreads>(s_col, s_sc, tile_r, tile_c,
+                                              rows, cols, col_codes, col_scales);
+    __syncthreads();  // the next copies overwrite this buffer
   }
   cp_async_wait<0>();
 }
@@ -726,7 +816,8 @@ static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
                           ((cols + T::kCols - 1) / T::kCols);
   if (VEC) {
     auto kern = k_quant_cols_pipe<BF16, SR, EVEN, BIG>;
-    constexpr size_t smem = 2 * kTileRows * T::kChunksPerRow * sizeof(uint4);
+    constexpr size_t smem = 2 * kTileRows * T::kChunksPerRow * sizeof(uint4) +
+                            ColStage<T::kCols>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(
         reinterpret_cast<const void*>(kern),
         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
       const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + e0);
       uint4 q[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) q[i] = ld_stream(p + i);
+      for (int i = 0; i < 4; ++i) q[i] = ld_l1(p + i);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t w4[4] = {q[i].x ^ flip[4 * i], q[i].y ^ flip[4 * i + 1],
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
       const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(x) + e0);
       uint4 q[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) q[i] = ld_stream(p + i);
+      for (int i = 0; i < 8; ++i) q[i] = ld_l1(p + i);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         y[4 * i] = __uint_as_float(q[i].x ^ flip[4 * i]);
