@@ -59,16 +59,16 @@ __host__ __forceinline__ RngKey make_key(uint64_t seed, uint32_t stream) {
   return r;
 }
 
-// mix32 on the device. The right shifts are written as high halves of
-// multiplies by powers of two (h >> k == umulhi(h, 2^(32-k))), which issue
-// on the multiply-add pipe and leave the integer logic pipe, the limit of the
-// stochastic-rounding kernels, to the XORs.
+// mix32 on the device. The stochastic-rounding kernels are bound by the
+// integer logic pipe and the multiply pipe together; the two multiplies
+// already load the latter, so the shifts stay plain shifts (measured: moving
+// them onto the multiply pipe as high halves of products was slower).
 __device__ __forceinline__ uint32_t mix32_d(uint32_t h) {
-  h ^= __umulhi(h, 1u << 16);
+  h ^= h >> 16;
   h *= 0x85EBCA6Bu;
-  h ^= __umulhi(h, 1u << 19);
+  h ^= h >> 13;
   h *= 0xC2B2AE35u;
-  h ^= __umulhi(h, 1u << 16);
+  h ^= h >> 16;
   return h;
 }
 
@@ -151,8 +151,8 @@ __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
   const float a = fabsf(v);
   float y = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
   y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
-  const uint32_t m = __umulhi(__float_as_uint(y) + noise, 1u << 10);  // >> 22
-  return m + __umulhi(__float_as_uint(v), 2u) * 8u;                  // sign
+  const uint32_t m = (__float_as_uint(y) + noise) >> 22;
+  return m + (__float_as_uint(v) >> 31) * 8u;  // sign
 }
 
 // Stochastic codes of 8 values; pair k of the 8 values takes its two random
