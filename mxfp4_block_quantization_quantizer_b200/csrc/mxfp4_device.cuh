@@ -97,9 +97,10 @@ __device__ __forceinline__ float inv_scale(uint32_t sb) {
   return __uint_as_float((254u - b) << 23);
 }
 
-// 2^e as fp32 for byte sb (sb = 0 gives the subnormal 2^-127).
+// 2^e as fp32 for byte sb (sb = 0 gives the subnormal 2^-127, whose pattern
+// 0x00400000 lies below every normal one; sb = 0xFF gives +inf).
 __device__ __forceinline__ float scale_value(uint32_t sb) {
-  return __uint_as_float(sb ? (sb << 23) : 0x00400000u);
+  return __uint_as_float(max(sb << 23, 0x00400000u));
 }
 
 // ---------------------------------------------------------------------------
@@ -147,10 +148,13 @@ __device__ __forceinline__ uint32_t sr_noise_hi(uint32_t h) {  // r = h >> 16
   return sr_noise(__umulhi(h, 1u << 16));
 }
 
+// SAT = false leaves out the saturation, for callers whose |v| never exceeds
+// 6.
+template <bool SAT = true>
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
   const float a = fabsf(v);
   float y = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
-  y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
+  if (SAT) y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
   const uint32_t m = (__float_as_uint(y) + noise) >> 22;
   return m + (__float_as_uint(v) >> 31) * 8u;  // sign
 }
@@ -228,6 +232,15 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) {
 }
 __device__ __forceinline__ float bf16_hi(uint32_t w) {
   return __uint_as_float(w & 0xFFFF0000u);
+}
+
+// max(|a|, m) for m >= 0 or NaN, propagating NaN (a NaN a or m gives NaN).
+__device__ __forceinline__ float absmax_nan(float a, float m) {
+  float d;
+  asm("{\n\t.reg .f32 t;\n\tabs.f32 t, %1;\n\tmax.NaN.f32 %0, t, %2;\n\t}"
+      : "=f"(d)
+      : "f"(a), "f"(m));
+  return d;
 }
 
 // Per-half unsigned max of two packed 16-bit pairs.

@@ -164,7 +164,7 @@ struct ColPair {
 // Quantize the two adjacent columns c0, c0+1 over the 32 rows r0 .. r0+31.
 // get(j) returns the values of row r0+j (x: column c0, y: column c0+1); ma
 // and mb are the fp32 bit patterns of the two columns' absolute maxima.
-template <bool SR, bool EVEN, bool BIG, typename Get>
+template <bool SR, bool EVEN, bool BIG, bool SAT = true, typename Get>
 __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
                                                      uint32_t mb, int64_t r0,
                                                      int64_t c0, int64_t cols,
@@ -182,8 +182,8 @@ __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
       uint32_t na, nb;
       column_noise<EVEN, BIG>(key, i0, cols, j, na, nb);
       const float2 v = get(j);
-      o.wa[j >> 3] += e2m1_sr(v.x * mula, na) * (1u << (4 * (j & 7)));
-      o.wb[j >> 3] += e2m1_sr(v.y * mulb, nb) * (1u << (4 * (j & 7)));
+      o.wa[j >> 3] += e2m1_sr<SAT>(v.x * mula, na) * (1u << (4 * (j & 7)));
+      o.wb[j >> 3] += e2m1_sr<SAT>(v.y * mulb, nb) * (1u << (4 * (j & 7)));
     }
   } else {
 #pragma unroll
@@ -660,9 +660,14 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
 
 // Column pass of the double quantizer over the staged Q_D(X) codes: decode
 // columns 2cp, 2cp+1 of rows 32rg.. (one shared byte per row holds both
-// codes; a row group of scale 0xFF decodes to NaN as 0 x inf), then
+// codes; a row group of scale 0xFF decodes to NaN as 0 x inf, and the
+// NaN-propagating maximum carries it into the column scale), then
 // stochastic rounding along the 32x1 groups. The caller checks that the row
 // group lies inside the tensor.
+//
+// No saturation is needed: every decoded value is G[m] 2^k, two significant
+// bits, and the column scale puts the column maximum in [4, 8), so a scaled
+// value is at most 6 (the only such values in [4, 8) are 4 and 6).
 template <bool BIG>
 __device__ __forceinline__ ColPair dq_column_pass(
     const uint32_t* s_codes, const uint8_t* s_scales, int rg, int cp,
@@ -670,7 +675,7 @@ __device__ __forceinline__ ColPair dq_column_pass(
   const int64_t r0 = tile_r + 32 * rg;
   const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
   float a[32], b[32];
-  uint32_t ma = 0, mb = 0;
+  float ma = 0.0f, mb = 0.0f;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     uint32_t w4 = 0;
@@ -687,14 +692,14 @@ __device__ __forceinline__ ColPair dq_column_pass(
     for (int i = 0; i < 4; ++i) {
       a[4 * q + i] = f[2 * i] * sv[i];
       b[4 * q + i] = f[2 * i + 1] * sv[i];
-      ma = max(ma, __float_as_uint(a[4 * q + i]) & 0x7FFFFFFFu);
-      mb = max(mb, __float_as_uint(b[4 * q + i]) & 0x7FFFFFFFu);
+      ma = absmax_nan(a[4 * q + i], ma);
+      mb = absmax_nan(b[4 * q + i], mb);
     }
   }
   // cols is a multiple of 32 here, so every pair index is even-aligned
-  return column_pair_codes<true, true, BIG>(
-      [&](int j) { return make_float2(a[j], b[j]); }, ma, mb, r0,
-      tile_c + 2 * cp, cols, key);
+  return column_pair_codes<true, true, BIG, false>(
+      [&](int j) { return make_float2(a[j], b[j]); }, __float_as_uint(ma),
+      __float_as_uint(mb), r0, tile_c + 2 * cp, cols, key);
 }
 
 // Fused double quantization of bf16 X, double-buffered: the raw tiles are
