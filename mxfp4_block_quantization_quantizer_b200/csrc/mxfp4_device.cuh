@@ -59,17 +59,25 @@ __host__ __forceinline__ RngKey make_key(uint64_t seed, uint32_t stream) {
   return r;
 }
 
-// mix32 on the device. The stochastic-rounding kernels are bound by the
-// integer logic pipe and the multiply pipe together; the two multiplies
-// already load the latter, so the shifts stay plain shifts (measured: moving
-// them onto the multiply pipe as high halves of products was slower).
-__device__ __forceinline__ uint32_t mix32_d(uint32_t h) {
+// mix32 on the device, in two parts: mix32_pre is every step but the last
+// xor-shift, so mix32(x) = g ^ (g >> 16) with g = mix32_pre(x). Consumers of
+// the two 16-bit halves take them from g directly: the high half of mix32 is
+// g >> 16 (the xor only touches the low half) and the low half is
+// (g ^ (g >> 16)) & 0xFFFF; the top bit of mix32 is the top bit of g. The
+// stochastic-rounding kernels are bound by the integer logic pipe and the
+// multiply pipe together; the two multiplies already load the latter, so the
+// shifts stay plain shifts (measured: issuing them on the multiply pipe as
+// high halves of products was slower).
+__device__ __forceinline__ uint32_t mix32_pre(uint32_t h) {
   h ^= h >> 16;
   h *= 0x85EBCA6Bu;
   h ^= h >> 13;
   h *= 0xC2B2AE35u;
-  h ^= h >> 16;
   return h;
+}
+__device__ __forceinline__ uint32_t mix32_d(uint32_t h) {
+  const uint32_t g = mix32_pre(h);
+  return g ^ (g >> 16);
 }
 
 // Inner hash for counters whose high word is `hi` (0 for every tensor below
@@ -141,11 +149,13 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 __device__ __forceinline__ uint32_t sr_noise(uint32_t r) {
   return r * 0xFFFFFFC0u + 0xC13FFFDFu;  // (2^22 - 33 - 64r) - 0x3F000000
 }
-__device__ __forceinline__ uint32_t sr_noise_lo(uint32_t h) {  // r = h & 0xFFFF
-  return sr_noise(h & 0xFFFFu);
+// The noises of the pair whose hash is mix32 = g ^ (g >> 16), g = mix32_pre
+// of its counter: the even element takes the low half, the odd one the high.
+__device__ __forceinline__ uint32_t sr_noise_lo(uint32_t g) {
+  return sr_noise((g ^ (g >> 16)) & 0xFFFFu);
 }
-__device__ __forceinline__ uint32_t sr_noise_hi(uint32_t h) {  // r = h >> 16
-  return sr_noise(__umulhi(h, 1u << 16));
+__device__ __forceinline__ uint32_t sr_noise_hi(uint32_t g) {
+  return sr_noise(__umulhi(g, 1u << 16));  // g >> 16 on the multiply pipe
 }
 
 // SAT = false leaves out the saturation, for callers whose |v| never exceeds
@@ -160,14 +170,15 @@ __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
 }
 
 // Stochastic codes of 8 values; pair k of the 8 values takes its two random
-// numbers from h[k] (low half for the even element).
+// numbers from the hash whose mix32_pre is g[k] (low half for the even
+// element).
 __device__ __forceinline__ uint32_t e2m1x8_sr(const float* v,
-                                              const uint32_t* h) {
+                                              const uint32_t* g) {
   uint32_t out = 0;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    out += e2m1_sr(v[2 * k], sr_noise_lo(h[k])) * (1u << (8 * k));
-    out += e2m1_sr(v[2 * k + 1], sr_noise_hi(h[k])) * (1u << (8 * k + 4));
+    out += e2m1_sr(v[2 * k], sr_noise_lo(g[k])) * (1u << (8 * k));
+    out += e2m1_sr(v[2 * k + 1], sr_noise_hi(g[k])) * (1u << (8 * k + 4));
   }
   return out;
 }

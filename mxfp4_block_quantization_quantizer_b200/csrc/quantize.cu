@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kRowThreads)
         const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
         uint32_t h[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) h[k] = mix32_d(kh + uint32_t(p0) + k);
+        for (int k = 0; k < 4; ++k) h[k] = mix32_pre(kh + uint32_t(p0) + k);
         word = e2m1x8_sr(v[u], h);
       } else {
         word = e2m1x8_rn(v[u]);
@@ -134,20 +134,20 @@ __device__ __forceinline__ void column_noise(RngKey key, uint64_t i0,
                                              int64_t cols, int j, uint32_t& na,
                                              uint32_t& nb) {
   if (EVEN && !BIG) {
-    const uint32_t h = mix32_d(key.k0 + uint32_t(i0 >> 1) +
-                               uint32_t(j) * uint32_t(uint64_t(cols) >> 1));
+    const uint32_t h = mix32_pre(key.k0 + uint32_t(i0 >> 1) +
+                                 uint32_t(j) * uint32_t(uint64_t(cols) >> 1));
     na = sr_noise_lo(h);
     nb = sr_noise_hi(h);
   } else {
     const uint64_t i = i0 + uint64_t(j) * uint64_t(cols);
     const uint64_t p = i >> 1;
-    const uint32_t h = mix32_d(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
+    const uint32_t h = mix32_pre(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
     if ((i & 1) == 0) {
       na = sr_noise_lo(h);
       nb = sr_noise_hi(h);
     } else {
       const uint64_t p2 = p + 1;
-      const uint32_t h2 = mix32_d(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
+      const uint32_t h2 = mix32_pre(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
       na = sr_noise_hi(h);
       nb = sr_noise_lo(h2);
     }

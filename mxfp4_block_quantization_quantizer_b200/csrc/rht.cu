@@ -40,9 +40,10 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
   const int64_t n_cgroups = cols / 32;
   {
     // warp w hashes the 32 column signs of column group blockIdx.x*8 + w
+    // (bit 31 of mix32 is bit 31 of mix32_pre)
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t c = uint32_t((int64_t(blockIdx.x) * kRhtGroupsX + w) * 32 + lane);
-    const unsigned neg = __ballot_sync(0xFFFFFFFFu, (mix32_d(sign_key + c) >> 31) != 0);
+    const unsigned neg = __ballot_sync(0xFFFFFFFFu, (mix32_pre(sign_key + c) >> 31) != 0);
     if (lane == 0) sign_bits[w] = neg;
   }
   __syncthreads();
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
         const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
         uint32_t h[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) h[t] = mix32_d(kh + uint32_t(p0) + t);
+        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + uint32_t(p0) + t);
         wq[q] = e2m1x8_sr(v, h);
       } else {
         wq[q] = e2m1x8_rn(v);
