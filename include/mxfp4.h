@@ -198,6 +198,32 @@ mxfp4_status mxfp4_qema_quantize(const float* w, float* w_ema, int64_t rows,
                                  int64_t cols, float beta, uint8_t* codes,
                                  uint8_t* scales, void* stream);
 
+/*
+ * Scale bytes in the blocked order that block-scaled tensor-core GEMMs read.
+ * Source: "Oscillation-Reduced MXFP4 Training for Vision Transformers",
+ * abstract (the MX format is supported by the Blackwell architecture); the
+ * order itself is NVIDIA's published one-dimensional block-scaling-factor
+ * layout of its block-scaled GEMMs (a reading: the pages name the hardware,
+ * not the layout). Both GEMM operands of an MXFP4 product are K-major with
+ * one scale per 32 elements along K, which is what mxfp4_quantize writes: a
+ * ROWS quantization of X [R, C] is an operand with rows = R, groups = C/32;
+ * a COLS quantization (and the column output of mxfp4_double_quantize) is
+ * the operand X^T with rows = C, groups = R/32.
+ *
+ * The matrix scales[rows][groups] (row-major) is cut into tiles of 128 rows
+ * by 4 groups, zero-padded at the edges; tiles are stored one after another,
+ * along the groups first, then for the next 128 rows, 512 bytes each; inside
+ * a tile the scale of tile row r and tile group g is byte
+ * 16*(r mod 32) + 4*(r div 32) + g.
+ *   scales   device, [rows][groups] bytes, any alignment, read only
+ *   blocked  device, ceil(rows/128)*128 * ceil(groups/4)*4 bytes, 16-byte
+ *            aligned, written entirely (padding included)
+ * rows, groups > 0 and within the size limit of the other entry points.
+ */
+mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
+                                     int64_t groups, uint8_t* blocked,
+                                     void* stream);
+
 /* Static text for a status code; never NULL. */
 const char* mxfp4_status_string(int status);
 

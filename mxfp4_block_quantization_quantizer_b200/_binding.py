@@ -22,7 +22,7 @@ RNE, SR = 0, 1
 SYMBOLS = ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_double_quantize",
            "mxfp4_rht_quantize", "mxfp4_osc_step",
            "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
-           "mxfp4_status_string")
+           "mxfp4_scales_to_blocked", "mxfp4_status_string")
 
 
 class Mxfp4Error(RuntimeError):
@@ -60,6 +60,7 @@ def lib():
                                            ctypes.c_float, vp],
             "mxfp4_qema_quantize": [vp, vp, i64, i64, ctypes.c_float, vp, vp,
                                     vp],
+            "mxfp4_scales_to_blocked": [vp, i64, i64, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -221,6 +222,23 @@ def qema_quantize(w, w_ema, beta=0.998, out=None, stream=None):
     return codes, scales
 
 
+def scales_to_blocked(scales, out=None, stream=None):
+    """mxfp4_scales_to_blocked: the [rows, groups] uint8 CUDA scales in the
+    blocked order of block-scaled GEMMs, returned as a
+    [ceil(rows/128)*128, ceil(groups/4)*4] uint8 tensor (storage order)."""
+    _cuda2d(scales, "scales")
+    if scales.dtype != torch.uint8:
+        raise TypeError("scales must be uint8")
+    rows, groups = scales.shape
+    if out is None:
+        out = _empty_u8((-(-rows // 128) * 128, -(-groups // 4) * 4),
+                        scales.device)
+    _check(lib().mxfp4_scales_to_blocked(_ptr(scales), rows, groups, _ptr(out),
+                                         _stream(scales.device, stream)),
+           "mxfp4_scales_to_blocked")
+    return out
+
+
 # The C names, for callers that prefer them.
 mxfp4_quantize = quantize
 mxfp4_dequantize = dequantize
@@ -229,4 +247,5 @@ mxfp4_rht_quantize = rht_quantize
 mxfp4_osc_step = osc_step
 mxfp4_osc_synthetic_update = osc_synthetic_update
 mxfp4_qema_quantize = qema_quantize
+mxfp4_scales_to_blocked = scales_to_blocked
 mxfp4_status_string = status_string

@@ -132,6 +132,16 @@ mxfp4_status mxfp4_qema_quantize(const float* w, float* w_ema, int64_t rows,
                                             codes, scales, as_stream(stream)));
 }
 
+mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
+                                     int64_t groups, uint8_t* blocked,
+                                     void* stream) {
+  if (!scales || !blocked) return MXFP4_ERR_NULL;
+  if (!dims_ok(rows, groups)) return MXFP4_ERR_SHAPE;
+  if (!aligned16(blocked)) return MXFP4_ERR_ALIGN;
+  return from_cuda(mxfp4::launch_scales_blocked(scales, rows, groups, blocked,
+                                                as_stream(stream)));
+}
+
 const char* mxfp4_status_string(int status) {
   switch (status) {
     case MXFP4_OK: return "ok";

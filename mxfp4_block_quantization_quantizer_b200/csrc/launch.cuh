@@ -49,4 +49,9 @@ cudaError_t launch_qema_quant(const float* w, float* w_ema, int64_t rows,
 cudaError_t launch_osc_update(float* w, int64_t n, uint64_t seed,
                               uint32_t step, float rel_step, cudaStream_t s);
 
+// Scales [rows][groups] -> the blocked order of block-scaled GEMMs.
+cudaError_t launch_scales_blocked(const uint8_t* scales, int64_t rows,
+                                  int64_t groups, uint8_t* blocked,
+                                  cudaStream_t s);
+
 }  // namespace mxfp4

@@ -77,6 +77,7 @@ def _declare(L):
                                       ctypes.c_float], i32),
         "orc_qema_quantize": ([_fp, _fp, i64, i64, ctypes.c_float, _u8p,
                                _u8p], i32),
+        "orc_scales_to_blocked": ([_u8p, i64, i64, _u8p], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -232,6 +233,18 @@ class Oracle:
                                     _u8(codes), _u8(scales)):
             raise ValueError("bad shape for the oracle Q-EMA")
         return codes.reshape(R, C // 2), scales.reshape(R, C // 32)
+
+    def scales_to_blocked(self, scales):
+        """The [rows, groups] scale bytes in the blocked layout of
+        block-scaled GEMMs, as a [ceil(rows/128)*128, ceil(groups/4)*4]
+        uint8 array (the bytes in storage order)."""
+        s = np.ascontiguousarray(scales, np.uint8)
+        rows, groups = s.shape
+        pr, pg = -(-rows // 128) * 128, -(-groups // 4) * 4
+        out = np.zeros(pr * pg, np.uint8)
+        if self.L.orc_scales_to_blocked(_u8(s.reshape(-1)), rows, groups, _u8(out)):
+            raise ValueError("bad shape for the blocked scale layout")
+        return out.reshape(pr, pg)
 
 
 _default = None

@@ -504,3 +504,33 @@ int orc_qema_quantize(const float* w, float* w_ema, int64_t rows, int64_t cols,
   return orc_quantize(w_ema, DT_F32, rows, cols, 0, AX_ROWS, RND_RNE, 0,
                       codes, scales);
 }
+
+/* ------------------------------------------------------------------ */
+/* Blocked scale layout for block-scaled GEMMs. [TJ] abstract: the MX   */
+/* format is supported by the Blackwell architecture; its block-scaled  */
+/* tensor-core GEMMs (and NVIDIA's library GEMMs over them) read the    */
+/* scales of an operand [rows, K], one byte per 32-element group along  */
+/* K, in NVIDIA's published one-dimensional block-scaling-factor layout */
+/* (a reading: the pages name the hardware, not the layout).            */
+/* ------------------------------------------------------------------ */
+
+/* The scale matrix [rows][groups] is cut into tiles of 128 rows by 4
+ * groups, padded with zero bytes; tiles are stored one after another,
+ * across the groups first, then for the next 128 rows; each tile is 512
+ * bytes, and inside it the scale of tile row r and tile group g is byte
+ * 16 * (r mod 32) + 4 * (r div 32) + g. out holds
+ * ceil(rows/128) * 128 * ceil(groups/4) * 4 bytes. */
+int orc_scales_to_blocked(const uint8_t* s, int64_t rows, int64_t groups,
+                          uint8_t* out) {
+  if (rows <= 0 || groups <= 0) return -1;
+  const int64_t row_tiles = (rows + 127) / 128, group_tiles = (groups + 3) / 4;
+  memset(out, 0, (size_t)(row_tiles * group_tiles * 512));
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t g = 0; g < groups; ++g) {
+      const int64_t tile = (r / 128) * group_tiles + g / 4;
+      const int64_t tr = r % 128, tg = g % 4;
+      out[tile * 512 + 16 * (tr % 32) + 4 * (tr / 32) + tg] = s[r * groups + g];
+    }
+  }
+  return 0;
+}

@@ -89,6 +89,12 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_qema_quantize(P, NUL, 64, 64, 0.998, P, P, NUL) == NULL
     assert L.mxfp4_qema_quantize(P, P, 64, 48, 0.998, P, P, NUL) == SHAPE
     assert L.mxfp4_qema_quantize(P, PODD, 64, 64, 0.998, P, P, NUL) == ALIGN
+    assert L.mxfp4_scales_to_blocked(NUL, 128, 4, P, NUL) == NULL
+    assert L.mxfp4_scales_to_blocked(P, 128, 4, NUL, NUL) == NULL
+    assert L.mxfp4_scales_to_blocked(P, 0, 4, P, NUL) == SHAPE
+    assert L.mxfp4_scales_to_blocked(P, 128, -4, P, NUL) == SHAPE
+    assert L.mxfp4_scales_to_blocked(P, 1 << 32, 4, P, NUL) == SHAPE
+    assert L.mxfp4_scales_to_blocked(PODD, 128, 4, PODD, NUL) == ALIGN
 
 
 def test_binding_refuses_host_tensors():

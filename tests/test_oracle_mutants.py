@@ -3,7 +3,8 @@ pins catch every one: a wrong scale offset, ties to odd, a lost sign of zero,
 swapped nibbles, a reversed stochastic comparison, a transposed index, a wrong
 Hadamard entry or normalisation, a wrong random stream, the tracker without
 its absolute value, a reversed flag test, snapping to the old bin, a missing
-reset, column groups built from X instead of Q_D(X). Mistakes are planted in
+reset, column groups built from X instead of Q_D(X), a wrong blocked scale
+order. Mistakes are planted in
 the oracle only, on the CPU; the real oracle source is never modified.
 """
 import os
@@ -18,6 +19,11 @@ SRC = os.path.join(os.path.dirname(O.__file__), "mxfp4_oracle.c")
 
 # (name, original text, mutated text, pins that must fail)
 MUTANTS = [
+    ("blocked lines and slots swapped", "16 * (tr % 32) + 4 * (tr / 32)",
+     "4 * (tr % 32) + 16 * (tr / 32)",
+     ["test_blocked_scales_line_by_line", "test_blocked_scales_is_a_padded_permutation"]),
+    ("blocked tiles down the rows first", "(r / 128) * group_tiles + g / 4",
+     "(g / 4) * row_tiles + r / 128", ["test_blocked_scales_line_by_line"]),
     ("scale offset", "int e = (E - 1) - 2;", "int e = (E - 1) - 1;",
      ["test_scale_exponent_exhaustive_bf16"]),
     ("ties to odd", "(dm == db && (m % 2) == 0)", "(dm == db && (m % 2) == 1)",
@@ -84,7 +90,8 @@ MUTANTS = [
 
 PARAMS = {"test_tiny_tensors_brute_force_layout": [((32, 96), O.COLS),
                                                    ((64, 96), O.ROWS)],
-          "test_qema_matches_the_geometric_closed_form": [(0.9, 200, 40)]}
+          "test_qema_matches_the_geometric_closed_form": [(0.9, 200, 40)],
+          "test_blocked_scales_line_by_line": [((300, 13),)]}
 
 
 def _build(tmp_path, name, src_text):

@@ -585,3 +585,47 @@ def test_qema_codes_are_the_quantized_ema():
     c, s = O.qema_quantize(w, e, 0.998)
     c2, s2 = O.quantize(e, O.ROWS, O.RNE)
     assert np.array_equal(c, c2) and np.array_equal(s, s2)
+
+
+# ---------------------------------------------------------------------------
+# Blocked scale layout (the scale order block-scaled tensor-core GEMMs read)
+# ---------------------------------------------------------------------------
+
+def _blocked_line_by_line(s):
+    """The layout built the way NVIDIA's documentation draws it: a 128 x 4
+    tile of scales is 32 lines of 16 bytes, line i holding the 4 scales of
+    row i, then of rows i+32, i+64 and i+96; tiles follow each other along
+    the groups, then down the rows; padding is zero."""
+    rows, groups = s.shape
+    pr, pg = -(-rows // 128) * 128, -(-groups // 4) * 4
+    p = np.zeros((pr, pg), np.uint8)
+    p[:rows, :groups] = s
+    lines = []
+    for rt in range(pr // 128):
+        for gt in range(pg // 4):
+            tile = p[128 * rt:128 * rt + 128, 4 * gt:4 * gt + 4]
+            for i in range(32):
+                lines.append(np.concatenate([tile[i + 32 * k] for k in range(4)]))
+    return np.concatenate(lines).reshape(pr, pg)
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (128, 4), (130, 5), (256, 8),
+                                   (300, 13), (32, 896)])
+def test_blocked_scales_line_by_line(shape):
+    g = np.random.Generator(np.random.PCG64(40 + shape[0]))
+    s = g.integers(0, 256, size=shape, dtype=np.uint8)
+    assert np.array_equal(O.scales_to_blocked(s), _blocked_line_by_line(s))
+
+
+def test_blocked_scales_is_a_padded_permutation():
+    s = np.arange(1, 1 + 40 * 6, dtype=np.uint8).reshape(40, 6)
+    b = O.scales_to_blocked(s)
+    assert b.shape == (128, 8)
+    vals, counts = np.unique(b, return_counts=True)
+    assert np.array_equal(vals[1:], np.arange(1, 241)) and np.all(counts[1:] == 1)
+    assert counts[0] == 128 * 8 - 240
+    # row 161, group 6 of a 256 x 8 matrix: tile 1*2 + 1, line 1, slot 1
+    s = np.zeros((256, 8), np.uint8)
+    s[161, 6] = 7
+    flat = O.scales_to_blocked(s).reshape(-1)
+    assert np.flatnonzero(flat).tolist() == [3 * 512 + 16 + 4 + 2]
