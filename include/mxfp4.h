@@ -224,6 +224,31 @@ mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
                                      int64_t groups, uint8_t* blocked,
                                      void* stream);
 
+/*
+ * MXFP4 GEMM on the block-scaled tensor cores, consuming quantizer outputs:
+ *   C[m][n] = sum_k A[m][k] * B[n][k]      (fp32 accumulate, fp32 out)
+ * where A[i][k] = G(a_codes)[i][k] * 2^(a scale of group k/32 of row i - 127)
+ * and likewise B. Source: "Oscillation-Reduced MXFP4 Training for Vision
+ * Transformers", abstract and rebuttal Question 2 (forward and backward
+ * GEMMs on MXFP4 operands quantized along the reduction axis; MX on
+ * Blackwell tensor cores).
+ *   a_codes   device, [m][k/2], K-major (the ROWS codes of an [m, k] tensor,
+ *             or the COLS codes of a [k, m] tensor), 16-byte aligned
+ *   a_scales  device, the scales of a_codes in the blocked order of
+ *             mxfp4_scales_to_blocked (rows = m, groups = k/32), 16-byte
+ *             aligned
+ *   b_codes, b_scales  the same for B with n rows
+ *   c         device fp32 [m][n], written (every element)
+ * k must be a multiple of 32; m, n, k > 0 within the size limit. The result
+ * equals the exact sum of the products up to fp32 accumulation rounding (the
+ * order of the additions is the hardware's). A tile whose tensor-core work
+ * does not complete within a bounded wait is written as NaN.
+ */
+mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                        const uint8_t* b_codes, const uint8_t* b_scales,
+                        int64_t m, int64_t n, int64_t k, float* c,
+                        void* stream);
+
 /* Static text for a status code; never NULL. */
 const char* mxfp4_status_string(int status);
 

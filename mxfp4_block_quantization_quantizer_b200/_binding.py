@@ -22,7 +22,7 @@ RNE, SR = 0, 1
 SYMBOLS = ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_double_quantize",
            "mxfp4_rht_quantize", "mxfp4_osc_step",
            "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
-           "mxfp4_scales_to_blocked", "mxfp4_status_string")
+           "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_status_string")
 
 
 class Mxfp4Error(RuntimeError):
@@ -61,6 +61,7 @@ def lib():
             "mxfp4_qema_quantize": [vp, vp, i64, i64, ctypes.c_float, vp, vp,
                                     vp],
             "mxfp4_scales_to_blocked": [vp, i64, i64, vp, vp],
+            "mxfp4_gemm": [vp, vp, vp, vp, i64, i64, i64, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -239,6 +240,29 @@ def scales_to_blocked(scales, out=None, stream=None):
     return out
 
 
+def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None):
+    """mxfp4_gemm: C = A B^T in fp32 for MXFP4 operands given as K-major
+    codes [rows, k/2] and blocked scales (from scales_to_blocked)."""
+    for name, t in (("a_codes", a_codes), ("a_blocked", a_blocked),
+                    ("b_codes", b_codes), ("b_blocked", b_blocked)):
+        _cuda2d(t, name)
+        if t.dtype != torch.uint8:
+            raise TypeError("%s must be uint8" % name)
+    m, n = a_codes.shape[0], b_codes.shape[0]
+    if a_codes.shape[1] * 2 != k or b_codes.shape[1] * 2 != k:
+        raise ValueError("codes must have k/2 bytes per row")
+    for name, t, rows in (("a_blocked", a_blocked, m), ("b_blocked", b_blocked, n)):
+        need = -(-rows // 128) * 128 * (-(-k // 128) * 4)
+        if t.numel() != need:
+            raise ValueError("%s must hold %d bytes" % (name, need))
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=a_codes.device)
+    _check(lib().mxfp4_gemm(_ptr(a_codes), _ptr(a_blocked), _ptr(b_codes),
+                            _ptr(b_blocked), m, n, k, _ptr(out),
+                            _stream(a_codes.device, stream)), "mxfp4_gemm")
+    return out
+
+
 # The C names, for callers that prefer them.
 mxfp4_quantize = quantize
 mxfp4_dequantize = dequantize
@@ -248,4 +272,5 @@ mxfp4_osc_step = osc_step
 mxfp4_osc_synthetic_update = osc_synthetic_update
 mxfp4_qema_quantize = qema_quantize
 mxfp4_scales_to_blocked = scales_to_blocked
+mxfp4_gemm = gemm
 mxfp4_status_string = status_string

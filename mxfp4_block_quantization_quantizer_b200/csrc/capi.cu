@@ -142,6 +142,23 @@ mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
                                                 as_stream(stream)));
 }
 
+mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                        const uint8_t* b_codes, const uint8_t* b_scales,
+                        int64_t m, int64_t n, int64_t k, float* c,
+                        void* stream) {
+  if (!a_codes || !a_scales || !b_codes || !b_scales || !c)
+    return MXFP4_ERR_NULL;
+  if (!dims_ok(m, k) || !dims_ok(n, k) || !dims_ok(m, n) || k % 32)
+    return MXFP4_ERR_SHAPE;
+  if ((m + 127) / 128 > 65535) return MXFP4_ERR_SHAPE;  // grid y
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) ||
+      !aligned16(b_scales) || !aligned16(c))
+    return MXFP4_ERR_ALIGN;
+  return from_cuda(mxfp4::launch_gemm_mxf4(a_codes, a_scales, b_codes,
+                                           b_scales, m, n, k, c,
+                                           as_stream(stream)));
+}
+
 const char* mxfp4_status_string(int status) {
   switch (status) {
     case MXFP4_OK: return "ok";

@@ -1,0 +1,264 @@
+// MXFP4 x MXFP4 -> fp32 GEMM on the block-scaled tensor cores of sm_100a,
+// consuming the quantizer's outputs directly.
+//
+// Source: "Oscillation-Reduced MXFP4 Training for Vision Transformers",
+// abstract and rebuttal Question 2 (the forward and backward GEMMs run on
+// MXFP4 operands quantized along their reduction axis; the MX format is
+// supported by the Blackwell architecture).
+//
+//   C[m][n] = sum_k A[m][k] * B[n][k]
+//
+// A and B are K-major MXFP4 operands: codes [rows][K/2] with one E8M0 scale
+// per 32 elements along K, the scales in the blocked order written by
+// mxfp4_scales_to_blocked. A ROWS quantization of X is such an operand; so
+// is a COLS quantization (the operand X^T, K along the rows of X).
+//
+// Design (one CTA per 128x128 tile of C, 128 threads):
+//   - the K loop stages 256 K-elements (128 bytes per row) of A and B with
+//     asynchronous copies into the canonical K-major layout without swizzle
+//     that the matrix descriptors describe: 16-byte columns ("core matrix"
+//     rows) of 8 rows, the 8-row groups 128 bytes apart (stride byte
+//     offset), the 16-byte K columns 2048 bytes apart (leading byte offset);
+//   - the two 512-byte blocked scale tiles of A and of B for those 256
+//     elements are staged beside them and copied into tensor memory with
+//     tcgen05.cp (32 lines of 16 bytes, broadcast to the four lane
+//     quarters: lane 32q+i holds line i, whose bytes 4q..4q+3 are the
+//     scales of row 32q+i, which is the row the lane accumulates);
+//   - one thread issues four tcgen05.mma kind::mxf4 (K = 64 each, two
+//     scales per row per instruction, the scale byte inside the 32-bit
+//     tensor-memory cell selected by the scale-factor id) into a 128x128
+//     fp32 accumulator in tensor memory, then tcgen05.commit arrives on an
+//     mbarrier that every thread waits on before the stage is reused;
+//   - the epilogue reads the accumulator with tcgen05.ld (warp w owns lanes
+//     32w..32w+31, i.e. rows) and writes fp32 C.
+// Every wait is bounded: a wait that runs out marks the tile, whose output
+// is then NaN, instead of spinning forever.
+#include "launch.cuh"
+#include "mxfp4_device.cuh"
+
+namespace mxfp4 {
+
+namespace {
+
+constexpr int kGM = 128, kGN = 128;  // C tile
+constexpr int kGKBytes = 128;        // K bytes of A/B per stage (256 elements)
+constexpr int kGChunks = kGKBytes / 16;
+constexpr int kGThreads = 128;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kAccCol = 0;    // 128 fp32 columns
+constexpr uint32_t kSfaCol = 128;  // two 4-column scale tiles
+constexpr uint32_t kSfbCol = 136;
+constexpr long long kWaitLimit = 1ll << 22;
+
+struct __align__(1024) GemmSmem {
+  uint8_t a[kGChunks][kGM][16];
+  uint8_t b[kGChunks][kGN][16];
+  uint8_t sfa[2][512];
+  uint8_t sfb[2][512];
+  unsigned long long mbar;
+  uint32_t tmem_base;
+  int failed;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Matrix descriptor of a K-major operand in shared memory without swizzle:
+// start address, leading byte offset (between 16-byte K columns), stride
+// byte offset (between 8-row groups), all in 16-byte units; version 1.
+__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo,
+                                              uint32_t sbo) {
+  uint64_t d = (smem_u32(p) >> 4) & 0x3FFFu;
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4: E2M1 A and B (format 1), K-major
+// both, N/8 at bit 17, E8M0 scales (bit 23), M/16 at bit 24; the scale
+// factor ids of A (bits 29-30) and B (bits 4-5) are ORed in per MMA.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) |
+                            (uint32_t(kGN >> 3) << 17) | (1u << 23) |
+                            (uint32_t(kGM >> 4) << 24);
+
+__device__ __forceinline__ void mma_mxf4(uint32_t tmem_c, uint64_t adesc,
+                                         uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate, uint32_t tsfa,
+                                         uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, "
+      "%3, [%5], [%6], p;\n\t}\n" ::"r"(tmem_c),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa),
+      "r"(tsfb));
+}
+
+__device__ __forceinline__ void copy_scales_to_tmem(uint32_t taddr,
+                                                    const void* tile) {
+  // 32 lines of 16 bytes, contiguous: one 8-line core matrix every 128 bytes
+  const uint64_t d = smem_desc(tile, 16, 128);
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr),
+               "l"(d));
+}
+
+__device__ __forceinline__ bool wait_parity(unsigned long long* bar,
+                                            uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (long long i = 0; i < kWaitLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(kGThreads)
+    k_gemm_mxf4(const uint8_t* __restrict__ a, const uint8_t* __restrict__ sfa,
+                const uint8_t* __restrict__ b, const uint8_t* __restrict__ sfb,
+                int64_t m, int64_t n, int64_t k, float* __restrict__ c) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  GemmSmem& sm = *reinterpret_cast<GemmSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = int64_t(blockIdx.y) * kGM, n0 = int64_t(blockIdx.x) * kGN;
+  const int64_t kbytes = k / 2;                    // bytes per operand row
+  const int64_t k_tiles = (k + 127) / 128;         // blocked scale tiles along K
+  const int64_t a_tile0 = (m0 / 128) * k_tiles, b_tile0 = (n0 / 128) * k_tiles;
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.mbar)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    sm.failed = 0;
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;");
+  const uint32_t tmem = sm.tmem_base;
+
+  const int64_t n_kb = (kbytes + kGKBytes - 1) / kGKBytes;
+  bool ok = true;
+  for (int64_t kb = 0; kb < n_kb && ok; ++kb) {
+    // stage A and B: 128 rows x 8 chunks of 16 bytes each
+#pragma unroll
+    for (int i = 0; i < kGM * kGChunks / kGThreads; ++i) {
+      const int idx = i * kGThreads + tid;
+      const int row = idx / kGChunks, ch = idx % kGChunks;
+      const int64_t kofs = kb * kGKBytes + 16 * ch;
+      const bool va = m0 + row < m && kofs < kbytes;
+      const bool vb = n0 + row < n && kofs < kbytes;
+      cp_async16(&sm.a[ch][row][0], a + (va ? (m0 + row) * kbytes + kofs : 0), va);
+      cp_async16(&sm.b[ch][row][0], b + (vb ? (n0 + row) * kbytes + kofs : 0), vb);
+    }
+    // stage the scale tiles of this K block: 2 tiles of A, 2 of B
+    {
+      const int which = tid >> 6, j = (tid >> 5) & 1, line = tid & 31;
+      const int64_t kt = 2 * kb + j;
+      const bool v = kt < k_tiles;
+      const uint8_t* src = which == 0 ? sfa + (a_tile0 + kt) * 512 + 16 * line
+                                      : sfb + (b_tile0 + kt) * 512 + 16 * line;
+      uint8_t* dst = which == 0 ? &sm.sfa[j][16 * line] : &sm.sfb[j][16 * line];
+      cp_async16(dst, v ? src : (which == 0 ? sfa : sfb), v);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    // make this thread's shared-memory writes visible to the tensor cores
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        copy_scales_to_tmem(tmem + kSfaCol + 4 * j, &sm.sfa[j][0]);
+        copy_scales_to_tmem(tmem + kSfbCol + 4 * j, &sm.sfb[j][0]);
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t sf_id = 2u * (s & 1);
+        const uint32_t idesc = kIdesc | (sf_id << 29) | (sf_id << 4);
+        const uint32_t tsfa = (tmem + kSfaCol + 4 * (s >> 1)) | (sf_id << 30);
+        const uint32_t tsfb = (tmem + kSfbCol + 4 * (s >> 1)) | (sf_id << 30);
+        const uint64_t ad = smem_desc(&sm.a[2 * s][0][0], kGM * 16, 128);
+        const uint64_t bd = smem_desc(&sm.b[2 * s][0][0], kGN * 16, 128);
+        mma_mxf4(tmem + kAccCol, ad, bd, idesc, (kb > 0 || s > 0) ? 1u : 0u,
+                 tsfa, tsfb);
+      }
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+          ::"r"(smem_u32(&sm.mbar)));
+    }
+    ok = wait_parity(&sm.mbar, uint32_t(kb & 1));
+    if (!ok) atomicExch(&sm.failed, 1);
+    __syncthreads();
+    ok = sm.failed == 0;
+  }
+
+  // epilogue: warp w reads accumulator rows 32w..32w+31
+  asm volatile("tcgen05.fence::after_thread_sync;");
+  const int64_t row = m0 + 32 * warp + lane;
+  const bool failed = sm.failed != 0;
+#pragma unroll 1
+  for (int cb = 0; cb < kGN / 32; ++cb) {
+    uint32_t v[32];
+    const uint32_t taddr = tmem + (uint32_t(32 * warp) << 16) + kAccCol + 32 * cb;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
+        "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
+        "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]),
+          "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]),
+          "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+          "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+          "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    if (row < m) {
+      float* out = c + row * n + n0 + 32 * cb;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + 32 * cb + j < n)
+          out[j] = failed ? __uint_as_float(kNaNf32) : __uint_as_float(v[j]);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 ::"r"(tmem), "r"(kTmemCols));
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
+                             const uint8_t* b, const uint8_t* b_scales,
+                             int64_t m, int64_t n, int64_t k, float* c,
+                             cudaStream_t s) {
+  // Two CTAs per SM at most: each holds 256 of the SM's 512 tensor-memory
+  // columns, so the shared memory request keeps a third from being resident
+  // (and blocking in its allocation).
+  constexpr size_t smem = 100 * 1024;
+  static_assert(sizeof(GemmSmem) <= smem, "gemm smem");
+  cudaError_t e = cudaFuncSetAttribute(
+      reinterpret_cast<const void*>(k_gemm_mxf4),
+      cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(unsigned((n + kGN - 1) / kGN), unsigned((m + kGM - 1) / kGM));
+  k_gemm_mxf4<<<grid, kGThreads, smem, s>>>(a, a_scales, b, b_scales, m, n, k, c);
+  return cudaGetLastError();
+}
+
+}  // namespace mxfp4

@@ -54,4 +54,11 @@ cudaError_t launch_scales_blocked(const uint8_t* scales, int64_t rows,
                                   int64_t groups, uint8_t* blocked,
                                   cudaStream_t s);
 
+// C[m][n] = sum_k A[m][k] B[n][k] on MXFP4 operands (K-major codes,
+// blocked scales), fp32 out, on the block-scaled tensor cores.
+cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
+                             const uint8_t* b, const uint8_t* b_scales,
+                             int64_t m, int64_t n, int64_t k, float* c,
+                             cudaStream_t s);
+
 }  // namespace mxfp4

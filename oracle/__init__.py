@@ -247,6 +247,17 @@ class Oracle:
         return out.reshape(pr, pg)
 
 
+    def gemm(self, a_codes, a_scales, b_codes, b_scales, k):
+        """C = A B^T in fp64 for two K-major MXFP4 operands given as codes
+        [rows, k/2] and plain scales [rows, k/32]: both are dequantized
+        exactly (each value is an E2M1 magnitude times a power of two) and
+        multiplied with numpy's fp64 matmul."""
+        m, n = a_codes.shape[0], b_codes.shape[0]
+        da = self.dequantize(a_codes, a_scales, m, k, ROWS, "f32").astype(np.float64)
+        db = self.dequantize(b_codes, b_scales, n, k, ROWS, "f32").astype(np.float64)
+        return da @ db.T
+
+
 _default = None
 
 

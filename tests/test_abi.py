@@ -95,6 +95,11 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_scales_to_blocked(P, 128, -4, P, NUL) == SHAPE
     assert L.mxfp4_scales_to_blocked(P, 1 << 32, 4, P, NUL) == SHAPE
     assert L.mxfp4_scales_to_blocked(PODD, 128, 4, PODD, NUL) == ALIGN
+    assert L.mxfp4_gemm(P, P, P, NUL, 128, 128, 256, P, NUL) == NULL
+    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 48, P, NUL) == SHAPE
+    assert L.mxfp4_gemm(P, P, P, P, 0, 128, 256, P, NUL) == SHAPE
+    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, PODD, NUL) == ALIGN
+    assert L.mxfp4_gemm(P, PODD, P, P, 128, 128, 256, P, NUL) == ALIGN
 
 
 def test_binding_refuses_host_tensors():

@@ -629,3 +629,25 @@ def test_blocked_scales_is_a_padded_permutation():
     s[161, 6] = 7
     flat = O.scales_to_blocked(s).reshape(-1)
     assert np.flatnonzero(flat).tolist() == [3 * 512 + 16 + 4 + 2]
+
+
+def test_gemm_is_the_sum_of_dequantized_products():
+    """The oracle GEMM against the definition written as loops (tiny case)."""
+    g = np.random.Generator(np.random.PCG64(50))
+    ca = g.integers(0, 256, size=(3, 32), dtype=np.uint8)
+    cb = g.integers(0, 256, size=(2, 32), dtype=np.uint8)
+    sa = g.integers(120, 134, size=(3, 2), dtype=np.uint8)
+    sb = g.integers(120, 134, size=(2, 2), dtype=np.uint8)
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+    def val(codes, scales, i, kk):
+        byte = int(codes[i, kk // 2])
+        c = (byte >> 4) if kk % 2 else (byte & 15)
+        v = grid[c & 7] * 2.0 ** (int(scales[i, kk // 32]) - 127)
+        return -v if c & 8 else v
+
+    c = O.gemm(ca, sa, cb, sb, 64)
+    for i in range(3):
+        for j in range(2):
+            want = sum(val(ca, sa, i, kk) * val(cb, sb, j, kk) for kk in range(64))
+            assert c[i, j] == want
