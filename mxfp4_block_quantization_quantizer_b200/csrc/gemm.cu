@@ -33,6 +33,9 @@
 //     32w..32w+31, i.e. rows) and writes fp32 C.
 // Every wait is bounded: a wait that runs out marks the tile, whose output
 // is then NaN, instead of spinning forever.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "launch.cuh"
 #include "mxfp4_device.cuh"
 
@@ -241,12 +244,281 @@ __global__ void __launch_bounds__(kGThreads)
                  ::"r"(tmem), "r"(kTmemCols));
 }
 
+// ---------------------------------------------------------------------------
+// Pipelined version (K a multiple of 256): TMA loads in the 128-byte swizzled
+// K-major layout, a kPS-stage ring of full/empty mbarriers, warp roles.
+//   warp 0: one thread issues the tensor-memory-access (TMA) loads of A and B
+//           and the bulk copies of their scale tiles into a free stage;
+//   warp 1: allocates tensor memory; one thread copies each stage's scales
+//           into tensor memory and issues the MMAs, whose completion
+//           (tcgen05.commit) frees the stage;
+//   warps 2-5: epilogue, one lane quarter (32 accumulator rows) each.
+// The C tile is 128 x 256: two 128-column accumulators, each MMA of K = 64
+// issued once per half with that half's B rows and scales.
+// ---------------------------------------------------------------------------
+
+constexpr int kPS = 4;            // pipeline stages
+constexpr int kPN = 256;          // C tile columns
+constexpr int kPThreads = 192;
+constexpr uint32_t kPTmemCols = 512;
+constexpr uint32_t kPSfCol = 256;  // per stage: 8 SFA columns, then 16 SFB
+constexpr uint32_t kPSfStride = 24;
+
+struct __align__(1024) PipeSmem {
+  uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
+  uint8_t b[kPS][kPN][128];
+  uint8_t sfa[kPS][2][512];       // 2 blocked tiles (256 K elements)
+  uint8_t sfb[kPS][2][2][512];    // [N half][K tile]
+  unsigned long long full[kPS], empty[kPS], acc_full;
+  uint32_t tmem_base;
+  int failed;
+};
+
+// Descriptor of a 128-byte-swizzled K-major operand: 8-row groups 1024
+// bytes apart; the start address moves 32 bytes per K = 64 step inside the
+// 128-byte swizzle row.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
+  uint64_t d = (smem_u32(p) >> 4) & 0x3FFFu;
+  d |= uint64_t(1) << 16;                  // leading byte offset (unused)
+  d |= uint64_t(1024 >> 4) << 32;          // stride byte offset
+  d |= uint64_t(1) << 46;                  // version
+  d |= uint64_t(2) << 61;                  // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x,
+                                            int y, unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+      "%2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool failed_flag(const int* f) {
+  return *static_cast<const volatile int*>(f) != 0;
+}
+
+__device__ __forceinline__ void commit_to(unsigned long long* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar)));
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    k_gemm_mxf4_pipe(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
+                     int64_t m, int64_t n, int64_t k, float* __restrict__ c) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128-byte swizzle wants 1024-byte aligned tiles: align the base by
+  // hand (the launch requests 1 KB of slack)
+  PipeSmem& sm = *reinterpret_cast<PipeSmem*>(
+      smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t m0 = int64_t(blockIdx.y) * kGM, n0 = int64_t(blockIdx.x) * kPN;
+  const int64_t k_tiles = k / 128;
+  const int64_t n_kb = k / 256;
+  const int64_t n_row_tiles = (n + 127) / 128;
+
+  if (tid == 0) {
+    for (int s = 0; s < kPS; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.full[s])));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.empty[s])));
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.acc_full)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    sm.failed = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&sm.tmem_base)), "r"(kPTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;");
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int64_t kb = 0; kb < n_kb; ++kb) {
+        const int s = int(kb % kPS);
+        const uint32_t ph = uint32_t((kb / kPS) & 1);
+        if (!wait_parity(&sm.empty[s], ph ^ 1u) || failed_flag(&sm.failed)) {
+          atomicExch(&sm.failed, 1);
+          break;
+        }
+        const int64_t rb = n0 / 128;
+        const bool half1 = rb + 1 < n_row_tiles;
+        const uint32_t bytes = kGM * 128 + kPN * 128 + 1024 + (half1 ? 2048 : 1024);
+        expect_tx(&sm.full[s], bytes);
+        tma_load_2d(&sm.a[s][0][0], &tm_a, int(kb * 128), int(m0), &sm.full[s]);
+        tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb * 128), int(n0), &sm.full[s]);
+        bulk_load(&sm.sfa[s][0][0], sfa + ((m0 / 128) * k_tiles + 2 * kb) * 512, 1024,
+                  &sm.full[s]);
+        bulk_load(&sm.sfb[s][0][0][0], sfb + (rb * k_tiles + 2 * kb) * 512, 1024,
+                  &sm.full[s]);
+        if (half1)
+          bulk_load(&sm.sfb[s][1][0][0], sfb + ((rb + 1) * k_tiles + 2 * kb) * 512, 1024,
+                    &sm.full[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int64_t kb = 0; kb < n_kb; ++kb) {
+        const int s = int(kb % kPS);
+        const uint32_t ph = uint32_t((kb / kPS) & 1);
+        if (!wait_parity(&sm.full[s], ph) || failed_flag(&sm.failed)) {
+          atomicExch(&sm.failed, 1);
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        const uint32_t sf = tmem + kPSfCol + kPSfStride * uint32_t(s);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          copy_scales_to_tmem(sf + 4 * j, &sm.sfa[s][j][0]);
+          copy_scales_to_tmem(sf + 8 + 4 * j, &sm.sfb[s][0][j][0]);
+          copy_scales_to_tmem(sf + 16 + 4 * j, &sm.sfb[s][1][j][0]);
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t sf_id = 2u * (t & 1);
+          const uint32_t idesc = kIdesc | (sf_id << 29) | (sf_id << 4);
+          const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
+          const uint64_t ad = smem_desc_sw128(&sm.a[s][0][32 * t]);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t tsfb = (sf + 8 + 8 * h + 4 * (t >> 1)) | (sf_id << 30);
+            const uint64_t bd = smem_desc_sw128(&sm.b[s][128 * h][32 * t]);
+            mma_mxf4(tmem + 128 * h, ad, bd, idesc, (kb > 0 || t > 0) ? 1u : 0u, tsfa,
+                     tsfb);
+          }
+        }
+        commit_to(&sm.empty[s]);
+      }
+      commit_to(&sm.acc_full);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;  // lane quarter this warp may read
+    const bool ok = wait_parity(&sm.acc_full, 0);
+    if (!ok) atomicExch(&sm.failed, 1);
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    const bool failed = !ok || failed_flag(&sm.failed);
+    const int64_t row = m0 + 32 * q + lane;
+#pragma unroll 1
+    for (int cb = 0; cb < kPN / 32; ++cb) {
+      uint32_t v[32];
+      const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + 32 * cb;
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
+          "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
+          "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]),
+            "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]),
+            "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+            "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+            "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+            "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+            "=r"(v[30]), "=r"(v[31])
+          : "r"(taddr));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      const int64_t col = n0 + 32 * cb;
+      if (row < m && col < n) {
+        float* out = c + row * n + col;
+        if (col + 32 <= n && (n & 3) == 0) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(out + j) =
+                failed ? make_float4(__uint_as_float(kNaNf32), __uint_as_float(kNaNf32),
+                                     __uint_as_float(kNaNf32), __uint_as_float(kNaNf32))
+                       : make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                     __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col + j < n) out[j] = failed ? __uint_as_float(kNaNf32) : __uint_as_float(v[j]);
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;");
+  __syncthreads();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 ::"r"(tmem), "r"(kPTmemCols));
+}
+
+}  // namespace
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over K-major codes [rows][k/2]: boxes of 128 bytes x box_rows,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k,
+                      uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(k / 2), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(k / 2)};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
                              const uint8_t* b, const uint8_t* b_scales,
                              int64_t m, int64_t n, int64_t k, float* c,
                              cudaStream_t s) {
+  if (k % 256 == 0) {
+    CUtensorMap ma, mb;
+    if (encode_codes_map(&ma, a, m, k, kGM) && encode_codes_map(&mb, b, n, k, kPN)) {
+      constexpr size_t smem = sizeof(PipeSmem) + 1024;
+      cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k_gemm_mxf4_pipe),
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(smem));
+      if (e != cudaSuccess) return e;
+      const dim3 grid(unsigned((n + kPN - 1) / kPN), unsigned((m + kGM - 1) / kGM));
+      k_gemm_mxf4_pipe<<<grid, kPThreads, smem, s>>>(ma, mb, a_scales, b_scales, m, n, k,
+                                                     c);
+      return cudaGetLastError();
+    }
+  }
   // Two CTAs per SM at most: each holds 256 of the SM's 512 tensor-memory
   // columns, so the shared memory request keeps a third from being resident
   // (and blocking in its allocation).
