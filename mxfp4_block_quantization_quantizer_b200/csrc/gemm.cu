@@ -253,11 +253,13 @@ __global__ void __launch_bounds__(kGThreads)
 //           into tensor memory and issues the MMAs, whose completion
 //           (tcgen05.commit) frees the stage;
 //   warps 2-5: epilogue, one lane quarter (32 accumulator rows) each.
-// The C tile is 128 x 256: two 128-column accumulators, each MMA of K = 64
-// issued once per half with that half's B rows and scales.
+// The C tile is 128 x 256: one M = 128, N = 256 MMA per K = 64 step.
 // ---------------------------------------------------------------------------
 
 constexpr int kPS = 4;            // pipeline stages
+// kind::mxf4 instruction descriptor for M = 128, N = 256
+constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
+                                (1u << 23) | (uint32_t(kGM >> 4) << 24);
 constexpr int kPN = 256;          // C tile columns
 constexpr int kPThreads = 192;
 constexpr uint32_t kPTmemCols = 512;
@@ -268,7 +270,7 @@ struct __align__(1024) PipeSmem {
   uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
   uint8_t b[kPS][kPN][128];
   uint8_t sfa[kPS][2][512];       // 2 blocked tiles (256 K elements)
-  uint8_t sfb[kPS][2][2][512];    // [N half][K tile]
+  uint8_t sfb[kPS][2][2][512];    // [128-row block][K tile]
   unsigned long long full[kPS], empty[kPS], acc_full;
   uint32_t tmem_base;
   int failed;
@@ -391,25 +393,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         asm volatile("tcgen05.fence::after_thread_sync;");
         const uint32_t sf = tmem + kPSfCol + kPSfStride * uint32_t(s);
+        // scale factors in tensor memory: row r of an operand in lane r % 32,
+        // 32-bit column r / 32 (A: 4 columns per K tile; B, 256 rows: 8,
+        // its two 128-row tiles side by side), one byte per 32-element group
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           copy_scales_to_tmem(sf + 4 * j, &sm.sfa[s][j][0]);
-          copy_scales_to_tmem(sf + 8 + 4 * j, &sm.sfb[s][0][j][0]);
-          copy_scales_to_tmem(sf + 16 + 4 * j, &sm.sfb[s][1][j][0]);
+          copy_scales_to_tmem(sf + 8 + 8 * j, &sm.sfb[s][0][j][0]);
+          copy_scales_to_tmem(sf + 8 + 8 * j + 4, &sm.sfb[s][1][j][0]);
         }
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint32_t sf_id = 2u * (t & 1);
-          const uint32_t idesc = kIdesc | (sf_id << 29) | (sf_id << 4);
+          const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
           const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
-          const uint64_t ad = smem_desc_sw128(&sm.a[s][0][32 * t]);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t tsfb = (sf + 8 + 8 * h + 4 * (t >> 1)) | (sf_id << 30);
-            const uint64_t bd = smem_desc_sw128(&sm.b[s][128 * h][32 * t]);
-            mma_mxf4(tmem + 128 * h, ad, bd, idesc, (kb > 0 || t > 0) ? 1u : 0u, tsfa,
-                     tsfb);
-          }
+          const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
+          mma_mxf4(tmem, smem_desc_sw128(&sm.a[s][0][32 * t]),
+                   smem_desc_sw128(&sm.b[s][0][32 * t]), idesc,
+                   (kb > 0 || t > 0) ? 1u : 0u, tsfa, tsfb);
         }
         commit_to(&sm.empty[s]);
       }
