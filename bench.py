@@ -48,7 +48,9 @@ OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
 
 
 # Further operations built beyond the step (Q-EMA), timed on their own.
-NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336))}
+NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336)),
+            # Y = Q_D(X) Q_D(W)^T: X the sweep, W a second 8192-row tensor
+            "gemm_mxf4": (None, (8192, 8192, 28672))}
 
 
 def alg_bytes(op):
@@ -104,6 +106,16 @@ def measured_traffic(op):
         if len(parts) >= 3 and parts[0] == op and parts[2] == "src=" + digest:
             return float(parts[1])
     return None
+
+
+def measured_fp4_peak():
+    """Dense FP4 tensor peak: the measured bf16 GEMM burst x 4 (the nominal
+    fp4/bf16 ratio, 9 / 2.25 PFLOP/s); 1.59 PFLOP/s bf16 if unmeasured."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 4"
+    except Exception:
+        return 4.0 * 1590.0, "fallback bf16 x 4"
 
 
 def measured_peaks():
@@ -454,6 +466,38 @@ def run_ours(args):
                                   "launches": args.steps}
         del qw, qe, qout
 
+        # MXFP4 GEMM on the block-scaled tensor cores, consuming the step's
+        # ROWS codes of the sweep as the activation operand
+        gM, gN, gK = NEXT_OPS["gemm_mxf4"][1]
+        if (R, C) == (gM, gK):
+            w2 = torch.from_numpy(W.normal_bf16(gN, gK, 6 + rank).view(np.int16)).view(
+                torch.bfloat16).to(dev)
+            bc, bs = m.quantize(w2, m.ROWS, m.RNE)
+            del w2
+            ac, as_ = m.quantize(buf0["x"], m.ROWS, m.RNE)
+            ab, bb = m.scales_to_blocked(as_), m.scales_to_blocked(bs)
+            gout = torch.empty(gM, gN, dtype=torch.float32, device=dev)
+            for _ in range(args.warmup):
+                m.gemm(ac, ab, bc, bb, gK, out=gout)
+            gev = []
+            for _ in range(args.steps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                m.gemm(ac, ab, bc, bb, gK, out=gout)
+                b.record(stream)
+                gev.append((a, b))
+            torch.cuda.synchronize(dev)
+            d = statistics.mean(a.elapsed_time(b) for a, b in gev) * 1e-3
+            d = reduce_max(d, world, dev)
+            flops = 2.0 * gM * gN * gK
+            peak, kind = measured_fp4_peak()
+            next_ops["gemm_mxf4"] = {"us": d * 1e6, "TFLOP_s": flops / d / 1e12,
+                                     "flops": flops, "shape": [gM, gN, gK],
+                                     "launches": args.steps, "peak_TFLOP_s": peak,
+                                     "peak_kind": kind,
+                                     "frac": flops / d / 1e12 / peak}
+            del ac, as_, bc, bs, ab, bb, gout
+
     # end to end: pinned host input -> device -> kernels -> host results
     if args.no_e2e:
         if rank == 0:
@@ -547,7 +591,8 @@ def run_ours(args):
             "e2e": {"value": job_gbs(world, STEP_BYTES, args.e2e_steps, e2e_ms),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "next_ops": {k: dict(v, frac=v["GB_s"] / peak) for k, v in next_ops.items()},
+            "next_ops": {k: (dict(v, frac=v["GB_s"] / peak) if "GB_s" in v else v)
+                         for k, v in next_ops.items()},
             "gpu_launches": len(ops) * args.steps,
             "clocks": clocks,
         }
