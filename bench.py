@@ -82,11 +82,16 @@ def job_gbs(world, bytes_per_step, steps, elapsed_ms_max):
     return world * bytes_per_step * steps / (elapsed_ms_max * 1e-3) / 1e9
 
 
+# Sources of the kernels whose DRAM traffic profiles/dram_traffic.txt records.
+TRAFFIC_SOURCES = ("quantize.cu", "rht.cu", "osc.cu", "mxfp4_device.cuh",
+                   "launch.cuh")
+
+
 def kernel_source_digest():
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "mxfp4_block_quantization_quantizer_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in TRAFFIC_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:12]
@@ -140,7 +145,44 @@ def parse_args():
                     help="comma-separated ops to run (profiling); default all")
     ap.add_argument("--rows", type=int, default=SWEEP[0],
                     help="rows of the sweep workload (profiling a smaller case)")
+    ap.add_argument("--gemm", default="",
+                    help="M,N,K: time only the MXFP4 GEMM at that shape "
+                         "(profiling); prints one line")
     return ap.parse_args()
+
+
+def run_gemm_only(args):
+    """The MXFP4 GEMM alone on ROWS quantizations of two seeded N(0,1)
+    tensors [M, K] and [N, K] (profiling a case of a chosen size)."""
+    import numpy as np
+    import torch
+
+    import mxfp4_block_quantization_quantizer_b200 as m
+    from mxfp4_block_quantization_quantizer_b200 import workloads as W
+
+    M, N, K = (int(v) for v in args.gemm.split(","))
+    dev = torch.device("cuda", 0)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    ac, as_ = m.quantize(to(W.normal_bf16(M, K, 11)), m.ROWS, m.RNE)
+    bc, bs = m.quantize(to(W.normal_bf16(N, K, 12)), m.ROWS, m.RNE)
+    ab, bb = m.scales_to_blocked(as_), m.scales_to_blocked(bs)
+    out = torch.empty(M, N, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        m.gemm(ac, ab, bc, bb, K, out=out)
+    evs = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        m.gemm(ac, ab, bc, bb, K, out=out)
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize(dev)
+    d = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e-3
+    peak, kind = measured_fp4_peak()
+    tf = 2.0 * M * N * K / d / 1e12
+    print(json.dumps({"profile_run": True, "op": "gemm_mxf4", "shape": [M, N, K],
+                      "us": d * 1e6, "TFLOP_s": tf, "frac": tf / peak,
+                      "peak_kind": kind}), flush=True)
 
 
 def config_block(args, world):
@@ -606,6 +648,9 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.gemm:
+        run_gemm_only(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
