@@ -106,20 +106,32 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
         }
       }
     }
-    uint32_t amax = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      y[j] *= kInvSqrt32;
-      amax = max(amax, __float_as_uint(y[j]) & 0x7FFFFFFFu);
-    }
+    // The rotated value is fl(z * c), z the butterfly output and c = 1/sqrt(32),
+    // and the quantizer scales it by 2^-e. Without the rotated output both
+    // multiplies fold into one, fl(z * (c 2^-e)) = fl(z c) 2^-e (a power of
+    // two commutes with rounding; a result below the normal range only
+    // differs in values that quantize to 0 either way), and the group
+    // maximum is fl(max|z| c), rounding being monotonic.
+    uint32_t amax;
     if (ROT) {
+      amax = 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        y[j] *= kInvSqrt32;
+        amax = max(amax, __float_as_uint(y[j]) & 0x7FFFFFFFu);
+      }
       float4* o = reinterpret_cast<float4*>(rotated + e0);
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         __stcs(o + i, make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]));
+    } else {
+      float zmax = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) zmax = absmax_nan(y[j], zmax);
+      amax = __float_as_uint(zmax * kInvSqrt32);
     }
     const uint32_t sb = scale_byte(amax);
-    const float mul = inv_scale(sb);
+    const float mul = ROT ? inv_scale(sb) : inv_scale(sb) * kInvSqrt32;
     uint32_t wq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
