@@ -82,16 +82,25 @@ def job_gbs(world, bytes_per_step, steps, elapsed_ms_max):
     return world * bytes_per_step * steps / (elapsed_ms_max * 1e-3) / 1e9
 
 
-# Sources of the kernels whose DRAM traffic profiles/dram_traffic.txt records.
-TRAFFIC_SOURCES = ("quantize.cu", "rht.cu", "osc.cu", "mxfp4_device.cuh",
-                   "launch.cuh")
+# Sources of each op's kernel: a DRAM traffic figure in
+# profiles/dram_traffic.txt holds while the digest of these files is unchanged.
+_COMMON_SOURCES = ("mxfp4_device.cuh", "launch.cuh")
+OP_SOURCES = {
+    "quant_rows_rne": ("quantize.cu",) + _COMMON_SOURCES,
+    "quant_cols_sr": ("quantize.cu",) + _COMMON_SOURCES,
+    "double_quant": ("quantize.cu",) + _COMMON_SOURCES,
+    "dequant_rows": ("quantize.cu",) + _COMMON_SOURCES,
+    "rht_quant_sr": ("rht.cu",) + _COMMON_SOURCES,
+    "osc_update": ("osc.cu",) + _COMMON_SOURCES,
+    "osc_step": ("osc.cu",) + _COMMON_SOURCES,
+}
 
 
-def kernel_source_digest():
+def kernel_source_digest(op):
     import hashlib
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "mxfp4_block_quantization_quantizer_b200", "csrc")
-    for name in TRAFFIC_SOURCES:
+    for name in OP_SOURCES[op]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:12]
@@ -105,7 +114,7 @@ def measured_traffic(op):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    digest = kernel_source_digest()
+    digest = kernel_source_digest(op)
     for line in lines:
         parts = line.split()
         if len(parts) >= 3 and parts[0] == op and parts[2] == "src=" + digest:
