@@ -245,23 +245,30 @@ __global__ void __launch_bounds__(kGThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Pipelined version (K a multiple of 256): TMA loads in the 128-byte swizzled
-// K-major layout, a kPS-stage ring of full/empty mbarriers, warp roles.
+// Pipelined, persistent version (K a multiple of 256): one CTA per SM loops
+// over 128 x 256 tiles of C. TMA loads in the 128-byte swizzled K-major
+// layout through a kPS-stage ring of full/empty mbarriers; warp roles:
 //   warp 0: one thread issues the tensor-memory-access (TMA) loads of A and B
-//           and the bulk copies of their scale tiles into a free stage;
-//   warp 1: allocates tensor memory; one thread copies each stage's scales
-//           into tensor memory and issues the MMAs, whose completion
-//           (tcgen05.commit) frees the stage;
-//   warps 2-5: epilogue, one lane quarter (32 accumulator rows) each.
-// The C tile is 128 x 256: one M = 128, N = 256 MMA per K = 64 step.
+//           and the bulk copies of their scale tiles into a free stage, tile
+//           after tile without pause;
+//   warp 1: allocates tensor memory; one thread waits until the epilogue has
+//           read the accumulator, then per stage copies the scales into
+//           tensor memory and issues one M = 128, N = 256 MMA per K = 64
+//           step, whose completion (tcgen05.commit) frees the stage, and
+//           finally commits the tile to the epilogue;
+//   warps 2-9: epilogue, two warps per lane quarter (32 accumulator rows),
+//           128 columns each held in registers: the accumulator is released
+//           as soon as it is read and the stores of C overlap the next
+//           tile's main loop.
 // ---------------------------------------------------------------------------
 
-constexpr int kPS = 4;            // pipeline stages
+constexpr int kPS = 3;            // pipeline stages
 // kind::mxf4 instruction descriptor for M = 128, N = 256
 constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
                                 (1u << 23) | (uint32_t(kGM >> 4) << 24);
 constexpr int kPN = 256;          // C tile columns
-constexpr int kPThreads = 192;
+constexpr int kPEpiWarps = 8;
+constexpr int kPThreads = 32 * (2 + kPEpiWarps);
 constexpr uint32_t kPTmemCols = 512;
 constexpr uint32_t kPSfCol = 256;  // per stage: 8 SFA columns, then 16 SFB
 constexpr uint32_t kPSfStride = 24;
@@ -269,9 +276,10 @@ constexpr uint32_t kPSfStride = 24;
 struct __align__(1024) PipeSmem {
   uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
   uint8_t b[kPS][kPN][128];
+  uint8_t epi[kPEpiWarps][32][128];  // per epilogue warp: 32 rows x 32 fp32, 128B-swizzled
   uint8_t sfa[kPS][2][512];       // 2 blocked tiles (256 K elements)
   uint8_t sfb[kPS][2][2][512];    // [128-row block][K tile]
-  unsigned long long full[kPS], empty[kPS], acc_full;
+  unsigned long long full[kPS], empty[kPS], acc_full, acc_empty;
   uint32_t tmem_base;
   int failed;
 };
@@ -312,6 +320,27 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// TMA store of a 2-D box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y,
+                                             const void* src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_u32(src))
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until every committed bulk store of this thread has finished reading
+// its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ bool failed_flag(const int* f) {
   return *static_cast<const volatile int*>(f) != 0;
 }
@@ -325,6 +354,7 @@ __device__ __forceinline__ void commit_to(unsigned long long* bar) {
 __global__ void __launch_bounds__(kPThreads, 1)
     k_gemm_mxf4_pipe(const __grid_constant__ CUtensorMap tm_a,
                      const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_c, bool tma_store,
                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                      int64_t m, int64_t n, int64_t k, float* __restrict__ c) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -333,10 +363,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   PipeSmem& sm = *reinterpret_cast<PipeSmem*>(
       smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t m0 = int64_t(blockIdx.y) * kGM, n0 = int64_t(blockIdx.x) * kPN;
   const int64_t k_tiles = k / 128;
   const int64_t n_kb = k / 256;
   const int64_t n_row_tiles = (n + 127) / 128;
+  const int64_t m_tiles = (m + kGM - 1) / kGM;
+  const int64_t n_tiles = m_tiles * ((n + kPN - 1) / kPN);
 
   if (tid == 0) {
     for (int s = 0; s < kPS; ++s) {
@@ -344,6 +375,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.empty[s])));
     }
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.acc_full)));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.acc_empty)),
+                 "r"(kPEpiWarps));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     sm.failed = 0;
   }
@@ -357,109 +390,160 @@ __global__ void __launch_bounds__(kPThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;");
   const uint32_t tmem = sm.tmem_base;
 
+  // Tiles in M-fastest order, CTA i taking tiles i, i + grid, ...: the CTAs
+  // running at one time share B's rows and stream all of A once.
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t kb = 0; kb < n_kb; ++kb) {
-        const int s = int(kb % kPS);
-        const uint32_t ph = uint32_t((kb / kPS) & 1);
-        if (!wait_parity(&sm.empty[s], ph ^ 1u) || failed_flag(&sm.failed)) {
-          atomicExch(&sm.failed, 1);
-          break;
-        }
+      int64_t it = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int64_t m0 = (tile % m_tiles) * kGM, n0 = (tile / m_tiles) * kPN;
         const int64_t rb = n0 / 128;
         const bool half1 = rb + 1 < n_row_tiles;
-        const uint32_t bytes = kGM * 128 + kPN * 128 + 1024 + (half1 ? 2048 : 1024);
-        expect_tx(&sm.full[s], bytes);
-        tma_load_2d(&sm.a[s][0][0], &tm_a, int(kb * 128), int(m0), &sm.full[s]);
-        tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb * 128), int(n0), &sm.full[s]);
-        bulk_load(&sm.sfa[s][0][0], sfa + ((m0 / 128) * k_tiles + 2 * kb) * 512, 1024,
-                  &sm.full[s]);
-        bulk_load(&sm.sfb[s][0][0][0], sfb + (rb * k_tiles + 2 * kb) * 512, 1024,
-                  &sm.full[s]);
-        if (half1)
-          bulk_load(&sm.sfb[s][1][0][0], sfb + ((rb + 1) * k_tiles + 2 * kb) * 512, 1024,
+        for (int64_t kb = 0; kb < n_kb; ++kb, ++it) {
+          const int s = int(it % kPS);
+          const uint32_t ph = uint32_t((it / kPS) & 1);
+          if (!wait_parity(&sm.empty[s], ph ^ 1u) || failed_flag(&sm.failed)) {
+            atomicExch(&sm.failed, 1);
+            tile = n_tiles;
+            break;
+          }
+          const uint32_t bytes = kGM * 128 + kPN * 128 + 1024 + (half1 ? 2048 : 1024);
+          expect_tx(&sm.full[s], bytes);
+          tma_load_2d(&sm.a[s][0][0], &tm_a, int(kb * 128), int(m0), &sm.full[s]);
+          tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb * 128), int(n0), &sm.full[s]);
+          bulk_load(&sm.sfa[s][0][0], sfa + ((m0 / 128) * k_tiles + 2 * kb) * 512, 1024,
                     &sm.full[s]);
+          bulk_load(&sm.sfb[s][0][0][0], sfb + (rb * k_tiles + 2 * kb) * 512, 1024,
+                    &sm.full[s]);
+          if (half1)
+            bulk_load(&sm.sfb[s][1][0][0], sfb + ((rb + 1) * k_tiles + 2 * kb) * 512, 1024,
+                      &sm.full[s]);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int64_t kb = 0; kb < n_kb; ++kb) {
-        const int s = int(kb % kPS);
-        const uint32_t ph = uint32_t((kb / kPS) & 1);
-        if (!wait_parity(&sm.full[s], ph) || failed_flag(&sm.failed)) {
+      int64_t it = 0, ti = 0;
+      const uint32_t sf = tmem + kPSfCol;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
+        // the epilogue has read the previous tile's accumulator
+        if (!wait_parity(&sm.acc_empty, uint32_t(ti & 1) ^ 1u) || failed_flag(&sm.failed)) {
           atomicExch(&sm.failed, 1);
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;");
-        const uint32_t sf = tmem + kPSfCol + kPSfStride * uint32_t(s);
-        // scale factors in tensor memory: row r of an operand in lane r % 32,
-        // 32-bit column r / 32 (A: 4 columns per K tile; B, 256 rows: 8,
-        // its two 128-row tiles side by side), one byte per 32-element group
+        bool ok = true;
+        for (int64_t kb = 0; kb < n_kb; ++kb, ++it) {
+          const int s = int(it % kPS);
+          const uint32_t ph = uint32_t((it / kPS) & 1);
+          if (!wait_parity(&sm.full[s], ph) || failed_flag(&sm.failed)) {
+            atomicExch(&sm.failed, 1);
+            ok = false;
+            break;
+          }
+          asm volatile("tcgen05.fence::after_thread_sync;");
+          // scale factors in tensor memory: row r of an operand in lane r % 32,
+          // 32-bit column r / 32 (A: 4 columns per K tile; B, 256 rows: 8,
+          // its two 128-row tiles side by side), one byte per 32-element
+          // group; tensor-core operations of one thread run in order, so the
+          // next stage's copy may reuse the columns
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          copy_scales_to_tmem(sf + 4 * j, &sm.sfa[s][j][0]);
-          copy_scales_to_tmem(sf + 8 + 8 * j, &sm.sfb[s][0][j][0]);
-          copy_scales_to_tmem(sf + 8 + 8 * j + 4, &sm.sfb[s][1][j][0]);
-        }
+          for (int j = 0; j < 2; ++j) {
+            copy_scales_to_tmem(sf + 4 * j, &sm.sfa[s][j][0]);
+            copy_scales_to_tmem(sf + 8 + 8 * j, &sm.sfb[s][0][j][0]);
+            copy_scales_to_tmem(sf + 8 + 8 * j + 4, &sm.sfb[s][1][j][0]);
+          }
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t sf_id = 2u * (t & 1);
-          const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
-          const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
-          const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
-          mma_mxf4(tmem, smem_desc_sw128(&sm.a[s][0][32 * t]),
-                   smem_desc_sw128(&sm.b[s][0][32 * t]), idesc,
-                   (kb > 0 || t > 0) ? 1u : 0u, tsfa, tsfb);
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t sf_id = 2u * (t & 1);
+            const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
+            const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
+            const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
+            mma_mxf4(tmem, smem_desc_sw128(&sm.a[s][0][32 * t]),
+                     smem_desc_sw128(&sm.b[s][0][32 * t]), idesc,
+                     (kb > 0 || t > 0) ? 1u : 0u, tsfa, tsfb);
+          }
+          commit_to(&sm.empty[s]);
         }
-        commit_to(&sm.empty[s]);
+        commit_to(&sm.acc_full);
+        if (!ok) break;
       }
-      commit_to(&sm.acc_full);
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;  // lane quarter this warp may read
-    const bool ok = wait_parity(&sm.acc_full, 0);
-    if (!ok) atomicExch(&sm.failed, 1);
-    asm volatile("tcgen05.fence::after_thread_sync;");
-    const bool failed = !ok || failed_flag(&sm.failed);
-    const int64_t row = m0 + 32 * q + lane;
-#pragma unroll 1
-    for (int cb = 0; cb < kPN / 32; ++cb) {
-      uint32_t v[32];
-      const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + 32 * cb;
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
-          "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
-          "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]),
-            "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]),
-            "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-            "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-            "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-            "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
-            "=r"(v[30]), "=r"(v[31])
-          : "r"(taddr));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      const int64_t col = n0 + 32 * cb;
-      if (row < m && col < n) {
-        float* out = c + row * n + col;
-        if (col + 32 <= n && (n & 3) == 0) {
+    // epilogue: 8 warps, two per lane quarter, each taking 128 of the 256
+    // columns into registers; the accumulator is released as soon as they
+    // are read, and the stores overlap the next tile's main loop
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    int64_t ti = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
+      const int64_t m0 = (tile % m_tiles) * kGM, n0 = (tile / m_tiles) * kPN;
+      const bool ok = wait_parity(&sm.acc_full, uint32_t(ti & 1));
+      if (!ok) atomicExch(&sm.failed, 1);
+      asm volatile("tcgen05.fence::after_thread_sync;");
+      uint32_t v[128];
+      const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + 128u * uint32_t(half);
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(out + j) =
-                failed ? make_float4(__uint_as_float(kNaNf32), __uint_as_float(kNaNf32),
-                                     __uint_as_float(kNaNf32), __uint_as_float(kNaNf32))
-                       : make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                     __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col + j < n) out[j] = failed ? __uint_as_float(kNaNf32) : __uint_as_float(v[j]);
-        }
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t* d = v + 32 * cb;
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
+            "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
+            "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]),
+              "=r"(d[5]), "=r"(d[6]), "=r"(d[7]), "=r"(d[8]), "=r"(d[9]),
+              "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]),
+              "=r"(d[15]), "=r"(d[16]), "=r"(d[17]), "=r"(d[18]), "=r"(d[19]),
+              "=r"(d[20]), "=r"(d[21]), "=r"(d[22]), "=r"(d[23]), "=r"(d[24]),
+              "=r"(d[25]), "=r"(d[26]), "=r"(d[27]), "=r"(d[28]), "=r"(d[29]),
+              "=r"(d[30]), "=r"(d[31])
+            : "r"(tbase + 32u * uint32_t(cb)));
       }
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;");
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sm.acc_empty))
+                     : "memory");
+      const bool failed = !ok || failed_flag(&sm.failed);
+      if (failed) {
+#pragma unroll
+        for (int j = 0; j < 128; ++j) v[j] = kNaNf32;
+      }
+      const int64_t row = m0 + 32 * q + lane;
+      const int64_t col0 = n0 + 128 * half;
+      if (tma_store) {
+        // 4 boxes of 32 x 32 fp32 through this warp's staging tile: lane r
+        // writes row r, 16-byte chunk j at chunk position j ^ (r % 8) (the
+        // 128-byte swizzle the tensor map undoes; conflict-free), then lane 0
+        // stores the box; the tile is rewritten once the store has read it
+        uint8_t* tile = &sm.epi[warp - 2][0][0];
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(tile + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(v[32 * cb + 4 * j], v[32 * cb + 4 * j + 1],
+                           v[32 * cb + 4 * j + 2], v[32 * cb + 4 * j + 3]);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0 && col0 + 32 * cb < n && m0 + 32 * q < m)
+            tma_store_2d(&tm_c, int(col0 + 32 * cb), int(m0 + 32 * q), tile);
+        }
+      } else if (row < m && col0 < n) {
+        float* out = c + row * n + col0;
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+          if (col0 + j < n) out[j] = __uint_as_float(v[j]);
+      }
+      if (!ok) break;
     }
   }
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // C stores complete
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
   if (warp == 1)
@@ -500,6 +584,21 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
          CUDA_SUCCESS;
 }
 
+// 2-D map over fp32 C [m][n] for the epilogue's stores: 32 x 32 boxes,
+// 128-byte swizzle (the staging tiles' layout).
+bool encode_c_map(CUtensorMap* map, float* c, int64_t m, int64_t n) {
+  auto enc = tensor_map_encoder();
+  if (!enc || n % 4) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(n), cuuint64_t(m)};
+  const cuuint64_t strides[1] = {cuuint64_t(n) * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
@@ -507,16 +606,20 @@ cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
                              int64_t m, int64_t n, int64_t k, float* c,
                              cudaStream_t s) {
   if (k % 256 == 0) {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, mb, mc;
     if (encode_codes_map(&ma, a, m, k, kGM) && encode_codes_map(&mb, b, n, k, kPN)) {
+      const bool tma_store = encode_c_map(&mc, c, m, n);
+      if (!tma_store) mc = ma;  // unused
       constexpr size_t smem = sizeof(PipeSmem) + 1024;
       cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k_gemm_mxf4_pipe),
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            int(smem));
       if (e != cudaSuccess) return e;
-      const dim3 grid(unsigned((n + kPN - 1) / kPN), unsigned((m + kGM - 1) / kGM));
-      k_gemm_mxf4_pipe<<<grid, kPThreads, smem, s>>>(ma, mb, a_scales, b_scales, m, n, k,
-                                                     c);
+      const int64_t tiles = ((m + kGM - 1) / kGM) * ((n + kPN - 1) / kPN);
+      const int grid = persistent_grid(reinterpret_cast<const void*>(k_gemm_mxf4_pipe),
+                                       kPThreads, smem, tiles);
+      k_gemm_mxf4_pipe<<<grid, kPThreads, smem, s>>>(ma, mb, mc, tma_store, a_scales,
+                                                     b_scales, m, n, k, c);
       return cudaGetLastError();
     }
   }
