@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kGThreads)
 //           tile's main loop.
 // ---------------------------------------------------------------------------
 
-constexpr int kPS = 3;            // pipeline stages
+constexpr int kPS = 4;            // pipeline stages
 // kind::mxf4 instruction descriptor for M = 128, N = 256
 constexpr uint32_t kIdescN256 = (1u << 7) | (1u << 10) | (uint32_t(256 >> 3) << 17) |
                                 (1u << 23) | (uint32_t(kGM >> 4) << 24);
@@ -276,7 +276,7 @@ constexpr uint32_t kPSfStride = 24;
 struct __align__(1024) PipeSmem {
   uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
   uint8_t b[kPS][kPN][128];
-  uint8_t epi[kPEpiWarps][32][128];  // per epilogue warp: 32 rows x 32 fp32, 128B-swizzled
+  uint8_t epi[kPEpiWarps][32][64];   // per epilogue warp: 32 rows x 16 fp32, 64B-swizzled
   uint8_t sfa[kPS][2][512];       // 2 blocked tiles (256 K elements)
   uint8_t sfb[kPS][2][2][512];    // [128-row block][K tile]
   unsigned long long full[kPS], empty[kPS], acc_full, acc_empty;
@@ -515,24 +515,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const int64_t row = m0 + 32 * q + lane;
       const int64_t col0 = n0 + 128 * half;
       if (tma_store) {
-        // 4 boxes of 32 x 32 fp32 through this warp's staging tile: lane r
-        // writes row r, 16-byte chunk j at chunk position j ^ (r % 8) (the
-        // 128-byte swizzle the tensor map undoes; conflict-free), then lane 0
-        // stores the box; the tile is rewritten once the store has read it
+        // 8 boxes of 32 rows x 16 fp32 through this warp's 2 KB staging
+        // tile: lane r writes row r, 16-byte chunk j at chunk position
+        // j ^ ((r / 2) % 4) (the 64-byte swizzle the tensor map undoes;
+        // conflict-free), then lane 0 stores the box; the tile is rewritten
+        // once the store has read it
         uint8_t* tile = &sm.epi[warp - 2][0][0];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 0; cb < 8; ++cb) {
           if (lane == 0) bulk_wait_read();
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint4*>(tile + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                make_uint4(v[32 * cb + 4 * j], v[32 * cb + 4 * j + 1],
-                           v[32 * cb + 4 * j + 2], v[32 * cb + 4 * j + 3]);
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(tile + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(v[16 * cb + 4 * j], v[16 * cb + 4 * j + 1],
+                           v[16 * cb + 4 * j + 2], v[16 * cb + 4 * j + 3]);
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           __syncwarp();
-          if (lane == 0 && col0 + 32 * cb < n && m0 + 32 * q < m)
-            tma_store_2d(&tm_c, int(col0 + 32 * cb), int(m0 + 32 * q), tile);
+          if (lane == 0 && col0 + 16 * cb < n && m0 + 32 * q < m)
+            tma_store_2d(&tm_c, int(col0 + 16 * cb), int(m0 + 32 * q), tile);
         }
       } else if (row < m && col0 < n) {
         float* out = c + row * n + col0;
@@ -584,17 +585,17 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int6
          CUDA_SUCCESS;
 }
 
-// 2-D map over fp32 C [m][n] for the epilogue's stores: 32 x 32 boxes,
-// 128-byte swizzle (the staging tiles' layout).
+// 2-D map over fp32 C [m][n] for the epilogue's stores: boxes of 32 rows x
+// 16 columns, 64-byte swizzle (the staging tiles' layout).
 bool encode_c_map(CUtensorMap* map, float* c, int64_t m, int64_t n) {
   auto enc = tensor_map_encoder();
   if (!enc || n % 4) return false;
   const cuuint64_t dims[2] = {cuuint64_t(n), cuuint64_t(m)};
   const cuuint64_t strides[1] = {cuuint64_t(n) * 4};
-  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t box[2] = {16, 32};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, c, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
