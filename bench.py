@@ -517,6 +517,26 @@ def run_ours(args):
                                   "launches": args.steps}
         del qw, qe, qout
 
+        # the overflow-aware scale rule on the sweep (ROWS, RNE)
+        oout = (u8(R, C // 2), u8(R, C // 32))
+        for _ in range(args.warmup):
+            m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)
+        oev = []
+        for _ in range(args.steps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)
+            b.record(stream)
+            oev.append((a, b))
+        torch.cuda.synchronize(dev)
+        d = statistics.mean(a.elapsed_time(b) for a, b in oev) * 1e-3
+        d = reduce_max(d, world, dev)
+        nbytes = BYTES_PER_ELEM["quant_rows_rne"] * R * C
+        next_ops["quant_rows_rne_oas"] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9,
+                                          "bytes": nbytes, "shape": [R, C],
+                                          "launches": args.steps}
+        del oout
+
         # MXFP4 GEMM on the block-scaled tensor cores, consuming the step's
         # ROWS codes of the sweep as the activation operand
         gM, gN, gK = NEXT_OPS["gemm_mxf4"][1]

@@ -95,6 +95,21 @@ mxfp4_status mxfp4_quantize(const void* x, int dtype, int64_t rows,
                             void* stream);
 
 /*
+ * mxfp4_quantize with the overflow-aware scale: e is the smallest exponent
+ * with absmax * 2^-e <= 6 (instead of floor(log2 absmax) - 2), so no element
+ * saturates and stochastic rounding is unbiased for every input; e is the
+ * OCP exponent, or one more where the OCP-scaled maximum exceeds 6. Same
+ * arguments, layouts, statuses and non-finite handling as mxfp4_quantize.
+ * Source: "Unveiling the Potential of Quantization with MXFP4", abstract
+ * (overflow-aware scaling under power-of-two block scales); the page gives
+ * the idea, not a formula, so the rule above is a reading.
+ */
+mxfp4_status mxfp4_quantize_oas(const void* x, int dtype, int64_t rows,
+                                int64_t cols, int axis, int rounding,
+                                uint64_t seed, uint8_t* codes, uint8_t* scales,
+                                void* stream);
+
+/*
  * Decode codes and scales back to values: y = (-1)^sign * G[m] * 2^e, exact
  * in bf16 and fp32 (a scale byte of 0xFF decodes to NaN).
  * Source: ALTO explainer, Jargon: MXFP4 (a block of 32 4-bit values sharing

@@ -19,7 +19,8 @@ ROWS, COLS = 0, 1
 RNE, SR = 0, 1
 
 # Every symbol include/mxfp4.h declares.
-SYMBOLS = ("mxfp4_quantize", "mxfp4_dequantize", "mxfp4_double_quantize",
+SYMBOLS = ("mxfp4_quantize", "mxfp4_quantize_oas", "mxfp4_dequantize",
+           "mxfp4_double_quantize",
            "mxfp4_rht_quantize", "mxfp4_osc_step",
            "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
            "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_status_string")
@@ -49,6 +50,7 @@ def lib():
                                   ctypes.c_int)
         sig = {
             "mxfp4_quantize": [vp, i32, i64, i64, i32, i32, u64, vp, vp, vp],
+            "mxfp4_quantize_oas": [vp, i32, i64, i64, i32, i32, u64, vp, vp, vp],
             "mxfp4_dequantize": [vp, vp, i64, i64, i32, vp, i32, vp],
             "mxfp4_double_quantize": [vp, i32, i64, i64, u64, vp, vp, vp, vp,
                                       vp],
@@ -110,10 +112,11 @@ def _empty_u8(shape, device):
     return torch.empty(shape, dtype=torch.uint8, device=device)
 
 
-def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None):
-    """mxfp4_quantize: returns (codes, scales) in the layout of `axis`:
-    ROWS -> codes [R, C/2], scales [R, C/32]; COLS -> codes [C, R/2],
-    scales [C, R/32]."""
+def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None,
+             oas=False):
+    """mxfp4_quantize (mxfp4_quantize_oas with oas=True): returns (codes,
+    scales) in the layout of `axis`: ROWS -> codes [R, C/2], scales
+    [R, C/32]; COLS -> codes [C, R/2], scales [C, R/32]."""
     _cuda2d(x, "x")
     R, C = x.shape
     if out is None:
@@ -121,9 +124,9 @@ def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None):
         shape_s = (R, C // 32) if axis == ROWS else (C, R // 32)
         out = (_empty_u8(shape_c, x.device), _empty_u8(shape_s, x.device))
     codes, scales = out
-    _check(lib().mxfp4_quantize(_ptr(x), _dtype_code(x), R, C, axis, rounding,
-                                seed, _ptr(codes), _ptr(scales),
-                                _stream(x.device, stream)), "mxfp4_quantize")
+    fn = lib().mxfp4_quantize_oas if oas else lib().mxfp4_quantize
+    _check(fn(_ptr(x), _dtype_code(x), R, C, axis, rounding, seed, _ptr(codes),
+              _ptr(scales), _stream(x.device, stream)), "mxfp4_quantize")
     return codes, scales
 
 
@@ -265,6 +268,12 @@ def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None):
 
 # The C names, for callers that prefer them.
 mxfp4_quantize = quantize
+
+
+def mxfp4_quantize_oas(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None):
+    return quantize(x, axis, rounding, seed, out, stream, oas=True)
+
+
 mxfp4_dequantize = dequantize
 mxfp4_double_quantize = double_quantize
 mxfp4_rht_quantize = rht_quantize

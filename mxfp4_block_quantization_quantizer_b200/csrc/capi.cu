@@ -35,10 +35,12 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-mxfp4_status mxfp4_quantize(const void* x, int dtype, int64_t rows,
-                            int64_t cols, int axis, int rounding,
-                            uint64_t seed, uint8_t* codes, uint8_t* scales,
-                            void* stream) {
+namespace {
+
+mxfp4_status quantize_with_rule(const void* x, int dtype, int64_t rows,
+                                int64_t cols, int axis, int rounding,
+                                uint64_t seed, uint8_t* codes,
+                                uint8_t* scales, void* stream, bool oas) {
   if (!dtype_ok(dtype) || !axis_ok(axis) || !rounding_ok(rounding))
     return MXFP4_ERR_ENUM;
   if (!x || !codes || !scales) return MXFP4_ERR_NULL;
@@ -48,9 +50,29 @@ mxfp4_status mxfp4_quantize(const void* x, int dtype, int64_t rows,
   const bool bf16 = dtype == MXFP4_BF16, sr = rounding == MXFP4_SR;
   if (axis == MXFP4_ROWS)
     return from_cuda(mxfp4::launch_quant_rows(x, bf16, rows, cols, sr, seed,
-                                              codes, scales, as_stream(stream)));
+                                              codes, scales, as_stream(stream),
+                                              oas));
   return from_cuda(mxfp4::launch_quant_cols(x, bf16, rows, cols, sr, seed,
-                                            codes, scales, as_stream(stream)));
+                                            codes, scales, as_stream(stream),
+                                            oas));
+}
+
+}  // namespace
+
+mxfp4_status mxfp4_quantize(const void* x, int dtype, int64_t rows,
+                            int64_t cols, int axis, int rounding,
+                            uint64_t seed, uint8_t* codes, uint8_t* scales,
+                            void* stream) {
+  return quantize_with_rule(x, dtype, rows, cols, axis, rounding, seed, codes,
+                            scales, stream, false);
+}
+
+mxfp4_status mxfp4_quantize_oas(const void* x, int dtype, int64_t rows,
+                                int64_t cols, int axis, int rounding,
+                                uint64_t seed, uint8_t* codes, uint8_t* scales,
+                                void* stream) {
+  return quantize_with_rule(x, dtype, rows, cols, axis, rounding, seed, codes,
+                            scales, stream, true);
 }
 
 mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales,

@@ -12,13 +12,16 @@ namespace mxfp4 {
 int persistent_grid(const void* kernel, int threads, size_t smem,
                     int64_t work_blocks);
 
+// oas: the overflow-aware scale rule instead of the OCP one.
 cudaError_t launch_quant_rows(const void* x, bool bf16, int64_t rows,
                               int64_t cols, bool sr, uint64_t seed,
-                              uint8_t* codes, uint8_t* scales, cudaStream_t s);
+                              uint8_t* codes, uint8_t* scales, cudaStream_t s,
+                              bool oas = false);
 
 cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
                               int64_t cols, bool sr, uint64_t seed,
-                              uint8_t* codes, uint8_t* scales, cudaStream_t s);
+                              uint8_t* codes, uint8_t* scales, cudaStream_t s,
+                              bool oas = false);
 
 // Flat decode of n_groups groups (rows of the output are contiguous runs of
 // whole groups in both layouts).

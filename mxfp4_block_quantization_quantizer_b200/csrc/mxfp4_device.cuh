@@ -99,9 +99,23 @@ __device__ __forceinline__ uint32_t scale_byte(uint32_t abs_bits) {
   return abs_bits >= 0x7F800000u ? 0xFFu : (E > 2u ? E - 2u : 0u);
 }
 
-// 2^-e as fp32 for byte sb = e + 127 <= 252: biased exponent 254 - sb.
+// Overflow-aware variant ("Unveiling the Potential of Quantization with
+// MXFP4", abstract: overflow-aware scaling): the smallest e with
+// absmax 2^-e <= 6. The OCP exponent leaves absmax 2^-e in [4, 8); it moves
+// up by one exactly when that exceeds 6, i.e. when the mantissa of absmax is
+// above 1.5 (mantissa field > 0x400000). Below the exponent field 2 the OCP
+// byte is clamped at 0 and the scaled maximum stays under 4.
+__device__ __forceinline__ uint32_t scale_byte_oas(uint32_t abs_bits) {
+  const uint32_t sb = scale_byte(abs_bits);
+  const bool up = abs_bits >= (2u << 23) && abs_bits < 0x7F800000u &&
+                  (abs_bits & 0x7FFFFFu) > 0x400000u;
+  return sb + (up ? 1u : 0u);
+}
+
+// 2^-e as fp32 for byte sb = e + 127 <= 253 (the OCP rule reaches 252, the
+// overflow-aware one 253): biased exponent 254 - sb, normal throughout.
 __device__ __forceinline__ float inv_scale(uint32_t sb) {
-  uint32_t b = sb > 252u ? 252u : sb;
+  uint32_t b = sb > 253u ? 253u : sb;
   return __uint_as_float((254u - b) << 23);
 }
 

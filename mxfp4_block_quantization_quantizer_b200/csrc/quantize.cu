@@ -34,7 +34,7 @@ namespace {
 
 constexpr int kRowThreads = 256;
 
-template <bool BF16, bool SR, int U>
+template <bool BF16, bool SR, int U, bool OAS = false>
 __global__ void __launch_bounds__(kRowThreads)
     k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey key,
                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kRowThreads)
       }
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      const uint32_t sb = scale_byte(amax);
+      const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
       const float mul = inv_scale(sb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[u][j] *= mul;
@@ -164,14 +164,15 @@ struct ColPair {
 // Quantize the two adjacent columns c0, c0+1 over the 32 rows r0 .. r0+31.
 // get(j) returns the values of row r0+j (x: column c0, y: column c0+1); ma
 // and mb are the fp32 bit patterns of the two columns' absolute maxima.
-template <bool SR, bool EVEN, bool BIG, bool SAT = true, typename Get>
+template <bool SR, bool EVEN, bool BIG, bool SAT = true, bool OAS = false,
+          typename Get>
 __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
                                                      uint32_t mb, int64_t r0,
                                                      int64_t c0, int64_t cols,
                                                      RngKey key) {
   ColPair o;
-  o.sa = scale_byte(ma);
-  o.sb = scale_byte(mb);
+  o.sa = OAS ? scale_byte_oas(ma) : scale_byte(ma);
+  o.sb = OAS ? scale_byte_oas(mb) : scale_byte(mb);
   const float mula = inv_scale(o.sa), mulb = inv_scale(o.sb);
 #pragma unroll
   for (int q = 0; q < 4; ++q) o.wa[q] = o.wb[q] = 0;
@@ -280,7 +281,7 @@ __device__ __forceinline__ void store_staged_columns(
 // the caller checks tile_r + 32rg < rows). The tile is read twice (maxima,
 // then codes) rather than held in registers. A warp reads 32 consecutive
 // 32-bit words (bf16) or 64-bit words (fp32) of one row: no bank conflicts.
-template <bool BF16, bool SR, bool EVEN, bool BIG>
+template <bool BF16, bool SR, bool EVEN, bool BIG, bool OAS = false>
 __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
                                                     int kcols, int rg, int cp,
                                                     int64_t tile_r,
@@ -295,7 +296,7 @@ __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
     for (int j = 0; j < 32; ++j) m = umax16x2(m, s[j * (kcols / 2)] & 0x7FFF7FFFu);
     ma = m << 16;
     mb = m & 0xFFFF0000u;
-    return column_pair_codes<SR, EVEN, BIG>(
+    return column_pair_codes<SR, EVEN, BIG, true, OAS>(
         [&](int j) {
           const uint32_t w = s[j * (kcols / 2)];
           return make_float2(bf16_lo(w), bf16_hi(w));
@@ -309,7 +310,7 @@ __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
     ma = max(ma, __float_as_uint(w.x) & 0x7FFFFFFFu);
     mb = max(mb, __float_as_uint(w.y) & 0x7FFFFFFFu);
   }
-  return column_pair_codes<SR, EVEN, BIG>([&](int j) { return s[j * (kcols / 2)]; },
+  return column_pair_codes<SR, EVEN, BIG, true, OAS>([&](int j) { return s[j * (kcols / 2)]; },
                                           ma, mb, r0, tile_c + 2 * cp, cols, key);
 }
 
@@ -380,7 +381,7 @@ __device__ __forceinline__ void stage_tile_async(const void* __restrict__ x,
 }
 
 // Column groups, general shapes: one staged tile at a time, plain loads.
-template <bool BF16, bool SR, bool EVEN, bool BIG>
+template <bool BF16, bool SR, bool EVEN, bool BIG, bool OAS = false>
 __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     k_quant_cols(const void* __restrict__ x, int64_t rows, int64_t cols,
                  RngKey key, uint8_t* __restrict__ codes,
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
     __syncthreads();
     const int64_t r0 = tile_r + 32 * rg;
     if (r0 < rows)
-      store_column_pair(column_tile_pass<BF16, SR, EVEN, BIG>(
+      store_column_pair(column_tile_pass<BF16, SR, EVEN, BIG, OAS>(
                             tile, T::kCols, rg, cp, tile_r, tile_c, cols, key),
                         r0, tile_c + 2 * cp, rows, cols, codes, scales);
     __syncthreads();
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
 // Column groups, 16-byte aligned rows: double-buffered. The copies of the
 // CTA's next tile are in flight while the current tile is quantized; the
 // tile's column codes are staged and leave as whole 64-byte runs.
-template <bool BF16, bool SR, bool EVEN, bool BIG>
+template <bool BF16, bool SR, bool EVEN, bool BIG, bool OAS = false>
 __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
     k_quant_cols_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
                       RngKey key, uint8_t* __restrict__ codes,
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
     const int64_t tile_r = (t / tiles_c) * kTileRows;
     const int64_t tile_c = (t % tiles_c) * T::kCols;
     if (tile_r + 32 * rg < rows)
-      stage_column_pair(column_tile_pass<BF16, SR, EVEN, BIG>(
+      stage_column_pair(column_tile_pass<BF16, SR, EVEN, BIG, OAS>(
                             smem + buf * kChunks, T::kCols, rg, cp, tile_r,
                             tile_c, cols, key),
                         cp, rg, s_col, s_sc);
@@ -784,12 +785,12 @@ int persistent_grid(const void* kernel, int threads, size_t smem,
   return static_cast<int>(g < 1 ? 1 : g);
 }
 
-template <bool BF16, bool SR>
+template <bool BF16, bool SR, bool OAS>
 static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
   constexpr int U = BF16 ? 4 : 2;  // 8 lowers occupancy and runs slower
-  auto kern = k_quant_rows<BF16, SR, U>;
+  auto kern = k_quant_rows<BF16, SR, U, OAS>;
   const int64_t groups_per_block = (kRowThreads / 4) * U;
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
                                    kRowThreads, 0,
@@ -799,20 +800,28 @@ static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
   return cudaGetLastError();
 }
 
+template <bool OAS>
+static cudaError_t quant_rows_rule(const void* x, bool bf16, int64_t n_groups,
+                                   bool sr, RngKey key, uint8_t* codes,
+                                   uint8_t* scales, cudaStream_t s) {
+  if (bf16)
+    return sr ? quant_rows_impl<true, true, OAS>(x, n_groups, key, codes, scales, s)
+              : quant_rows_impl<true, false, OAS>(x, n_groups, key, codes, scales, s);
+  return sr ? quant_rows_impl<false, true, OAS>(x, n_groups, key, codes, scales, s)
+            : quant_rows_impl<false, false, OAS>(x, n_groups, key, codes, scales, s);
+}
+
 cudaError_t launch_quant_rows(const void* x, bool bf16, int64_t rows,
                               int64_t cols, bool sr, uint64_t seed,
                               uint8_t* codes, uint8_t* scales,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool oas) {
   const int64_t n_groups = rows * cols / kGroup;
   const RngKey key = make_key(seed, 0);
-  if (bf16)
-    return sr ? quant_rows_impl<true, true>(x, n_groups, key, codes, scales, s)
-              : quant_rows_impl<true, false>(x, n_groups, key, codes, scales, s);
-  return sr ? quant_rows_impl<false, true>(x, n_groups, key, codes, scales, s)
-            : quant_rows_impl<false, false>(x, n_groups, key, codes, scales, s);
+  return oas ? quant_rows_rule<true>(x, bf16, n_groups, sr, key, codes, scales, s)
+             : quant_rows_rule<false>(x, bf16, n_groups, sr, key, codes, scales, s);
 }
 
-template <bool BF16, bool SR, bool VEC, bool EVEN, bool BIG>
+template <bool BF16, bool SR, bool VEC, bool EVEN, bool BIG, bool OAS>
 static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
@@ -820,7 +829,7 @@ static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + T::kCols - 1) / T::kCols);
   if (VEC) {
-    auto kern = k_quant_cols_pipe<BF16, SR, EVEN, BIG>;
+    auto kern = k_quant_cols_pipe<BF16, SR, EVEN, BIG, OAS>;
     constexpr size_t smem = 2 * kTileRows * T::kChunksPerRow * sizeof(uint4) +
                             ColStage<T::kCols>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(
@@ -831,7 +840,7 @@ static cudaError_t quant_cols_impl(const void* x, int64_t rows, int64_t cols,
                                      T::kThreads, smem, n_tiles);
     kern<<<grid, T::kThreads, smem, s>>>(x, rows, cols, key, codes, scales);
   } else {
-    auto kern = k_quant_cols<BF16, SR, EVEN, BIG>;
+    auto kern = k_quant_cols<BF16, SR, EVEN, BIG, OAS>;
     const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
                                      T::kThreads, 0, n_tiles);
     kern<<<grid, T::kThreads, 0, s>>>(x, rows, cols, key, codes, scales);
@@ -844,31 +853,34 @@ static bool big_tensor(int64_t rows, int64_t cols) {
   return rows * cols >= (int64_t(1) << 33);
 }
 
-template <bool BF16>
+template <bool BF16, bool OAS>
 static cudaError_t quant_cols_dispatch(const void* x, int64_t rows,
                                        int64_t cols, bool sr, RngKey key,
                                        uint8_t* codes, uint8_t* scales,
                                        cudaStream_t s) {
   const bool vec = cols % (BF16 ? 8 : 4) == 0;
   if (!sr)
-    return vec ? quant_cols_impl<BF16, false, true, true, false>(x, rows, cols, key, codes, scales, s)
-               : quant_cols_impl<BF16, false, false, true, false>(x, rows, cols, key, codes, scales, s);
+    return vec ? quant_cols_impl<BF16, false, true, true, false, OAS>(x, rows, cols, key, codes, scales, s)
+               : quant_cols_impl<BF16, false, false, true, false, OAS>(x, rows, cols, key, codes, scales, s);
   if (cols % 2 != 0)  // odd rows split column pairs over two hashes
-    return quant_cols_impl<BF16, true, false, false, true>(x, rows, cols, key, codes, scales, s);
+    return quant_cols_impl<BF16, true, false, false, true, OAS>(x, rows, cols, key, codes, scales, s);
   if (big_tensor(rows, cols))
-    return vec ? quant_cols_impl<BF16, true, true, true, true>(x, rows, cols, key, codes, scales, s)
-               : quant_cols_impl<BF16, true, false, true, true>(x, rows, cols, key, codes, scales, s);
-  return vec ? quant_cols_impl<BF16, true, true, true, false>(x, rows, cols, key, codes, scales, s)
-             : quant_cols_impl<BF16, true, false, true, false>(x, rows, cols, key, codes, scales, s);
+    return vec ? quant_cols_impl<BF16, true, true, true, true, OAS>(x, rows, cols, key, codes, scales, s)
+               : quant_cols_impl<BF16, true, false, true, true, OAS>(x, rows, cols, key, codes, scales, s);
+  return vec ? quant_cols_impl<BF16, true, true, true, false, OAS>(x, rows, cols, key, codes, scales, s)
+             : quant_cols_impl<BF16, true, false, true, false, OAS>(x, rows, cols, key, codes, scales, s);
 }
 
 cudaError_t launch_quant_cols(const void* x, bool bf16, int64_t rows,
                               int64_t cols, bool sr, uint64_t seed,
                               uint8_t* codes, uint8_t* scales,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool oas) {
   const RngKey key = make_key(seed, 0);
-  return bf16 ? quant_cols_dispatch<true>(x, rows, cols, sr, key, codes, scales, s)
-              : quant_cols_dispatch<false>(x, rows, cols, sr, key, codes, scales, s);
+  if (oas)
+    return bf16 ? quant_cols_dispatch<true, true>(x, rows, cols, sr, key, codes, scales, s)
+                : quant_cols_dispatch<false, true>(x, rows, cols, sr, key, codes, scales, s);
+  return bf16 ? quant_cols_dispatch<true, false>(x, rows, cols, sr, key, codes, scales, s)
+              : quant_cols_dispatch<false, false>(x, rows, cols, sr, key, codes, scales, s);
 }
 
 cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,

@@ -57,6 +57,9 @@ def _declare(L):
         "orc_rand16_range": ([u64, u32, u64, i64,
                               ctypes.POINTER(ctypes.c_uint32)], None),
         "orc_scale_exponent": ([dbl], i32),
+        "orc_scale_exponent_oas": ([dbl], i32),
+        "orc_quantize_oas": ([vp, i32, i64, i64, i64, i32, i32, u64, _u8p, _u8p],
+                             i32),
         "orc_rne_index": ([dbl], i32),
         "orc_sr_index": ([dbl, u32], i32),
         "orc_sr_count_up": ([dbl], i32),
@@ -116,6 +119,9 @@ class Oracle:
     def scale_exponent(self, absmax):
         return self.L.orc_scale_exponent(float(absmax))
 
+    def scale_exponent_oas(self, absmax):
+        return self.L.orc_scale_exponent_oas(absmax)
+
     def rne_index(self, a):
         return self.L.orc_rne_index(float(a))
 
@@ -135,16 +141,17 @@ class Oracle:
         return self.L.orc_rht_sign(sign_seed, c)
 
     # --- tensor entry points ---------------------------------------------
-    def quantize(self, x, axis=ROWS, rounding=RNE, seed=0, row0=0):
+    def quantize(self, x, axis=ROWS, rounding=RNE, seed=0, row0=0, oas=False):
         """Block quantize x [R, C]; returns (codes, scales), axis layout.
         x may be rows row0.. of a larger tensor (random numbers are keyed by
-        the index in that tensor)."""
+        the index in that tensor). oas: the overflow-aware scale rule."""
         x, dt = _as_input(x)
         R, C = x.shape
         codes = np.zeros(R * C // 2, np.uint8)
         scales = np.zeros(R * C // 32, np.uint8)
-        rc = self.L.orc_quantize(x.ctypes.data, dt, R, C, row0, axis,
-                                 rounding, seed, _u8(codes), _u8(scales))
+        fn = self.L.orc_quantize_oas if oas else self.L.orc_quantize
+        rc = fn(x.ctypes.data, dt, R, C, row0, axis, rounding, seed, _u8(codes),
+                _u8(scales))
         if rc != 0:
             raise ValueError("bad shape for the oracle quantizer: %s" % (x.shape,))
         if axis == ROWS:

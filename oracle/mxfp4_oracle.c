@@ -34,7 +34,12 @@
  *  - stochastic rounding goes up iff (r + 0.5) * 2^-16 < frac, r the 16-bit
  *    random number of the element, from the counter hash below;
  *  - the Hadamard transform is 1-D along each 1x32 row group;
- *  - the "bin centre" of a weight is its dequantized value.
+ *  - the "bin centre" of a weight is its dequantized value;
+ *  - the overflow-aware scale ([OAS]) is the smallest e with
+ *    absmax * 2^-e <= 6. The page names the idea without a formula: the
+ *    rule is pinned by its own properties (exhaustive minimality and
+ *    non-saturation, unbiased stochastic rounding), but its agreement with
+ *    the paper's OAS is parity unpinned.
  *
  * Parity pins: every function here is checked by tests against something
  * other than itself (a library E2M1 cast, exact comparisons with powers of
@@ -130,14 +135,30 @@ int orc_scale_exponent(double absmax) {
   return e;
 }
 
-/* E8M0 byte of a group: 0xFF if any element is not finite, else e + 127. */
-static int group_scale_byte(const double* g) {
+/* Overflow-aware scale ([OAS] abstract: overflow-aware scaling under
+ * power-of-two block scales; the page gives no formula, so this is a
+ * reading, parity unpinned by the pages): the smallest e in [-127, 127] with
+ * absmax * 2^-e <= 6, so no element of the group saturates. Found by exact
+ * comparisons, starting below the OCP exponent. */
+int orc_scale_exponent_oas(double absmax) {
+  int e = orc_scale_exponent(absmax) - 1;
+  if (e < -127) e = -127;
+  while (e < 127 && ldexp(absmax, -e) > 6.0) ++e;
+  return e;
+}
+
+enum { SCALE_OCP = 0, SCALE_OAS = 1 };
+
+/* E8M0 byte of a group: 0xFF if any element is not finite, else e + 127
+ * with e from the OCP rule or the overflow-aware one. */
+static int group_scale_byte(const double* g, int scale_rule) {
   double absmax = 0.0;
   for (int j = 0; j < 32; ++j) {
     if (!isfinite(g[j])) return 0xFF;
     if (fabs(g[j]) > absmax) absmax = fabs(g[j]);
   }
-  return orc_scale_exponent(absmax) + 127;
+  return (scale_rule == SCALE_OAS ? orc_scale_exponent_oas(absmax)
+                                  : orc_scale_exponent(absmax)) + 127;
 }
 
 /* ------------------------------------------------------------------ */
@@ -188,8 +209,8 @@ double orc_decode(int code, int sb) {
 /* ------------------------------------------------------------------ */
 
 static int quantize_group(const double* g, int rounding, uint64_t seed,
-                          const uint64_t* idx, int* codes_out) {
-  int sb = group_scale_byte(g);
+                          const uint64_t* idx, int scale_rule, int* codes_out) {
+  int sb = group_scale_byte(g, scale_rule);
   for (int j = 0; j < 32; ++j) {
     if (sb == 0xFF) {
       codes_out[j] = 0;
@@ -213,7 +234,8 @@ static void put_nibble(uint8_t* codes, int64_t byte, int high, int code) {
  * are keyed by the element's index in that larger tensor. */
 static void quantize_values(const double* xv, int64_t rows, int64_t cols,
                             int64_t row0, int axis, int rounding,
-                            uint64_t seed, uint8_t* codes, uint8_t* scales) {
+                            uint64_t seed, int scale_rule, uint8_t* codes,
+                            uint8_t* scales) {
   double g[32];
   uint64_t idx[32];
   int cq[32];
@@ -226,7 +248,7 @@ static void quantize_values(const double* xv, int64_t rows, int64_t cols,
           g[j] = xv[r * cols + c];
         }
         scales[r * (cols / 32) + k] =
-            (uint8_t)quantize_group(g, rounding, seed, idx, cq);
+            (uint8_t)quantize_group(g, rounding, seed, idx, scale_rule, cq);
         for (int j = 0; j < 32; ++j) {
           int64_t c = 32 * k + j;
           put_nibble(codes, r * (cols / 2) + c / 2, (int)(c & 1), cq[j]);
@@ -241,7 +263,7 @@ static void quantize_values(const double* xv, int64_t rows, int64_t cols,
           g[j] = xv[r * cols + c];
         }
         scales[c * (rows / 32) + k] =
-            (uint8_t)quantize_group(g, rounding, seed, idx, cq);
+            (uint8_t)quantize_group(g, rounding, seed, idx, scale_rule, cq);
         for (int j = 0; j < 32; ++j) {
           int64_t r = 32 * k + j;
           put_nibble(codes, c * (rows / 2) + r / 2, (int)(r & 1), cq[j]);
@@ -268,7 +290,23 @@ int orc_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
   if (rows <= 0 || cols <= 0) return -1;
   if ((axis == AX_ROWS ? cols : rows) % 32 != 0) return -1;
   double* xv = load_all(x, dtype, rows * cols);
-  quantize_values(xv, rows, cols, row0, axis, rounding, seed, codes, scales);
+  quantize_values(xv, rows, cols, row0, axis, rounding, seed, SCALE_OCP, codes,
+                  scales);
+  free(xv);
+  return 0;
+}
+
+/* orc_quantize with the overflow-aware scale (see orc_scale_exponent_oas):
+ * every scaled value is at most 6, so nothing saturates and stochastic
+ * rounding is unbiased for every input. */
+int orc_quantize_oas(const void* x, int dtype, int64_t rows, int64_t cols,
+                     int64_t row0, int axis, int rounding, uint64_t seed,
+                     uint8_t* codes, uint8_t* scales) {
+  if (rows <= 0 || cols <= 0) return -1;
+  if ((axis == AX_ROWS ? cols : rows) % 32 != 0) return -1;
+  double* xv = load_all(x, dtype, rows * cols);
+  quantize_values(xv, rows, cols, row0, axis, rounding, seed, SCALE_OAS, codes,
+                  scales);
   free(xv);
   return 0;
 }
@@ -323,11 +361,11 @@ int orc_double_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
   if (rows <= 0 || cols <= 0 || rows % 32 || cols % 32) return -1;
   int64_t n = rows * cols;
   double* xv = load_all(x, dtype, n);
-  quantize_values(xv, rows, cols, row0, AX_ROWS, RND_RNE, 0, row_codes,
+  quantize_values(xv, rows, cols, row0, AX_ROWS, RND_RNE, 0, SCALE_OCP, row_codes,
                   row_scales);
   double* d = (double*)malloc((size_t)n * sizeof(double));
   dequantize_values(row_codes, row_scales, rows, cols, AX_ROWS, d);
-  quantize_values(d, rows, cols, row0, AX_COLS, RND_SR, seed, col_codes,
+  quantize_values(d, rows, cols, row0, AX_COLS, RND_SR, seed, SCALE_OCP, col_codes,
                   col_scales);
   free(d);
   free(xv);
@@ -396,7 +434,7 @@ static void dq_rows(const float* w, int64_t rows, int64_t cols, double* out) {
     for (int64_t k = 0; k < cols / 32; ++k) {
       double g[32];
       for (int j = 0; j < 32; ++j) g[j] = (double)w[r * cols + 32 * k + j];
-      int sb = group_scale_byte(g);
+      int sb = group_scale_byte(g, SCALE_OCP);
       for (int j = 0; j < 32; ++j) {
         double v;
         if (sb == 0xFF)

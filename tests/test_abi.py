@@ -68,6 +68,14 @@ def test_quantize_rejects_bad_arguments(args, want):
     assert m.lib().mxfp4_quantize(*args) == want
 
 
+def test_quantize_oas_rejects_bad_arguments():
+    L = m.lib()
+    assert L.mxfp4_quantize_oas(P, 2, 64, 64, 0, 0, 0, P, P, NUL) == ENUM
+    assert L.mxfp4_quantize_oas(NUL, 1, 64, 64, 0, 0, 0, P, P, NUL) == NULL
+    assert L.mxfp4_quantize_oas(P, 1, 64, 48, 0, 0, 0, P, P, NUL) == SHAPE
+    assert L.mxfp4_quantize_oas(PODD, 1, 64, 64, 0, 0, 0, P, P, NUL) == ALIGN
+
+
 def test_other_entry_points_reject_bad_arguments():
     L = m.lib()
     assert L.mxfp4_dequantize(P, P, 64, 64, 0, P, 3, NUL) == ENUM

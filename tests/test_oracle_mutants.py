@@ -4,7 +4,7 @@ swapped nibbles, a reversed stochastic comparison, a transposed index, a wrong
 Hadamard entry or normalisation, a wrong random stream, the tracker without
 its absolute value, a reversed flag test, snapping to the old bin, a missing
 reset, column groups built from X instead of Q_D(X), a wrong blocked scale
-order. Mistakes are planted in
+order, an overflow-aware bound taken inclusively. Mistakes are planted in
 the oracle only, on the CPU; the real oracle source is never modified.
 """
 import os
@@ -19,6 +19,10 @@ SRC = os.path.join(os.path.dirname(O.__file__), "mxfp4_oracle.c")
 
 # (name, original text, mutated text, pins that must fail)
 MUTANTS = [
+    ("overflow-aware bound inclusive", "ldexp(absmax, -e) > 6.0",
+     "ldexp(absmax, -e) >= 6.0",
+     ["test_oas_scale_is_the_smallest_non_saturating_exponent",
+      "test_oas_moves_the_ocp_exponent_only_above_six"]),
     ("blocked lines and slots swapped", "16 * (tr % 32) + 4 * (tr / 32)",
      "4 * (tr % 32) + 16 * (tr / 32)",
      ["test_blocked_scales_line_by_line", "test_blocked_scales_is_a_padded_permutation"]),

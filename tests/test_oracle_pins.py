@@ -651,3 +651,60 @@ def test_gemm_is_the_sum_of_dequantized_products():
         for j in range(2):
             want = sum(val(ca, sa, i, kk) * val(cb, sb, j, kk) for kk in range(64))
             assert c[i, j] == want
+
+
+# ---------------------------------------------------------------------------
+# Overflow-aware scale (a reading: the MXFP4 strategies page names the idea,
+# not a formula; these pins fix the rule "smallest e with absmax 2^-e <= 6")
+# ---------------------------------------------------------------------------
+
+def _positive_bf16_values():
+    bits = np.arange(1, 0x7F80, dtype=np.uint32) << 16
+    return bits.view(np.float32).astype(np.float64)
+
+
+def test_oas_scale_is_the_smallest_non_saturating_exponent():
+    g = np.random.Generator(np.random.PCG64(60))
+    extra = [6.0 * 2.0 ** k for k in range(-120, 120)]
+    extra += [np.nextafter(v, np.inf) for v in extra]
+    extra += list(g.uniform(1e-30, 1e30, size=2000))
+    for a in list(_positive_bf16_values()) + extra:
+        e = O.scale_exponent_oas(a)
+        assert a * 2.0 ** -e <= 6.0
+        assert e == -127 or a * 2.0 ** -(e - 1) > 6.0
+
+
+def test_oas_moves_the_ocp_exponent_only_above_six():
+    for a in _positive_bf16_values():
+        e_ocp, e_oas = O.scale_exponent(a), O.scale_exponent_oas(a)
+        assert e_oas - e_ocp == (1 if a * 2.0 ** -e_ocp > 6.0 else 0)
+
+
+def test_oas_hand_worked_group():
+    # absmax 7: OCP e = 0 saturates 7 and 6 to 6.0 (index 7); OAS e = 1
+    # halves them: 3.5 ties between 3 (index 5) and 4 (index 6) and goes to
+    # the even index 6; 6 -> 3.0 (5); 2 -> 1.0 (2); 1 -> 0.5 (1);
+    # 0.5 -> 0.25, a tie between 0 and 0.5 -> 0; -3 -> -1.5 (sign | 3)
+    x = np.zeros((1, 32), np.float32)
+    x[0, :7] = [7.0, 6.0, 2.0, 1.0, 0.5, 0.25, -3.0]
+    c, s = O.quantize(x, O.ROWS, O.RNE, oas=True)
+    codes = unpack_nibbles(c)[0, :7].tolist()
+    assert s[0, 0] == 128 and codes == [6, 5, 2, 1, 0, 0, 8 | 3]
+    c, s = O.quantize(x, O.ROWS, O.RNE)
+    assert s[0, 0] == 127 and unpack_nibbles(c)[0, :7].tolist() == [7, 7, 4, 2, 1, 0, 8 | 5]
+
+
+def test_oas_stochastic_rounding_unbiased_where_ocp_saturates():
+    """A group whose OCP-scaled maximum lies in (6, 8): with the OCP scale
+    stochastic rounding clips it to 6 (biased), with the overflow-aware one
+    the mean over seeds matches the value."""
+    x = np.zeros((1, 32), np.float32)
+    x[0, 0], x[0, 1] = 7.3, 2.9
+    S = 4000
+    means = np.zeros(2)
+    for seed in range(S):
+        c, s = O.quantize(x, O.ROWS, O.SR, seed, oas=True)
+        means += O.dequantize(c, s, 1, 32, O.ROWS, "f32")[0, :2] / S
+    # one step at e = 1 is 2.0 around 7.3 and 1.0 around 2.9
+    assert abs(means[0] - 7.3) < 4 * 1.0 / np.sqrt(S) + 2.0 * 2.0 ** -17
+    assert abs(means[1] - 2.9) < 4 * 0.5 / np.sqrt(S) + 1.0 * 2.0 ** -17
