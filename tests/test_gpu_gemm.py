@@ -56,7 +56,12 @@ def test_gemm_single_scale_moves_single_row_and_group():
 
 
 @pytest.mark.parametrize("mnk", [(128, 128, 256), (200, 136, 96), (64, 40, 32),
-                                 (384, 256, 1024), (130, 520, 800)])
+                                 (384, 256, 1024), (130, 520, 800),
+                                 # the persistent TMA kernel (k % 256 == 0) on
+                                 # partial tiles: clipped TMA stores, a missing
+                                 # second B scale tile, direct stores (n % 4)
+                                 (200, 136, 512), (130, 130, 768), (64, 8, 256),
+                                 (1000, 600, 2048), (300, 1030, 256)])
 def test_gemm_quantized_operands(mnk):
     M, N, K = mnk
     x = W.normal_bf16(M, K, M + 1, 0.01, 20.0)
