@@ -232,6 +232,19 @@ def cpu_sample_step(x_band, w_band, osc_state, row0):
     return nb, n * 5 + w.size * 2
 
 
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline_sample(x_np, w_np, max_seconds=20.0):
     band = np.ascontiguousarray(x_np[:32])
     wb = np.ascontiguousarray(w_np[:16])
@@ -247,7 +260,7 @@ def cpu_baseline_sample(x_np, w_np, max_seconds=20.0):
             break
     dt = time.perf_counter() - t0
     return {"value": total_b / dt / 1e9, "unit": "GB/s", "cores": 1,
-            "kind": "oracle",
+            "kind": "oracle", "cpu": cpu_model(), "host_cores": os.cpu_count(),
             "sample": "%d reps of one 32x28672 band of the sweep per op (rows RNE, "
                       "cols SR, double quant, dequant, RHT+SR) and a 16x4096 band "
                       "of the tracker (update + step); single thread, %.1f s"
@@ -288,6 +301,7 @@ def cpu_baseline_all_cores(x_np, w_np, reps=8):
     nb = sum(r[0] for r in res)
     ne = sum(r[1] for r in res)
     return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": cores,
+            "cpu": cpu_model(),
             "kind": "oracle",
             "sample": "%d processes x %d reps of the one-band sample step "
                       "(each its own 32x28672 band), %.1f s wall" % (cores, reps, dt),
@@ -321,7 +335,7 @@ def run_reference(args):
             "data": "synthetic",
             "config": config_block(args, 1),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1,
-                             "kind": "oracle",
+                             "kind": "oracle", "cpu": cpu_model(),
                              "sample": "each step: one 32x28672 band of the sweep "
                                        "per op and a 16x4096 tracker band"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
