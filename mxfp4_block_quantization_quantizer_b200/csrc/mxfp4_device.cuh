@@ -160,27 +160,42 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
 // noise = 2^22 - 33 - 64r, the mantissa field plus noise carries into bit 22
 // exactly when the value goes up (the carry may run on into the exponent:
 // 1.5 -> 2, 3 -> 4). The bias 0.5 = 0x3F000000 is folded into the noise.
-__device__ __forceinline__ uint32_t sr_noise(uint32_t r) {
-  return r * 0xFFFFFFC0u + 0xC13FFFDFu;  // (2^22 - 33 - 64r) - 0x3F000000
+//
+// The sum lies in [31, 2^25), magnitude index in bits 22..24; it is formed
+// times 64 (one multiply-add), which puts the index in bits 28..30 with bit
+// 31 clear for the sign: the code is the top nibble, and codes are packed by
+// funnel shifts of those nibbles. sr_noise64(r) = 64 (2^22 - 33 - 64r) -
+// 64 * 0x3F000000 mod 2^32.
+__device__ __forceinline__ uint32_t sr_noise64(uint32_t r) {
+  return r * 0xFFFFF000u + 0x4FFFF7C0u;
 }
 // The noises of the pair whose hash is mix32 = g ^ (g >> 16), g = mix32_pre
-// of its counter: the even element takes the low half, the odd one the high.
-__device__ __forceinline__ uint32_t sr_noise_lo(uint32_t g) {
-  return sr_noise((g ^ (g >> 16)) & 0xFFFFu);
-}
-__device__ __forceinline__ uint32_t sr_noise_hi(uint32_t g) {
-  return sr_noise(__umulhi(g, 1u << 16));  // g >> 16 on the multiply pipe
+// of its counter: the even element takes the low half, the odd one the high
+// half (g >> 16: the xor only touches the low half).
+__device__ __forceinline__ void sr_noise64_pair(uint32_t g, uint32_t& n_even,
+                                                uint32_t& n_odd) {
+  const uint32_t hi = g >> 16;
+  n_even = sr_noise64((g ^ hi) & 0xFFFFu);
+  n_odd = sr_noise64(hi);
 }
 
-// SAT = false leaves out the saturation, for callers whose |v| never exceeds
-// 6.
+// The stochastic code of v in bits 28..31 (sign in bit 31; the bits below
+// are not part of it). SAT = false leaves out the saturation, for callers
+// whose |v| never exceeds 6.
 template <bool SAT = true>
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t noise) {
+__device__ __forceinline__ uint32_t e2m1_sr_top(float v, uint32_t noise64) {
   const float a = fabsf(v);
   float y = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
   if (SAT) y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
-  const uint32_t m = (__float_as_uint(y) + noise) >> 22;
-  return m + (__float_as_uint(v) >> 31) * 8u;  // sign
+  return (__float_as_uint(y) * 64u + noise64) |
+         (__float_as_uint(v) & 0x80000000u);
+}
+
+// Shift a packed code word up by one nibble and append the code held in the
+// top nibble of t: codes pushed in the order 7, 6, .., 0 land in nibbles
+// 7 .. 0.
+__device__ __forceinline__ uint32_t push_code(uint32_t acc, uint32_t t) {
+  return __funnelshift_l(t, acc, 4);
 }
 
 // Stochastic codes of 8 values; pair k of the 8 values takes its two random
@@ -190,9 +205,11 @@ __device__ __forceinline__ uint32_t e2m1x8_sr(const float* v,
                                               const uint32_t* g) {
   uint32_t out = 0;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    out += e2m1_sr(v[2 * k], sr_noise_lo(g[k])) * (1u << (8 * k));
-    out += e2m1_sr(v[2 * k + 1], sr_noise_hi(g[k])) * (1u << (8 * k + 4));
+  for (int k = 3; k >= 0; --k) {
+    uint32_t ne, no;
+    sr_noise64_pair(g[k], ne, no);
+    out = push_code(out, e2m1_sr_top(v[2 * k + 1], no));
+    out = push_code(out, e2m1_sr_top(v[2 * k], ne));
   }
   return out;
 }

@@ -123,11 +123,11 @@ struct ColTile {
   static constexpr int kChunksPerRow = kCols / kChunkElems;
 };
 
-// Random-number noise of the two adjacent elements (r0+j, c0), (r0+j, c0+1)
-// of a column pass. Element (r, c) has index i = r*cols + c; c0 is even.
-// EVEN (cols even): i is even, so both elements are the halves of pair
-// i/2, and the pair index of row r0+j is p0 + j*cols/2. Otherwise odd rows
-// split the two elements over adjacent pairs. BIG: the tensor has 2^33
+// Random-number noise (sr_noise64) of the two adjacent elements (r0+j, c0),
+// (r0+j, c0+1) of a column pass. Element (r, c) has index i = r*cols + c; c0
+// is even. EVEN (cols even): i is even, so both elements are the halves of
+// pair i/2, and the pair index of row r0+j is p0 + j*cols/2. Otherwise odd
+// rows split the two elements over adjacent pairs. BIG: the tensor has 2^33
 // elements or more, so the high word of a pair index can be nonzero.
 template <bool EVEN, bool BIG>
 __device__ __forceinline__ void column_noise(RngKey key, uint64_t i0,
@@ -136,20 +136,19 @@ __device__ __forceinline__ void column_noise(RngKey key, uint64_t i0,
   if (EVEN && !BIG) {
     const uint32_t h = mix32_pre(key.k0 + uint32_t(i0 >> 1) +
                                  uint32_t(j) * uint32_t(uint64_t(cols) >> 1));
-    na = sr_noise_lo(h);
-    nb = sr_noise_hi(h);
+    sr_noise64_pair(h, na, nb);
   } else {
     const uint64_t i = i0 + uint64_t(j) * uint64_t(cols);
     const uint64_t p = i >> 1;
     const uint32_t h = mix32_pre(inner_key(key, uint32_t(p >> 32)) + uint32_t(p));
     if ((i & 1) == 0) {
-      na = sr_noise_lo(h);
-      nb = sr_noise_hi(h);
+      sr_noise64_pair(h, na, nb);
     } else {
       const uint64_t p2 = p + 1;
       const uint32_t h2 = mix32_pre(inner_key(key, uint32_t(p2 >> 32)) + uint32_t(p2));
-      na = sr_noise_hi(h);
-      nb = sr_noise_lo(h2);
+      uint32_t unused;
+      sr_noise64_pair(h, unused, na);
+      sr_noise64_pair(h2, nb, unused);
     }
   }
 }
@@ -179,12 +178,12 @@ __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
   if (SR) {
     const uint64_t i0 = uint64_t(r0) * uint64_t(cols) + uint64_t(c0);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 31; j >= 0; --j) {  // push_code fills nibbles 7 .. 0
       uint32_t na, nb;
       column_noise<EVEN, BIG>(key, i0, cols, j, na, nb);
       const float2 v = get(j);
-      o.wa[j >> 3] += e2m1_sr<SAT>(v.x * mula, na) * (1u << (4 * (j & 7)));
-      o.wb[j >> 3] += e2m1_sr<SAT>(v.y * mulb, nb) * (1u << (4 * (j & 7)));
+      o.wa[j >> 3] = push_code(o.wa[j >> 3], e2m1_sr_top<SAT>(v.x * mula, na));
+      o.wb[j >> 3] = push_code(o.wb[j >> 3], e2m1_sr_top<SAT>(v.y * mulb, nb));
     }
   } else {
 #pragma unroll
