@@ -271,7 +271,6 @@ constexpr int kPEpiWarps = 8;
 constexpr int kPThreads = 32 * (2 + kPEpiWarps);
 constexpr uint32_t kPTmemCols = 512;
 constexpr uint32_t kPSfCol = 256;  // per stage: 8 SFA columns, then 16 SFB
-constexpr uint32_t kPSfStride = 24;
 
 struct __align__(1024) PipeSmem {
   uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled

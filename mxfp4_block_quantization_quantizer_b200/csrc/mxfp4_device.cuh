@@ -285,6 +285,16 @@ __device__ __forceinline__ float absmax_nan(float a, float m) {
   return d;
 }
 
+// max(|a|, |b|, m) for m >= 0 or NaN, propagating NaN.
+__device__ __forceinline__ float absmax3_nan(float a, float b, float m) {
+  float d;
+  asm("{\n\t.reg .f32 t, u;\n\tabs.f32 t, %1;\n\tabs.f32 u, %2;\n\t"
+      "max.NaN.f32 %0, t, u, %3;\n\t}"
+      : "=f"(d)
+      : "f"(a), "f"(b), "f"(m));
+  return d;
+}
+
 // Per-half unsigned max of two packed 16-bit pairs.
 __device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -292,13 +302,22 @@ __device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
-// fp32 bit pattern of the largest |value| among 8 packed bf16 values: the
-// absolute bit patterns of finite and non-finite values order like their
-// magnitudes, so a per-half integer max finds the group maximum (and any
-// Inf/NaN, whose pattern is at least 0x7F80).
+// Per-half max(|a|, |b|) of two packed bf16 pairs, propagating NaN (a NaN
+// half gives the canonical NaN); the sign bits of the result are not
+// defined, callers mask them.
+__device__ __forceinline__ uint32_t bf16x2_absmax_nan(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// fp32 bit pattern of the largest |value| among 8 packed bf16 values (any
+// Inf/NaN gives a pattern of at least 0x7F800000): the absolute bit patterns
+// order like the magnitudes, so the two halves combine with an integer max.
 __device__ __forceinline__ uint32_t bf16x8_absmax(uint4 w) {
-  const uint32_t m = umax16x2(umax16x2(w.x & 0x7FFF7FFFu, w.y & 0x7FFF7FFFu),
-                              umax16x2(w.z & 0x7FFF7FFFu, w.w & 0x7FFF7FFFu));
+  const uint32_t m = bf16x2_absmax_nan(bf16x2_absmax_nan(w.x, w.y),
+                                       bf16x2_absmax_nan(w.z, w.w)) &
+                     0x7FFF7FFFu;
   return max(m << 16, m & 0xFFFF0000u);
 }
 

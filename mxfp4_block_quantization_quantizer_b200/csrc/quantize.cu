@@ -292,7 +292,8 @@ __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
     const uint32_t* s = reinterpret_cast<const uint32_t*>(tile) + 32 * rg * (kcols / 2) + cp;
     uint32_t m = 0;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) m = umax16x2(m, s[j * (kcols / 2)] & 0x7FFF7FFFu);
+    for (int j = 0; j < 32; ++j) m = bf16x2_absmax_nan(m, s[j * (kcols / 2)]);
+    m &= 0x7FFF7FFFu;
     ma = m << 16;
     mb = m & 0xFFFF0000u;
     return column_pair_codes<SR, EVEN, BIG, true, OAS>(
@@ -634,14 +635,14 @@ __global__ void __launch_bounds__(kDqThreads)
 }
 
 // Row pass of one 1x32 group quarter (8 values of tile row tr, chunk ch):
-// returns the 4 code bytes; writes the row codes and scale to global memory
-// (when in range) and stages them in shared memory for the column pass.
+// writes the row codes and scale to global memory (when in range) and stages
+// the codes and the scale value 2^e in shared memory for the column pass.
 __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool ok,
                                              int64_t gr, int64_t gc, int64_t cols,
                                              int tr, int ch,
                                              uint8_t* __restrict__ row_codes,
                                              uint8_t* __restrict__ row_scales,
-                                             uint32_t* s_codes, uint8_t* s_scales) {
+                                             uint32_t* s_codes, float* s_scales) {
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   const uint32_t sb = scale_byte(amax);
@@ -655,12 +656,13 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
     if ((ch & 3) == 0) row_scales[gr * (cols / 32) + gc / 32] = uint8_t(sb);
   }
   s_codes[tr * (kDqCols / 8) + ch] = word;
-  if ((ch & 3) == 0) s_scales[tr * (kDqCols / 32) + ch / 4] = uint8_t(sb);
+  if ((ch & 3) == 0) s_scales[tr * (kDqCols / 32) + ch / 4] = scale_value(sb);
 }
 
 // Column pass of the double quantizer over the staged Q_D(X) codes: decode
 // columns 2cp, 2cp+1 of rows 32rg.. (one shared byte per row holds both
-// codes; a row group of scale 0xFF decodes to NaN as 0 x inf, and the
+// codes) and multiply by the row groups' staged scale values (a row group of
+// scale 0xFF has the value +inf and codes 0, so it decodes to NaN, and the
 // NaN-propagating maximum carries it into the column scale), then
 // stochastic rounding along the 32x1 groups. The caller checks that the row
 // group lies inside the tensor.
@@ -670,7 +672,7 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
 // value is at most 6 (the only such values in [4, 8) are 4 and 6).
 template <bool BIG>
 __device__ __forceinline__ ColPair dq_column_pass(
-    const uint32_t* s_codes, const uint8_t* s_scales, int rg, int cp,
+    const uint32_t* s_codes, const float* s_scales, int rg, int cp,
     int64_t tile_r, int64_t tile_c, int64_t cols, RngKey key) {
   const int64_t r0 = tile_r + 32 * rg;
   const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
@@ -684,7 +686,7 @@ __device__ __forceinline__ ColPair dq_column_pass(
     for (int i = 0; i < 4; ++i) {
       const int r = 32 * rg + 4 * q + i;
       w4 |= uint32_t(sc[r * (kDqCols / 2) + cp]) << (8 * i);
-      sv[i] = scale_value(s_scales[r * (kDqCols / 32) + cp / 16]);
+      sv[i] = s_scales[r * (kDqCols / 32) + cp / 16];
     }
     float f[8];
     e2m1x8_decode(w4, f);
@@ -692,8 +694,11 @@ __device__ __forceinline__ ColPair dq_column_pass(
     for (int i = 0; i < 4; ++i) {
       a[4 * q + i] = f[2 * i] * sv[i];
       b[4 * q + i] = f[2 * i + 1] * sv[i];
-      ma = absmax_nan(a[4 * q + i], ma);
-      mb = absmax_nan(b[4 * q + i], mb);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      ma = absmax3_nan(a[4 * q + i], a[4 * q + i + 1], ma);
+      mb = absmax3_nan(b[4 * q + i], b[4 * q + i + 1], mb);
     }
   }
   // cols is a multiple of 32 here, so every pair index is even-aligned
@@ -716,7 +721,7 @@ __global__ void __launch_bounds__(kDqThreads, 3)
   constexpr int kChunks = kTileRows * (kDqCols / 8);
   extern __shared__ uint4 smem[];  // two raw tiles, then the staged Q_D(X)
   uint32_t* s_codes = reinterpret_cast<uint32_t*>(smem + 2 * kChunks);
-  uint8_t* s_scales = reinterpret_cast<uint8_t*>(s_codes + kTileRows * (kDqCols / 8));
+  float* s_scales = reinterpret_cast<float*>(s_codes + kTileRows * (kDqCols / 8));
   const int64_t tiles_c = (cols + kDqCols - 1) / kDqCols;
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
   const int ch = threadIdx.x & 15, rr = threadIdx.x >> 4;
@@ -918,7 +923,8 @@ cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
   if (bf16) {
     auto kern = big ? k_double_quant_pipe<true> : k_double_quant_pipe<false>;
     constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) +
-                            kTileRows * (kDqCols / 8) * 4 + kTileRows * (kDqCols / 32);
+                            kTileRows * (kDqCols / 8) * 4 +
+                            kTileRows * (kDqCols / 32) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(
         reinterpret_cast<const void*>(kern),
         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
