@@ -107,6 +107,10 @@ __device__ __forceinline__ void copy_scales_to_tmem(uint32_t taddr,
                "l"(d));
 }
 
+// As copy_scales_to_tmem, with the source descriptor given.
+__device__ __forceinline__ void copy_scales_desc(uint32_t taddr, uint64_t d) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d));
+}
 __device__ __forceinline__ bool wait_parity(unsigned long long* bar,
                                             uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -272,6 +276,22 @@ constexpr int kPThreads = 32 * (2 + kPEpiWarps);
 constexpr uint32_t kPTmemCols = 512;
 constexpr uint32_t kPSfCol = 256;  // per stage: 8 SFA columns, then 16 SFB
 
+// Tile order: groups of kGroupM row tiles of C, each group swept across all
+// column tiles before the next (the last group may be narrower). The CTAs
+// running at one time then cover about kGroupM x (CTAs / kGroupM) tiles, so
+// their A and B panels stay in L2 while they stream through K.
+constexpr int64_t kGroupM = 16;
+__device__ __forceinline__ void tile_coords(int64_t tile, int64_t m_tiles,
+                                            int64_t nt_n, int64_t& m0,
+                                            int64_t& n0) {
+  const int64_t per_group = kGroupM * nt_n;
+  const int64_t g = tile / per_group, r = tile % per_group;
+  const int64_t rest = m_tiles - g * kGroupM;
+  const int64_t gm = rest < kGroupM ? rest : kGroupM;
+  m0 = (g * kGroupM + r % gm) * kGM;
+  n0 = (r / gm) * kPN;
+}
+
 struct __align__(1024) PipeSmem {
   uint8_t a[kPS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
   uint8_t b[kPS][kPN][128];
@@ -366,7 +386,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int64_t n_kb = k / 256;
   const int64_t n_row_tiles = (n + 127) / 128;
   const int64_t m_tiles = (m + kGM - 1) / kGM;
-  const int64_t n_tiles = m_tiles * ((n + kPN - 1) / kPN);
+  const int64_t n_col_tiles = (n + kPN - 1) / kPN;
+  const int64_t n_tiles = m_tiles * n_col_tiles;
 
   if (tid == 0) {
     for (int s = 0; s < kPS; ++s) {
@@ -389,42 +410,83 @@ __global__ void __launch_bounds__(kPThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;");
   const uint32_t tmem = sm.tmem_base;
 
-  // Tiles in M-fastest order, CTA i taking tiles i, i + grid, ...: the CTAs
-  // running at one time share B's rows and stream all of A once.
+  // CTA i takes tiles i, i + grid, ... in the grouped order of tile_coords.
+  // The two issuing threads keep their per-stage work small: the stage index
+  // and phase advance by increments, operand addresses and descriptors are
+  // computed once and offset by constants, and the MMA loop is unrolled over
+  // the stages when every tile starts at stage 0 (K/256 a multiple of kPS).
   if (warp == 0) {
     if (lane == 0) {
-      int64_t it = 0;
+      uint32_t s = 0, ph = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        const int64_t m0 = (tile % m_tiles) * kGM, n0 = (tile / m_tiles) * kPN;
+        int64_t m0, n0;
+        tile_coords(tile, m_tiles, n_col_tiles, m0, n0);
         const int64_t rb = n0 / 128;
         const bool half1 = rb + 1 < n_row_tiles;
-        for (int64_t kb = 0; kb < n_kb; ++kb, ++it) {
-          const int s = int(it % kPS);
-          const uint32_t ph = uint32_t((it / kPS) & 1);
-          if (!wait_parity(&sm.empty[s], ph ^ 1u) || failed_flag(&sm.failed)) {
+        const uint32_t bytes = kGM * 128 + kPN * 128 + 1024 + (half1 ? 2048 : 1024);
+        // blocked scales: 512-byte tiles of 128 rows x 4 groups, K tiles first
+        const uint8_t* pa = sfa + (m0 / 128) * k_tiles * 512;
+        const uint8_t* pb0 = sfb + rb * k_tiles * 512;
+        const uint8_t* pb1 = pb0 + k_tiles * 512;
+        bool stop = false;
+        for (int64_t kb = 0; kb < n_kb; ++kb) {
+          if (!wait_parity(&sm.empty[s], ph ^ 1u)) {
             atomicExch(&sm.failed, 1);
-            tile = n_tiles;
+            stop = true;
             break;
           }
-          const uint32_t bytes = kGM * 128 + kPN * 128 + 1024 + (half1 ? 2048 : 1024);
           expect_tx(&sm.full[s], bytes);
-          tma_load_2d(&sm.a[s][0][0], &tm_a, int(kb * 128), int(m0), &sm.full[s]);
-          tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb * 128), int(n0), &sm.full[s]);
-          bulk_load(&sm.sfa[s][0][0], sfa + ((m0 / 128) * k_tiles + 2 * kb) * 512, 1024,
-                    &sm.full[s]);
-          bulk_load(&sm.sfb[s][0][0][0], sfb + (rb * k_tiles + 2 * kb) * 512, 1024,
-                    &sm.full[s]);
-          if (half1)
-            bulk_load(&sm.sfb[s][1][0][0], sfb + ((rb + 1) * k_tiles + 2 * kb) * 512, 1024,
-                      &sm.full[s]);
+          tma_load_2d(&sm.a[s][0][0], &tm_a, int(kb) * 128, int(m0), &sm.full[s]);
+          tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb) * 128, int(n0), &sm.full[s]);
+          bulk_load(&sm.sfa[s][0][0], pa + kb * 1024, 1024, &sm.full[s]);
+          bulk_load(&sm.sfb[s][0][0][0], pb0 + kb * 1024, 1024, &sm.full[s]);
+          if (half1) bulk_load(&sm.sfb[s][1][0][0], pb1 + kb * 1024, 1024, &sm.full[s]);
+          if (++s == kPS) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
+        if (stop || failed_flag(&sm.failed)) break;
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      int64_t it = 0, ti = 0;
+      // scale factors in tensor memory: row r of an operand in lane r % 32,
+      // 32-bit column r / 32 (A: 4 columns per K tile; B, 256 rows: 8, its
+      // two 128-row tiles side by side), one byte per 32-element group;
+      // tensor-core operations of one thread run in order, so the next
+      // stage's copy may reuse the columns
       const uint32_t sf = tmem + kPSfCol;
+      const uint64_t a_d0 = smem_desc_sw128(&sm.a[0][0][0]);
+      const uint64_t b_d0 = smem_desc_sw128(&sm.b[0][0][0]);
+      const uint64_t sfa_d0 = smem_desc(&sm.sfa[0][0][0], 16, 128);
+      const uint64_t sfb_d0 = smem_desc(&sm.sfb[0][0][0][0], 16, 128);
+      // descriptor start-address steps (16-byte units): one stage of A, of
+      // B, of A's and of B's scales, one 512-byte scale tile; the K = 64
+      // step inside a 128-byte swizzle row is 32 bytes
+      constexpr uint32_t kAStep = (kGM * 128) >> 4, kBStep = (kPN * 128) >> 4;
+      constexpr uint32_t kSfaStep = 1024 >> 4, kSfbStep = 2048 >> 4, kSfTile = 512 >> 4;
+      auto issue_stage = [&](uint32_t st, bool first) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          copy_scales_desc(sf + 4 * j, sfa_d0 + (st * kSfaStep + j * kSfTile));
+          copy_scales_desc(sf + 8 + 8 * j, sfb_d0 + (st * kSfbStep + j * kSfTile));
+          copy_scales_desc(sf + 8 + 8 * j + 4, sfb_d0 + (st * kSfbStep + (2 + j) * kSfTile));
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t sf_id = 2u * (t & 1);
+          const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
+          const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
+          const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
+          mma_mxf4(tmem, a_d0 + (st * kAStep + 2 * t), b_d0 + (st * kBStep + 2 * t), idesc,
+                   (first && t == 0) ? 0u : 1u, tsfa, tsfb);
+        }
+        commit_to(&sm.empty[st]);
+      };
+      uint32_t s = 0, ph = 0;
+      int64_t ti = 0;
       for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
         // the epilogue has read the previous tile's accumulator
         if (!wait_parity(&sm.acc_empty, uint32_t(ti & 1) ^ 1u) || failed_flag(&sm.failed)) {
@@ -433,38 +495,34 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         asm volatile("tcgen05.fence::after_thread_sync;");
         bool ok = true;
-        for (int64_t kb = 0; kb < n_kb; ++kb, ++it) {
-          const int s = int(it % kPS);
-          const uint32_t ph = uint32_t((it / kPS) & 1);
-          if (!wait_parity(&sm.full[s], ph) || failed_flag(&sm.failed)) {
-            atomicExch(&sm.failed, 1);
-            ok = false;
-            break;
-          }
-          asm volatile("tcgen05.fence::after_thread_sync;");
-          // scale factors in tensor memory: row r of an operand in lane r % 32,
-          // 32-bit column r / 32 (A: 4 columns per K tile; B, 256 rows: 8,
-          // its two 128-row tiles side by side), one byte per 32-element
-          // group; tensor-core operations of one thread run in order, so the
-          // next stage's copy may reuse the columns
+        if (n_kb % kPS == 0) {
+          for (int64_t kb4 = 0; kb4 < n_kb && ok; kb4 += kPS) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            copy_scales_to_tmem(sf + 4 * j, &sm.sfa[s][j][0]);
-            copy_scales_to_tmem(sf + 8 + 8 * j, &sm.sfb[s][0][j][0]);
-            copy_scales_to_tmem(sf + 8 + 8 * j + 4, &sm.sfb[s][1][j][0]);
+            for (int st = 0; st < kPS; ++st) {
+              if (!wait_parity(&sm.full[st], ph)) {
+                ok = false;
+                break;
+              }
+              asm volatile("tcgen05.fence::after_thread_sync;");
+              issue_stage(uint32_t(st), kb4 == 0 && st == 0);
+            }
+            ph ^= 1u;
           }
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const uint32_t sf_id = 2u * (t & 1);
-            const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
-            const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
-            const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
-            mma_mxf4(tmem, smem_desc_sw128(&sm.a[s][0][32 * t]),
-                     smem_desc_sw128(&sm.b[s][0][32 * t]), idesc,
-                     (kb > 0 || t > 0) ? 1u : 0u, tsfa, tsfb);
+        } else {
+          for (int64_t kb = 0; kb < n_kb; ++kb) {
+            if (!wait_parity(&sm.full[s], ph)) {
+              ok = false;
+              break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;");
+            issue_stage(s, kb == 0);
+            if (++s == kPS) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
-          commit_to(&sm.empty[s]);
         }
+        if (!ok) atomicExch(&sm.failed, 1);
         commit_to(&sm.acc_full);
         if (!ok) break;
       }
@@ -478,7 +536,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int half = (warp - 2) >> 2;
     int64_t ti = 0;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
-      const int64_t m0 = (tile % m_tiles) * kGM, n0 = (tile / m_tiles) * kPN;
+      int64_t m0, n0;
+      tile_coords(tile, m_tiles, n_col_tiles, m0, n0);
       const bool ok = wait_parity(&sm.acc_full, uint32_t(ti & 1));
       if (!ok) atomicExch(&sm.failed, 1);
       asm volatile("tcgen05.fence::after_thread_sync;");
