@@ -90,7 +90,7 @@ OP_SOURCES = {
     "quant_cols_sr": ("quantize.cu",) + _COMMON_SOURCES,
     "double_quant": ("quantize.cu",) + _COMMON_SOURCES,
     "dequant_rows": ("quantize.cu",) + _COMMON_SOURCES,
-    "rht_quant_sr": ("rht.cu",) + _COMMON_SOURCES,
+    "rht_quant_sr": ("rht.cu", "tc_common.cuh") + _COMMON_SOURCES,
     "osc_update": ("osc.cu",) + _COMMON_SOURCES,
     "osc_step": ("osc.cu",) + _COMMON_SOURCES,
 }

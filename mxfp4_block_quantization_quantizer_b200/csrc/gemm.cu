@@ -38,6 +38,7 @@
 
 #include "launch.cuh"
 #include "mxfp4_device.cuh"
+#include "tc_common.cuh"
 
 namespace mxfp4 {
 
@@ -51,7 +52,6 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kAccCol = 0;    // 128 fp32 columns
 constexpr uint32_t kSfaCol = 128;  // two 4-column scale tiles
 constexpr uint32_t kSfbCol = 136;
-constexpr long long kWaitLimit = 1ll << 22;
 
 struct __align__(1024) GemmSmem {
   uint8_t a[kGChunks][kGM][16];
@@ -62,22 +62,6 @@ struct __align__(1024) GemmSmem {
   uint32_t tmem_base;
   int failed;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Matrix descriptor of a K-major operand in shared memory without swizzle:
-// start address, leading byte offset (between 16-byte K columns), stride
-// byte offset (between 8-row groups), all in 16-byte units; version 1.
-__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo,
-                                              uint32_t sbo) {
-  uint64_t d = (smem_u32(p) >> 4) & 0x3FFFu;
-  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
-  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
-  d |= uint64_t(1) << 46;
-  return d;
-}
 
 // Instruction descriptor of kind::mxf4: E2M1 A and B (format 1), K-major
 // both, N/8 at bit 17, E8M0 scales (bit 23), M/16 at bit 24; the scale
@@ -110,22 +94,6 @@ __device__ __forceinline__ void copy_scales_to_tmem(uint32_t taddr,
 // As copy_scales_to_tmem, with the source descriptor given.
 __device__ __forceinline__ void copy_scales_desc(uint32_t taddr, uint64_t d) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d));
-}
-__device__ __forceinline__ bool wait_parity(unsigned long long* bar,
-                                            uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  for (long long i = 0; i < kWaitLimit; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
 }
 
 __global__ void __launch_bounds__(kGThreads)
@@ -303,33 +271,6 @@ struct __align__(1024) PipeSmem {
   int failed;
 };
 
-// Descriptor of a 128-byte-swizzled K-major operand: 8-row groups 1024
-// bytes apart; the start address moves 32 bytes per K = 64 step inside the
-// 128-byte swizzle row.
-__device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
-  uint64_t d = (smem_u32(p) >> 4) & 0x3FFFu;
-  d |= uint64_t(1) << 16;                  // leading byte offset (unused)
-  d |= uint64_t(1024 >> 4) << 32;          // stride byte offset
-  d |= uint64_t(1) << 46;                  // version
-  d |= uint64_t(2) << 61;                  // 128-byte swizzle
-  return d;
-}
-
-__device__ __forceinline__ void expect_tx(unsigned long long* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x,
-                                            int y, unsigned long long* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           unsigned long long* bar) {
   asm volatile(
@@ -360,15 +301,6 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ bool failed_flag(const int* f) {
-  return *static_cast<const volatile int*>(f) != 0;
-}
-
-__device__ __forceinline__ void commit_to(unsigned long long* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar)));
-}
 
 __global__ void __launch_bounds__(kPThreads, 1)
     k_gemm_mxf4_pipe(const __grid_constant__ CUtensorMap tm_a,
@@ -614,33 +546,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 // 2-D map over K-major codes [rows][k/2]: boxes of 128 bytes x box_rows,
 // 128-byte swizzle, zero fill outside the tensor.
 bool encode_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t k,
                       uint32_t box_rows) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(k / 2), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(k / 2)};
-  const cuuint32_t box[2] = {128, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
-             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return encode_rows_sw128(map, codes, rows, k / 2, box_rows);
 }
 
 // 2-D map over fp32 C [m][n] for the epilogue's stores: boxes of 32 rows x
