@@ -367,15 +367,18 @@ __device__ __forceinline__ void stage_tile_async(const void* __restrict__ x,
                                                  uint4* tile) {
   using T = ColTile<BF16>;
   constexpr int kPer = kTileRows * T::kChunksPerRow / T::kThreads;
+  static_assert(T::kThreads % T::kChunksPerRow == 0, "whole rows per pass");
+  constexpr int kRowStep = T::kThreads / T::kChunksPerRow;  // rows per pass
+  // this thread's chunk column is the same in every pass
+  const int r0 = threadIdx.x / T::kChunksPerRow, ch = threadIdx.x % T::kChunksPerRow;
+  const int64_t gc = tile_c + int64_t(ch) * T::kChunkElems;
+  const bool col_ok = gc < cols;
+  const char* src = static_cast<const char*>(x) + ((tile_r + r0) * cols + gc) * T::kElemBytes;
+  const int64_t step = int64_t(kRowStep) * cols * T::kElemBytes;
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int idx = k * T::kThreads + threadIdx.x;
-    const int r = idx / T::kChunksPerRow, ch = idx % T::kChunksPerRow;
-    const int64_t gr = tile_r + r, gc = tile_c + int64_t(ch) * T::kChunkElems;
-    const bool ok = gr < rows && gc < cols;
-    const char* src = static_cast<const char*>(x) +
-                      (ok ? (gr * cols + gc) * T::kElemBytes : 0);
-    cp_async16(tile + idx, src, ok);
+  for (int k = 0; k < kPer; ++k, src += step) {
+    const bool ok = col_ok && tile_r + r0 + k * kRowStep < rows;
+    cp_async16(tile + k * T::kThreads + threadIdx.x, ok ? src : x, ok);
   }
   cp_async_commit();
 }
@@ -638,11 +641,9 @@ __global__ void __launch_bounds__(kDqThreads)
 // writes the row codes and scale to global memory (when in range) and stages
 // the codes and the scale value 2^e in shared memory for the column pass.
 __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool ok,
-                                             int64_t gr, int64_t gc, int64_t cols,
-                                             int tr, int ch,
-                                             uint8_t* __restrict__ row_codes,
-                                             uint8_t* __restrict__ row_scales,
-                                             uint32_t* s_codes, float* s_scales) {
+                                             int tr, int ch, uint8_t* __restrict__ rc,
+                                             uint8_t* __restrict__ rs, uint32_t* s_codes,
+                                             float* s_scales) {
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   const uint32_t sb = scale_byte(amax);
@@ -652,8 +653,8 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
   uint32_t word = e2m1x8_rn(v);
   if (sb == 0xFFu) word = 0;
   if (ok) {
-    *reinterpret_cast<uint32_t*>(row_codes + gr * (cols / 2) + gc / 2) = word;
-    if ((ch & 3) == 0) row_scales[gr * (cols / 32) + gc / 32] = uint8_t(sb);
+    *reinterpret_cast<uint32_t*>(rc) = word;
+    if ((ch & 3) == 0) *rs = uint8_t(sb);
   }
   s_codes[tr * (kDqCols / 8) + ch] = word;
   if ((ch & 3) == 0) s_scales[tr * (kDqCols / 32) + ch / 4] = scale_value(sb);
@@ -743,15 +744,19 @@ __global__ void __launch_bounds__(kDqThreads, 3)
     const int64_t tile_c = (t % tiles_c) * kDqCols;
     const int64_t gc = tile_c + 8 * ch;
     const uint4* raw = smem + buf * kChunks;
+    // this thread's row outputs: rows tile_r + rr + 16k, columns gc .. gc+7
+    uint8_t* rc = row_codes + (tile_r + rr) * (cols / 2) + gc / 2;
+    uint8_t* rs = row_scales + (tile_r + rr) * (cols / 32) + gc / 32;
+    const int64_t rc_step = 16 * (cols / 2), rs_step = 16 * (cols / 32);
+    const bool col_ok = gc < cols;
 #pragma unroll 2
-    for (int k = 0; k < kTileRows / 16; ++k) {
+    for (int k = 0; k < kTileRows / 16; ++k, rc += rc_step, rs += rs_step) {
       const int tr = rr + 16 * k;
-      const int64_t gr = tile_r + tr;
       const uint4 w = raw[tr * (kDqCols / 8) + ch];
       float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
                     bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-      dq_row_chunk(v, bf16x8_absmax(w), gr < rows && gc < cols, gr, gc, cols,
-                   tr, ch, row_codes, row_scales, s_codes, s_scales);
+      dq_row_chunk(v, bf16x8_absmax(w), col_ok && tile_r + tr < rows, tr, ch, rc, rs,
+                   s_codes, s_scales);
     }
     __syncthreads();
     static_assert(ColStage<kDqCols>::kBytes <= kChunks * 16, "stage fits a tile");
