@@ -409,6 +409,27 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads)
   }
 }
 
+// Row and column of the tiles first, first + stride, ... of a grid with
+// n_c tile columns (tile t = row * n_c + column), advanced without a 64-bit
+// division per step (one division when constructed).
+struct TileWalk {
+  int64_t r, c, dr, dc, n_c;
+  __device__ __forceinline__ TileWalk(int64_t first, int64_t stride, int64_t nc) : n_c(nc) {
+    r = first / nc;
+    c = first - r * nc;
+    dr = stride / nc;
+    dc = stride - dr * nc;
+  }
+  __device__ __forceinline__ void next() {
+    r += dr;
+    c += dc;
+    if (c >= n_c) {
+      c -= n_c;
+      ++r;
+    }
+  }
+};
+
 // Column groups, 16-byte aligned rows: double-buffered. The copies of the
 // CTA's next tile are in flight while the current tile is quantized; the
 // tile's column codes are staged and leave as whole 64-byte runs.
@@ -429,19 +450,20 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
   const int rg = threadIdx.x / (T::kCols / 2);
   int64_t t = blockIdx.x;
   if (t >= n_tiles) return;
-  stage_tile_async<BF16>(x, rows, cols, (t / tiles_c) * kTileRows,
-                         (t % tiles_c) * T::kCols, smem);
-  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+  TileWalk cur(t, gridDim.x, tiles_c), nxt = cur;
+  nxt.next();
+  stage_tile_async<BF16>(x, rows, cols, cur.r * kTileRows, cur.c * T::kCols, smem);
+  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
     const int64_t tn = t + gridDim.x;
     if (tn < n_tiles)
-      stage_tile_async<BF16>(x, rows, cols, (tn / tiles_c) * kTileRows,
-                             (tn % tiles_c) * T::kCols, smem + (buf ^ 1) * kChunks);
+      stage_tile_async<BF16>(x, rows, cols, nxt.r * kTileRows, nxt.c * T::kCols,
+                             smem + (buf ^ 1) * kChunks);
     else
       cp_async_commit();  // keep one group per iteration
     cp_async_wait<1>();   // this tile's copies (the older group) are done
     __syncthreads();
-    const int64_t tile_r = (t / tiles_c) * kTileRows;
-    const int64_t tile_c = (t % tiles_c) * T::kCols;
+    const int64_t tile_r = cur.r * kTileRows;
+    const int64_t tile_c = cur.c * T::kCols;
     if (tile_r + 32 * rg < rows)
       stage_column_pair(column_tile_pass<BF16, SR, EVEN, BIG, OAS>(
                             smem + buf * kChunks, T::kCols, rg, cp, tile_r,
@@ -729,19 +751,20 @@ __global__ void __launch_bounds__(kDqThreads, 3)
   const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
   int64_t t = blockIdx.x;
   if (t >= n_tiles) return;
-  stage_tile_async<true>(x, rows, cols, (t / tiles_c) * kTileRows,
-                         (t % tiles_c) * kDqCols, smem);
-  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1) {
+  TileWalk cur(t, gridDim.x, tiles_c), nxt = cur;
+  nxt.next();
+  stage_tile_async<true>(x, rows, cols, cur.r * kTileRows, cur.c * kDqCols, smem);
+  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
     const int64_t tn = t + gridDim.x;
     if (tn < n_tiles)
-      stage_tile_async<true>(x, rows, cols, (tn / tiles_c) * kTileRows,
-                             (tn % tiles_c) * kDqCols, smem + (buf ^ 1) * kChunks);
+      stage_tile_async<true>(x, rows, cols, nxt.r * kTileRows, nxt.c * kDqCols,
+                             smem + (buf ^ 1) * kChunks);
     else
       cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
-    const int64_t tile_r = (t / tiles_c) * kTileRows;
-    const int64_t tile_c = (t % tiles_c) * kDqCols;
+    const int64_t tile_r = cur.r * kTileRows;
+    const int64_t tile_c = cur.c * kDqCols;
     const int64_t gc = tile_c + 8 * ch;
     const uint4* raw = smem + buf * kChunks;
     // this thread's row outputs: rows tile_r + rr + 16k, columns gc .. gc+7

@@ -334,8 +334,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 #pragma unroll
     for (int s = 0; s < kRtStages; ++s) slot_cb[s] = -1;
     uint32_t s = 0, ph = 0;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-      const int64_t cb = t / n_rt, rt = t % n_rt;
+    int64_t cb = t_begin / n_rt, rt = t_begin % n_rt;
+    for (int64_t t = t_begin; t < t_end; ++t, rt = rt + 1 == n_rt ? 0 : rt + 1,
+                 cb += rt == 0 ? 1 : 0) {
       if (!wait_parity(&sm.empty[s], ph ^ 1u)) {
         atomicExch(&sm.failed, 1);
         break;
@@ -429,8 +430,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     const int q = warp & 3, gs = (warp - 2) >> 2;
     constexpr int kPer = kRtGroups / 4;  // groups per thread and tile
     uint32_t b = 0, bph = 0;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-      const int64_t cb = t / n_rt, rt = t % n_rt;
+    int64_t cb = t_begin / n_rt, rt = t_begin % n_rt;
+    for (int64_t t = t_begin; t < t_end; ++t, rt = rt + 1 == n_rt ? 0 : rt + 1,
+                 cb += rt == 0 ? 1 : 0) {
       const int64_t r = rt * 128 + 32 * q + lane;
       // after a failure every warp still runs every tile (without waiting),
       // so the quarter barriers of the staged stores stay matched
