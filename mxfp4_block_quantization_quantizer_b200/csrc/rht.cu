@@ -134,6 +134,9 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
     }
     const uint32_t sb = scale_byte(amax);
     const float mul = ROT ? inv_scale(sb) : inv_scale(sb) * kInvSqrt32;
+    // the group's 16 pairs share the high word of their index
+    const uint64_t pg = uint64_t(e0 >> 1);
+    const uint32_t kh = SR ? inner_key(key, uint32_t(pg >> 32)) : 0u;
     uint32_t wq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -141,11 +144,10 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
       if (SR) {
-        const uint64_t p0 = uint64_t(e0 >> 1) + 4 * q;
-        const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
+        const uint32_t p0 = uint32_t(pg) + 4 * q;
         uint32_t h[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + uint32_t(p0) + t);
+        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + p0 + t);
         wq[q] = e2m1x8_sr(v, h);
       } else {
         wq[q] = e2m1x8_rn(v);
@@ -259,6 +261,10 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
   }
   const uint32_t sb = failed ? 0xFFu : scale_byte(amax);
   const float mul = ROT ? inv_scale(sb) : inv_scale(sb) * kInvSqrt32;
+  // the group's 16 pairs start at a multiple of 16, so they share the high
+  // word of their index (2^32 is a multiple of 16): one inner key
+  const uint64_t pg = uint64_t(e0 >> 1);
+  const uint32_t kh = SR ? inner_key(key, uint32_t(pg >> 32)) : 0u;
   uint32_t wq[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -266,11 +272,10 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
     if (SR) {
-      const uint64_t p0 = uint64_t(e0 >> 1) + 4 * q;
-      const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
+      const uint32_t p0 = uint32_t(pg) + 4 * q;
       uint32_t h[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + uint32_t(p0) + t);
+      for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + p0 + t);
       wq[q] = e2m1x8_sr(v, h);
     } else {
       wq[q] = e2m1x8_rn(v);
