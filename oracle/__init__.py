@@ -71,9 +71,13 @@ def _declare(L):
         "orc_dequantize": ([_u8p, _u8p, i64, i64, i32, vp, i32], i32),
         "orc_double_quantize": ([vp, i32, i64, i64, i64, u64, _u8p, _u8p,
                                  _u8p, _u8p], i32),
+        "orc_double_quantize_oas": ([vp, i32, i64, i64, i64, u64, _u8p, _u8p,
+                                     _u8p, _u8p], i32),
         "orc_rht_rotate": ([vp, i32, i64, i64, u64, _fp], i32),
         "orc_rht_quantize": ([vp, i32, i64, i64, i64, u64, i32, u64, _u8p,
                               _u8p, _fp], i32),
+        "orc_rht_quantize_oas": ([vp, i32, i64, i64, i64, u64, i32, u64, _u8p,
+                                  _u8p, _fp], i32),
         "orc_osc_step": ([_fp, _fp, _fp, _fp, i64, i64, i32, ctypes.c_float],
                          i64),
         "orc_osc_synthetic_update": ([_fp, i64, i64, i64, u64, u32,
@@ -172,15 +176,15 @@ class Oracle:
                               y.ctypes.data, dt)
         return y.view(ml_dtypes.bfloat16) if dt == DT_BF16 else y
 
-    def double_quantize(self, x, seed, row0=0):
+    def double_quantize(self, x, seed, row0=0, oas=False):
         """Q_S(32x1)(Q_D(1x32)(x)): (row codes, row scales, col codes,
-        col scales)."""
+        col scales); oas: the overflow-aware scale in both passes."""
         x, dt = _as_input(x)
         R, C = x.shape
         out = [np.zeros(R * C // 2, np.uint8), np.zeros(R * C // 32, np.uint8),
                np.zeros(R * C // 2, np.uint8), np.zeros(R * C // 32, np.uint8)]
-        rc = self.L.orc_double_quantize(x.ctypes.data, dt, R, C, row0, seed,
-                                        *[_u8(a) for a in out])
+        fn = self.L.orc_double_quantize_oas if oas else self.L.orc_double_quantize
+        rc = fn(x.ctypes.data, dt, R, C, row0, seed, *[_u8(a) for a in out])
         if rc != 0:
             raise ValueError("bad shape for the oracle double quantizer")
         return (out[0].reshape(R, C // 2), out[1].reshape(R, C // 32),
@@ -194,17 +198,17 @@ class Oracle:
             raise ValueError("bad shape for the oracle rotation")
         return y
 
-    def rht_quantize(self, x, sign_seed, rounding, sr_seed, row0=0):
+    def rht_quantize(self, x, sign_seed, rounding, sr_seed, row0=0, oas=False):
         """Rotate each 1x32 row group, quantize along rows: (codes, scales,
-        rotated fp32)."""
+        rotated fp32); oas: the overflow-aware scale."""
         x, dt = _as_input(x)
         R, C = x.shape
         codes = np.zeros(R * C // 2, np.uint8)
         scales = np.zeros(R * C // 32, np.uint8)
         y = np.zeros((R, C), np.float32)
-        if self.L.orc_rht_quantize(x.ctypes.data, dt, R, C, row0, sign_seed,
-                                   rounding, sr_seed, _u8(codes),
-                                   _u8(scales), _f32(y)):
+        fn = self.L.orc_rht_quantize_oas if oas else self.L.orc_rht_quantize
+        if fn(x.ctypes.data, dt, R, C, row0, sign_seed, rounding, sr_seed, _u8(codes),
+              _u8(scales), _f32(y)):
             raise ValueError("bad shape for the oracle rotation")
         return codes.reshape(R, C // 2), scales.reshape(R, C // 32), y
 

@@ -353,23 +353,41 @@ int orc_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows,
   return 0;
 }
 
-/* [TJ] Question 2: Q_S along 32x1 groups of the dequantized Q_D(1x32)(X). */
-int orc_double_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
-                        int64_t row0, uint64_t seed, uint8_t* row_codes,
-                        uint8_t* row_scales, uint8_t* col_codes,
-                        uint8_t* col_scales) {
+/* [TJ] Question 2: Q_S along 32x1 groups of the dequantized Q_D(1x32)(X),
+ * both passes with the scale rule given. */
+static int double_quantize_rule(const void* x, int dtype, int64_t rows, int64_t cols,
+                                int64_t row0, uint64_t seed, int scale_rule,
+                                uint8_t* row_codes, uint8_t* row_scales,
+                                uint8_t* col_codes, uint8_t* col_scales) {
   if (rows <= 0 || cols <= 0 || rows % 32 || cols % 32) return -1;
   int64_t n = rows * cols;
   double* xv = load_all(x, dtype, n);
-  quantize_values(xv, rows, cols, row0, AX_ROWS, RND_RNE, 0, SCALE_OCP, row_codes,
+  quantize_values(xv, rows, cols, row0, AX_ROWS, RND_RNE, 0, scale_rule, row_codes,
                   row_scales);
   double* d = (double*)malloc((size_t)n * sizeof(double));
   dequantize_values(row_codes, row_scales, rows, cols, AX_ROWS, d);
-  quantize_values(d, rows, cols, row0, AX_COLS, RND_SR, seed, SCALE_OCP, col_codes,
+  quantize_values(d, rows, cols, row0, AX_COLS, RND_SR, seed, scale_rule, col_codes,
                   col_scales);
   free(d);
   free(xv);
   return 0;
+}
+
+int orc_double_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
+                        int64_t row0, uint64_t seed, uint8_t* row_codes,
+                        uint8_t* row_scales, uint8_t* col_codes,
+                        uint8_t* col_scales) {
+  return double_quantize_rule(x, dtype, rows, cols, row0, seed, SCALE_OCP, row_codes,
+                              row_scales, col_codes, col_scales);
+}
+
+/* orc_double_quantize with the overflow-aware scale in both passes. */
+int orc_double_quantize_oas(const void* x, int dtype, int64_t rows, int64_t cols,
+                            int64_t row0, uint64_t seed, uint8_t* row_codes,
+                            uint8_t* row_scales, uint8_t* col_codes,
+                            uint8_t* col_scales) {
+  return double_quantize_rule(x, dtype, rows, cols, row0, seed, SCALE_OAS, row_codes,
+                              row_scales, col_codes, col_scales);
 }
 
 /* Sign of column c for the randomized Hadamard transform: -1 iff bit 31 of
@@ -408,19 +426,39 @@ int orc_rht_rotate(const void* x, int dtype, int64_t rows, int64_t cols,
   return 0;
 }
 
-/* Rotate, then quantize the fp32 rotated values along rows. `rotated`
- * receives y when not NULL. */
+/* Rotate, then quantize the fp32 rotated values along rows (OCP or
+ * overflow-aware scale). `rotated` receives y when not NULL. */
+static int rht_quantize_rule(const void* x, int dtype, int64_t rows, int64_t cols,
+                             int64_t row0, uint64_t sign_seed, int rounding,
+                             uint64_t sr_seed, int scale_rule, uint8_t* codes,
+                             uint8_t* scales, float* rotated) {
+  if (rows <= 0 || cols <= 0 || cols % 32) return -1;
+  float* y = rotated ? rotated : (float*)malloc((size_t)(rows * cols) * 4);
+  orc_rht_rotate(x, dtype, rows, cols, sign_seed, y);
+  if (scale_rule == SCALE_OAS)
+    orc_quantize_oas(y, DT_F32, rows, cols, row0, AX_ROWS, rounding, sr_seed, codes,
+                     scales);
+  else
+    orc_quantize(y, DT_F32, rows, cols, row0, AX_ROWS, rounding, sr_seed, codes, scales);
+  if (!rotated) free(y);
+  return 0;
+}
+
 int orc_rht_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
                      int64_t row0, uint64_t sign_seed, int rounding,
                      uint64_t sr_seed, uint8_t* codes, uint8_t* scales,
                      float* rotated) {
-  if (rows <= 0 || cols <= 0 || cols % 32) return -1;
-  float* y = rotated ? rotated : (float*)malloc((size_t)(rows * cols) * 4);
-  orc_rht_rotate(x, dtype, rows, cols, sign_seed, y);
-  orc_quantize(y, DT_F32, rows, cols, row0, AX_ROWS, rounding, sr_seed,
-               codes, scales);
-  if (!rotated) free(y);
-  return 0;
+  return rht_quantize_rule(x, dtype, rows, cols, row0, sign_seed, rounding, sr_seed,
+                           SCALE_OCP, codes, scales, rotated);
+}
+
+/* orc_rht_quantize with the overflow-aware scale. */
+int orc_rht_quantize_oas(const void* x, int dtype, int64_t rows, int64_t cols,
+                         int64_t row0, uint64_t sign_seed, int rounding,
+                         uint64_t sr_seed, uint8_t* codes, uint8_t* scales,
+                         float* rotated) {
+  return rht_quantize_rule(x, dtype, rows, cols, row0, sign_seed, rounding, sr_seed,
+                           SCALE_OAS, codes, scales, rotated);
 }
 
 /* ------------------------------------------------------------------ */

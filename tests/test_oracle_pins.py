@@ -708,3 +708,50 @@ def test_oas_stochastic_rounding_unbiased_where_ocp_saturates():
     # one step at e = 1 is 2.0 around 7.3 and 1.0 around 2.9
     assert abs(means[0] - 7.3) < 4 * 1.0 / np.sqrt(S) + 2.0 * 2.0 ** -17
     assert abs(means[1] - 2.9) < 4 * 0.5 / np.sqrt(S) + 1.0 * 2.0 ** -17
+
+
+def _sweep_like(shape, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    x = g.standard_normal(shape).astype(np.float32)
+    x.reshape(-1)[:: 97] *= 100.0
+    return x.astype(BF16)
+
+
+def test_double_quantize_oas_is_the_composition_of_oas_quantizers():
+    """Overflow-aware double quantization: the row outputs are the
+    overflow-aware nearest quantization of X, the column outputs the
+    overflow-aware stochastic quantization of their decoded values."""
+    x = _sweep_like((96, 128), 61)
+    rc, rs, cc, cs = O.double_quantize(x, 7, oas=True)
+    wr, ws = O.quantize(x, O.ROWS, O.RNE, oas=True)
+    assert np.array_equal(rc, wr) and np.array_equal(rs, ws)
+    d = O.dequantize(rc, rs, 96, 128, O.ROWS, "f32")
+    wc, wcs = O.quantize(d, O.COLS, O.SR, 7, oas=True)
+    assert np.array_equal(cc, wc) and np.array_equal(cs, wcs)
+
+
+def test_double_quantize_oas_column_scales_equal_the_ocp_rule():
+    """Decoded values have two significant bits (mantissa 1 or 1.5), so a
+    column maximum never scales above 6 under the OCP exponent and the two
+    rules pick the same column scales and codes."""
+    x = _sweep_like((64, 96), 62)
+    rc, rs, cc, cs = O.double_quantize(x, 3, oas=True)
+    d = O.dequantize(rc, rs, 64, 96, O.ROWS, "f32")
+    oc, ocs = O.quantize(d, O.COLS, O.SR, 3)
+    assert np.array_equal(cc, oc) and np.array_equal(cs, ocs)
+    # while the row pass does move: some group maximum scaled above 6
+    _, rs_ocp, _, _ = O.double_quantize(x, 3)
+    assert np.any(rs != rs_ocp)
+
+
+def test_rht_quantize_oas_never_saturates():
+    """Overflow-aware rotation: the codes are the overflow-aware quantization
+    of the rotated values, and every group maximum scales to at most 6."""
+    x = _sweep_like((16, 256), 63)
+    for rnd in (O.RNE, O.SR):
+        c, s, y = O.rht_quantize(x, 5, rnd, 9, oas=True)
+        wc, ws = O.quantize(y, O.ROWS, rnd, 9, oas=True)
+        assert np.array_equal(c, wc) and np.array_equal(s, ws)
+        gmax = np.abs(y.astype(np.float64)).reshape(-1, 32).max(axis=1)
+        e = s.reshape(-1).astype(np.int64) - 127
+        assert np.all(gmax * np.exp2(-e.astype(np.float64)) <= 6.0)
