@@ -142,11 +142,28 @@ mxfp4_status mxfp4_double_quantize(const void* x, int dtype, int64_t rows,
                                    void* stream);
 
 /*
+ * mxfp4_double_quantize with the overflow-aware scale (as mxfp4_quantize_oas)
+ * in both passes. The row pass moves where a group maximum would scale above
+ * 6; the column pass then sees decoded values with two significant bits,
+ * whose maxima never scale above 6, so its scales follow the OCP rule as
+ * well. Same arguments, layouts and statuses as mxfp4_double_quantize.
+ * Source: "Unveiling the Potential of Quantization with MXFP4", abstract
+ * (overflow-aware scaling), with the double quantization above.
+ */
+mxfp4_status mxfp4_double_quantize_oas(const void* x, int dtype, int64_t rows,
+                                       int64_t cols, uint64_t seed,
+                                       uint8_t* row_codes, uint8_t* row_scales,
+                                       uint8_t* col_codes, uint8_t* col_scales,
+                                       void* stream);
+
+/*
  * Randomized Hadamard rotation of every 1x32 row group followed by 1x32
  * quantization: y_g = (1/sqrt(32)) * H32 * (s .* x_g), H32 the Sylvester
  * Hadamard matrix (H[j][k] = (-1)^popcount(j&k)), s_c = -1 iff bit 31 of
- * mix(K(sign_seed, 1) + c) is set for column c; fp32 arithmetic. y is then
- * quantized along ROWS with `rounding` (SR keyed by sr_seed).
+ * mix(K(sign_seed, 1) + c) is set for column c; fp32 arithmetic (bf16
+ * inputs: exact +-1 products summed in fp32 on the tensor cores; fp32
+ * inputs: a radix-2 butterfly). y is then quantized along ROWS with
+ * `rounding` (SR keyed by sr_seed).
  * Sources: ALTO explainer, Jargon: Randomized Hadamard transform; "Microscaling
  * FP4 Quantization: MR-GPTQ Achieves 6x Speedup", section "FP4 Quantization
  * with Micro-Rotated GPTQ Algorithm" (block-wise Hadamard transforms).
@@ -159,6 +176,16 @@ mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
                                 int rounding, uint64_t sr_seed,
                                 uint8_t* codes, uint8_t* scales,
                                 float* rotated, void* stream);
+
+/*
+ * mxfp4_rht_quantize with the overflow-aware scale (as mxfp4_quantize_oas)
+ * for the rotated values. Same arguments, layouts and statuses.
+ */
+mxfp4_status mxfp4_rht_quantize_oas(const void* x, int dtype, int64_t rows,
+                                    int64_t cols, uint64_t sign_seed,
+                                    int rounding, uint64_t sr_seed,
+                                    uint8_t* codes, uint8_t* scales,
+                                    float* rotated, void* stream);
 
 /*
  * One step of the weight-oscillation tracker on fp32 master weights w.

@@ -20,8 +20,8 @@ RNE, SR = 0, 1
 
 # Every symbol include/mxfp4.h declares.
 SYMBOLS = ("mxfp4_quantize", "mxfp4_quantize_oas", "mxfp4_dequantize",
-           "mxfp4_double_quantize",
-           "mxfp4_rht_quantize", "mxfp4_osc_step",
+           "mxfp4_double_quantize", "mxfp4_double_quantize_oas",
+           "mxfp4_rht_quantize", "mxfp4_rht_quantize_oas", "mxfp4_osc_step",
            "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
            "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_status_string")
 
@@ -54,8 +54,12 @@ def lib():
             "mxfp4_dequantize": [vp, vp, i64, i64, i32, vp, i32, vp],
             "mxfp4_double_quantize": [vp, i32, i64, i64, u64, vp, vp, vp, vp,
                                       vp],
+            "mxfp4_double_quantize_oas": [vp, i32, i64, i64, u64, vp, vp, vp,
+                                          vp, vp],
             "mxfp4_rht_quantize": [vp, i32, i64, i64, u64, i32, u64, vp, vp,
                                    vp, vp],
+            "mxfp4_rht_quantize_oas": [vp, i32, i64, i64, u64, i32, u64, vp,
+                                       vp, vp, vp],
             "mxfp4_osc_step": [vp, vp, vp, vp, i64, i64, i32, ctypes.c_float,
                                vp, vp],
             "mxfp4_osc_synthetic_update": [vp, i64, i64, u64, u32,
@@ -145,8 +149,9 @@ def dequantize(codes, scales, rows, cols, axis=ROWS, out_dtype=torch.bfloat16,
     return out
 
 
-def double_quantize(x, seed=0, out=None, stream=None):
-    """mxfp4_double_quantize: (row_codes, row_scales, col_codes, col_scales)."""
+def double_quantize(x, seed=0, out=None, stream=None, oas=False):
+    """mxfp4_double_quantize (mxfp4_double_quantize_oas when oas):
+    (row_codes, row_scales, col_codes, col_scales)."""
     _cuda2d(x, "x")
     R, C = x.shape
     if out is None:
@@ -154,16 +159,18 @@ def double_quantize(x, seed=0, out=None, stream=None):
         out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d),
                _empty_u8((C, R // 2), d), _empty_u8((C, R // 32), d))
     rc, rs, cc, cs = out
-    _check(lib().mxfp4_double_quantize(_ptr(x), _dtype_code(x), R, C, seed,
-                                       _ptr(rc), _ptr(rs), _ptr(cc), _ptr(cs),
-                                       _stream(x.device, stream)),
-           "mxfp4_double_quantize")
+    name = "mxfp4_double_quantize_oas" if oas else "mxfp4_double_quantize"
+    _check(getattr(lib(), name)(_ptr(x), _dtype_code(x), R, C, seed, _ptr(rc),
+                                _ptr(rs), _ptr(cc), _ptr(cs),
+                                _stream(x.device, stream)),
+           name)
     return out
 
 
 def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
-                 out=None, stream=None):
-    """mxfp4_rht_quantize: (codes, scales, rotated or None), ROWS layout."""
+                 out=None, stream=None, oas=False):
+    """mxfp4_rht_quantize (mxfp4_rht_quantize_oas when oas): (codes, scales,
+    rotated or None), ROWS layout."""
     _cuda2d(x, "x")
     R, C = x.shape
     if out is None:
@@ -171,11 +178,11 @@ def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
         rot = torch.empty((R, C), dtype=torch.float32, device=d) if want_rotated else None
         out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d), rot)
     codes, scales, rot = out
-    _check(lib().mxfp4_rht_quantize(_ptr(x), _dtype_code(x), R, C, sign_seed,
-                                    rounding, sr_seed, _ptr(codes),
-                                    _ptr(scales), _ptr(rot),
-                                    _stream(x.device, stream)),
-           "mxfp4_rht_quantize")
+    name = "mxfp4_rht_quantize_oas" if oas else "mxfp4_rht_quantize"
+    _check(getattr(lib(), name)(_ptr(x), _dtype_code(x), R, C, sign_seed, rounding,
+                                sr_seed, _ptr(codes), _ptr(scales), _ptr(rot),
+                                _stream(x.device, stream)),
+           name)
     return out
 
 

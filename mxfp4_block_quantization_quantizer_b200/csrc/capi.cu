@@ -88,11 +88,11 @@ mxfp4_status mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales,
                                          as_stream(stream)));
 }
 
-mxfp4_status mxfp4_double_quantize(const void* x, int dtype, int64_t rows,
-                                   int64_t cols, uint64_t seed,
-                                   uint8_t* row_codes, uint8_t* row_scales,
-                                   uint8_t* col_codes, uint8_t* col_scales,
-                                   void* stream) {
+static mxfp4_status double_quantize_with_rule(const void* x, int dtype, int64_t rows,
+                                              int64_t cols, uint64_t seed,
+                                              uint8_t* row_codes, uint8_t* row_scales,
+                                              uint8_t* col_codes, uint8_t* col_scales,
+                                              void* stream, bool oas) {
   if (!dtype_ok(dtype)) return MXFP4_ERR_ENUM;
   if (!x || !row_codes || !row_scales || !col_codes || !col_scales)
     return MXFP4_ERR_NULL;
@@ -101,14 +101,32 @@ mxfp4_status mxfp4_double_quantize(const void* x, int dtype, int64_t rows,
     return MXFP4_ERR_ALIGN;
   return from_cuda(mxfp4::launch_double_quant(
       x, dtype == MXFP4_BF16, rows, cols, seed, row_codes, row_scales,
-      col_codes, col_scales, as_stream(stream)));
+      col_codes, col_scales, as_stream(stream), oas));
 }
 
-mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
-                                int64_t cols, uint64_t sign_seed,
-                                int rounding, uint64_t sr_seed,
-                                uint8_t* codes, uint8_t* scales,
-                                float* rotated, void* stream) {
+mxfp4_status mxfp4_double_quantize(const void* x, int dtype, int64_t rows,
+                                   int64_t cols, uint64_t seed,
+                                   uint8_t* row_codes, uint8_t* row_scales,
+                                   uint8_t* col_codes, uint8_t* col_scales,
+                                   void* stream) {
+  return double_quantize_with_rule(x, dtype, rows, cols, seed, row_codes, row_scales,
+                                   col_codes, col_scales, stream, false);
+}
+
+mxfp4_status mxfp4_double_quantize_oas(const void* x, int dtype, int64_t rows,
+                                       int64_t cols, uint64_t seed,
+                                       uint8_t* row_codes, uint8_t* row_scales,
+                                       uint8_t* col_codes, uint8_t* col_scales,
+                                       void* stream) {
+  return double_quantize_with_rule(x, dtype, rows, cols, seed, row_codes, row_scales,
+                                   col_codes, col_scales, stream, true);
+}
+
+static mxfp4_status rht_quantize_with_rule(const void* x, int dtype, int64_t rows,
+                                           int64_t cols, uint64_t sign_seed,
+                                           int rounding, uint64_t sr_seed,
+                                           uint8_t* codes, uint8_t* scales,
+                                           float* rotated, void* stream, bool oas) {
   if (!dtype_ok(dtype) || !rounding_ok(rounding)) return MXFP4_ERR_ENUM;
   if (!x || !codes || !scales) return MXFP4_ERR_NULL;
   if (!dims_ok(rows, cols) || cols % 32) return MXFP4_ERR_SHAPE;
@@ -116,7 +134,25 @@ mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
     return MXFP4_ERR_ALIGN;
   return from_cuda(mxfp4::launch_rht_quant(
       x, dtype == MXFP4_BF16, rows, cols, sign_seed, rounding == MXFP4_SR,
-      sr_seed, codes, scales, rotated, as_stream(stream)));
+      sr_seed, codes, scales, rotated, as_stream(stream), oas));
+}
+
+mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
+                                int64_t cols, uint64_t sign_seed,
+                                int rounding, uint64_t sr_seed,
+                                uint8_t* codes, uint8_t* scales,
+                                float* rotated, void* stream) {
+  return rht_quantize_with_rule(x, dtype, rows, cols, sign_seed, rounding, sr_seed, codes,
+                                scales, rotated, stream, false);
+}
+
+mxfp4_status mxfp4_rht_quantize_oas(const void* x, int dtype, int64_t rows,
+                                    int64_t cols, uint64_t sign_seed,
+                                    int rounding, uint64_t sr_seed,
+                                    uint8_t* codes, uint8_t* scales,
+                                    float* rotated, void* stream) {
+  return rht_quantize_with_rule(x, dtype, rows, cols, sign_seed, rounding, sr_seed, codes,
+                                scales, rotated, stream, true);
 }
 
 mxfp4_status mxfp4_osc_step(float* w, float* w_snap, float* d_w, float* d_q,

@@ -29,16 +29,18 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
                            int64_t n_groups, void* y, bool bf16_out,
                            cudaStream_t s);
 
+// oas: the overflow-aware scale rule in both passes.
 cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
                                 int64_t cols, uint64_t seed,
                                 uint8_t* row_codes, uint8_t* row_scales,
                                 uint8_t* col_codes, uint8_t* col_scales,
-                                cudaStream_t s);
+                                cudaStream_t s, bool oas = false);
 
 cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
                              int64_t cols, uint64_t sign_seed, bool sr,
                              uint64_t sr_seed, uint8_t* codes,
-                             uint8_t* scales, float* rotated, cudaStream_t s);
+                             uint8_t* scales, float* rotated, cudaStream_t s,
+                             bool oas = false);
 
 cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                             int64_t rows, int64_t cols, bool window_end,

@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(kRowThreads)
 constexpr int kDqThreads = 256;
 constexpr int kDqCols = 128;
 
-template <bool BF16, bool BIG>
+template <bool BF16, bool BIG, bool OAS>
 __global__ void __launch_bounds__(kDqThreads)
     k_double_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
                    RngKey key, uint8_t* __restrict__ row_codes,
@@ -607,7 +607,7 @@ __global__ void __launch_bounds__(kDqThreads)
         amax = max(amax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
       amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      const uint32_t sb = scale_byte(amax);
+      const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
       const float mul = inv_scale(sb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] *= mul;
@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(kDqThreads)
         }
       }
       // cols is a multiple of 32 here, so every pair index is even-aligned
-      store_column_pair(column_pair_codes<true, true, BIG>(
+      store_column_pair(column_pair_codes<true, true, BIG, true, OAS>(
                             [&](int j) { return make_float2(a[j], b[j]); }, ma,
                             mb, r0, tile_c + 2 * cp, cols, key),
                         r0, tile_c + 2 * cp, rows, cols, col_codes, col_scales);
@@ -662,13 +662,14 @@ __global__ void __launch_bounds__(kDqThreads)
 // Row pass of one 1x32 group quarter (8 values of tile row tr, chunk ch):
 // writes the row codes and scale to global memory (when in range) and stages
 // the codes and the scale value 2^e in shared memory for the column pass.
+template <bool OAS>
 __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool ok,
                                              int tr, int ch, uint8_t* __restrict__ rc,
                                              uint8_t* __restrict__ rs, uint32_t* s_codes,
                                              float* s_scales) {
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
   amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-  const uint32_t sb = scale_byte(amax);
+  const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
   const float mul = inv_scale(sb);
 #pragma unroll
   for (int j = 0; j < 8; ++j) v[j] *= mul;
@@ -693,7 +694,7 @@ __device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool 
 // No saturation is needed: every decoded value is G[m] 2^k, two significant
 // bits, and the column scale puts the column maximum in [4, 8), so a scaled
 // value is at most 6 (the only such values in [4, 8) are 4 and 6).
-template <bool BIG>
+template <bool BIG, bool OAS>
 __device__ __forceinline__ ColPair dq_column_pass(
     const uint32_t* s_codes, const float* s_scales, int rg, int cp,
     int64_t tile_r, int64_t tile_c, int64_t cols, RngKey key) {
@@ -725,7 +726,7 @@ __device__ __forceinline__ ColPair dq_column_pass(
     }
   }
   // cols is a multiple of 32 here, so every pair index is even-aligned
-  return column_pair_codes<true, true, BIG, false>(
+  return column_pair_codes<true, true, BIG, false, OAS>(
       [&](int j) { return make_float2(a[j], b[j]); }, __float_as_uint(ma),
       __float_as_uint(mb), r0, tile_c + 2 * cp, cols, key);
 }
@@ -734,7 +735,7 @@ __device__ __forceinline__ ColPair dq_column_pass(
 // staged with asynchronous copies, so the next tile streams in while the
 // current one is quantized along rows and then along columns. Once the row
 // pass is done the current raw tile is free and holds the column stage.
-template <bool BIG>
+template <bool BIG, bool OAS>
 __global__ void __launch_bounds__(kDqThreads, 3)
     k_double_quant_pipe(const void* __restrict__ x, int64_t rows, int64_t cols,
                         RngKey key, uint8_t* __restrict__ row_codes,
@@ -778,15 +779,15 @@ __global__ void __launch_bounds__(kDqThreads, 3)
       const uint4 w = raw[tr * (kDqCols / 8) + ch];
       float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
                     bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-      dq_row_chunk(v, bf16x8_absmax(w), col_ok && tile_r + tr < rows, tr, ch, rc, rs,
-                   s_codes, s_scales);
+      dq_row_chunk<OAS>(v, bf16x8_absmax(w), col_ok && tile_r + tr < rows, tr, ch, rc,
+                        rs, s_codes, s_scales);
     }
     __syncthreads();
     static_assert(ColStage<kDqCols>::kBytes <= kChunks * 16, "stage fits a tile");
     uint4* s_col = smem + buf * kChunks;
     uint8_t* s_sc = reinterpret_cast<uint8_t*>(s_col + ColStage<kDqCols>::kChunks);
     if (tile_r + 32 * rg < rows)
-      stage_column_pair(dq_column_pass<BIG>(s_codes, s_scales, rg, cp, tile_r,
+      stage_column_pair(dq_column_pass<BIG, OAS>(s_codes, s_scales, rg, cp, tile_r,
                                             tile_c, cols, key),
                         cp, rg, s_col, s_sc);
     __syncthreads();
@@ -939,17 +940,16 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint8_t* scales,
 
 namespace mxfp4 {
 
-cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
-                                int64_t cols, uint64_t seed,
-                                uint8_t* row_codes, uint8_t* row_scales,
-                                uint8_t* col_codes, uint8_t* col_scales,
-                                cudaStream_t s) {
-  const RngKey key = make_key(seed, 0);
+template <bool OAS>
+static cudaError_t double_quant_impl(const void* x, bool bf16, int64_t rows,
+                                     int64_t cols, RngKey key, uint8_t* row_codes,
+                                     uint8_t* row_scales, uint8_t* col_codes,
+                                     uint8_t* col_scales, cudaStream_t s) {
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + kDqCols - 1) / kDqCols);
   const bool big = big_tensor(rows, cols);
   if (bf16) {
-    auto kern = big ? k_double_quant_pipe<true> : k_double_quant_pipe<false>;
+    auto kern = big ? k_double_quant_pipe<true, OAS> : k_double_quant_pipe<false, OAS>;
     constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) +
                             kTileRows * (kDqCols / 8) * 4 +
                             kTileRows * (kDqCols / 32) * sizeof(float);
@@ -963,12 +963,24 @@ cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
                                         row_scales, col_codes, col_scales);
     return cudaGetLastError();
   }
-  auto kern = big ? k_double_quant<false, true> : k_double_quant<false, false>;
+  auto kern = big ? k_double_quant<false, true, OAS> : k_double_quant<false, false, OAS>;
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
                                    kDqThreads, 0, n_tiles);
   kern<<<grid, kDqThreads, 0, s>>>(x, rows, cols, key, row_codes, row_scales,
                                    col_codes, col_scales);
   return cudaGetLastError();
+}
+
+cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
+                                int64_t cols, uint64_t seed,
+                                uint8_t* row_codes, uint8_t* row_scales,
+                                uint8_t* col_codes, uint8_t* col_scales,
+                                cudaStream_t s, bool oas) {
+  const RngKey key = make_key(seed, 0);
+  return oas ? double_quant_impl<true>(x, bf16, rows, cols, key, row_codes, row_scales,
+                                       col_codes, col_scales, s)
+             : double_quant_impl<false>(x, bf16, rows, cols, key, row_codes, row_scales,
+                                        col_codes, col_scales, s);
 }
 
 }  // namespace mxfp4

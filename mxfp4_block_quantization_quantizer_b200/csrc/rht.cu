@@ -33,7 +33,7 @@ constexpr int kRhtRowsY = 32;   // rows per CTA step
 // fp32 nearest to 1/sqrt(32).
 constexpr float kInvSqrt32 = 0.17677669529663687f;
 
-template <bool BF16, bool SR, bool ROT>
+template <bool BF16, bool SR, bool ROT, bool OAS>
 __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
     k_rht_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
                 uint32_t sign_key, RngKey key, uint8_t* __restrict__ codes,
@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
       for (int j = 0; j < 32; ++j) zmax = absmax_nan(y[j], zmax);
       amax = __float_as_uint(zmax * kInvSqrt32);
     }
-    const uint32_t sb = scale_byte(amax);
+    const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
     const float mul = ROT ? inv_scale(sb) : inv_scale(sb) * kInvSqrt32;
     // the group's 16 pairs share the high word of their index
     const uint64_t pg = uint64_t(e0 >> 1);
@@ -233,7 +233,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* d) {
 // Quantize the rotated group z (unnormalised) of row r, columns c0 ..
 // c0+31, as k_rht_quant does; the codes and scale go to *oc / *os when
 // STAGED, else to global memory; ROT also writes z / sqrt(32).
-template <bool SR, bool ROT, bool STAGED>
+template <bool SR, bool ROT, bool STAGED, bool OAS>
 __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64_t c0,
                                                       int64_t cols, RngKey key, bool failed,
                                                       uint8_t* __restrict__ codes,
@@ -259,7 +259,7 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
     for (int j = 0; j < 32; j += 2) zmax = absmax3_nan(y[j], y[j + 1], zmax);
     amax = __float_as_uint(zmax * kInvSqrt32);
   }
-  const uint32_t sb = failed ? 0xFFu : scale_byte(amax);
+  const uint32_t sb = failed ? 0xFFu : (OAS ? scale_byte_oas(amax) : scale_byte(amax));
   const float mul = ROT ? inv_scale(sb) : inv_scale(sb) * kInvSqrt32;
   // the group's 16 pairs start at a multiple of 16, so they share the high
   // word of their index (2^32 is a multiple of 16): one inner key
@@ -291,7 +291,7 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
   }
 }
 
-template <bool SR, bool ROT, bool STAGED>
+template <bool SR, bool ROT, bool STAGED, bool OAS>
 __global__ void __launch_bounds__(kRtThreads, 1)
     k_rht_tc(const __grid_constant__ CUtensorMap tm_x, int64_t rows, int64_t cols,
              uint32_t sign_key, RngKey key, uint8_t* __restrict__ codes,
@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
           float y[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(zb[j]);
-          rht_tc_quantize_group<SR, ROT, STAGED>(y, r, c0, cols, key,
+          rht_tc_quantize_group<SR, ROT, STAGED, OAS>(y, r, c0, cols, key,
                                                  !ok || failed_flag(&sm.failed), codes,
                                                  scales, rotated, oc, os);
         }
@@ -514,11 +514,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                  "r"(32 * kRtGroups * kRtAccBufs));
 }
 
-template <bool SR, bool ROT, bool STAGED>
+template <bool SR, bool ROT, bool STAGED, bool OAS>
 cudaError_t rht_tc_impl(const CUtensorMap& mx, int64_t rows, int64_t cols,
                         uint32_t sign_key, RngKey key, uint8_t* codes, uint8_t* scales,
                         float* rotated, cudaStream_t s) {
-  auto kern = k_rht_tc<SR, ROT, STAGED>;
+  auto kern = k_rht_tc<SR, ROT, STAGED, OAS>;
   constexpr size_t smem = sizeof(RhtSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
@@ -529,11 +529,11 @@ cudaError_t rht_tc_impl(const CUtensorMap& mx, int64_t rows, int64_t cols,
   return cudaGetLastError();
 }
 
-template <bool BF16, bool SR, bool ROT>
+template <bool BF16, bool SR, bool ROT, bool OAS>
 cudaError_t rht_impl(const void* x, int64_t rows, int64_t cols,
                      uint32_t sign_key, RngKey key, uint8_t* codes,
                      uint8_t* scales, float* rotated, cudaStream_t s) {
-  auto kern = k_rht_quant<BF16, SR, ROT>;
+  auto kern = k_rht_quant<BF16, SR, ROT, OAS>;
   const int64_t gx = (cols / 32 + kRhtGroupsX - 1) / kRhtGroupsX;
   const int64_t row_blocks = (rows + kRhtRowsY - 1) / kRhtRowsY;
   const int target = persistent_grid(reinterpret_cast<const void*>(kern),
@@ -551,37 +551,47 @@ cudaError_t rht_impl(const void* x, int64_t rows, int64_t cols,
 
 }  // namespace
 
-cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
-                             int64_t cols, uint64_t sign_seed, bool sr,
-                             uint64_t sr_seed, uint8_t* codes,
-                             uint8_t* scales, float* rotated,
-                             cudaStream_t s) {
-  const uint32_t sign_key = stream_key(sign_seed, 1);
-  const RngKey key = make_key(sr_seed, 0);
+template <bool OAS>
+static cudaError_t rht_dispatch(const void* x, bool bf16, int64_t rows, int64_t cols,
+                                uint32_t sign_key, RngKey key, bool sr, uint8_t* codes,
+                                uint8_t* scales, float* rotated, cudaStream_t s) {
   const bool rot = rotated != nullptr;
   if (bf16) {
     // X as a byte array [rows][2 cols] for the TMA: 128-byte boxes
     CUtensorMap mx;
     if (!encode_rows_sw128(&mx, x, rows, 2 * cols, 128)) return cudaErrorInvalidValue;
     if (sr)
-      return rot ? rht_tc_impl<true, true, false>(mx, rows, cols, sign_key, key, codes,
+      return rot ? rht_tc_impl<true, true, false, OAS>(mx, rows, cols, sign_key, key, codes,
+                                                       scales, rotated, s)
+                 : rht_tc_impl<true, false, false, OAS>(mx, rows, cols, sign_key, key, codes,
+                                                        scales, rotated, s);
+    return rot ? rht_tc_impl<false, true, false, OAS>(mx, rows, cols, sign_key, key, codes,
+                                                      scales, rotated, s)
+               : rht_tc_impl<false, false, true, OAS>(mx, rows, cols, sign_key, key, codes,
+                                                      scales, rotated, s);
+  }
+  if (sr)
+    return rot ? rht_impl<false, true, true, OAS>(x, rows, cols, sign_key, key, codes,
                                                   scales, rotated, s)
-                 : rht_tc_impl<true, false, false>(mx, rows, cols, sign_key, key, codes,
+               : rht_impl<false, true, false, OAS>(x, rows, cols, sign_key, key, codes,
                                                    scales, rotated, s);
-    return rot ? rht_tc_impl<false, true, false>(mx, rows, cols, sign_key, key, codes, scales,
+  return rot ? rht_impl<false, false, true, OAS>(x, rows, cols, sign_key, key, codes, scales,
                                                  rotated, s)
-               : rht_tc_impl<false, false, true>(mx, rows, cols, sign_key, key, codes, scales,
-                                                 rotated, s);
-  }
-#define MXFP4_RHT(B, S, R) \
-  return rht_impl<B, S, R>(x, rows, cols, sign_key, key, codes, scales, rotated, s)
-  if (sr) {
-    if (rot) MXFP4_RHT(false, true, true);
-    MXFP4_RHT(false, true, false);
-  }
-  if (rot) MXFP4_RHT(false, false, true);
-  MXFP4_RHT(false, false, false);
-#undef MXFP4_RHT
+             : rht_impl<false, false, false, OAS>(x, rows, cols, sign_key, key, codes, scales,
+                                                  rotated, s);
+}
+
+cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
+                             int64_t cols, uint64_t sign_seed, bool sr,
+                             uint64_t sr_seed, uint8_t* codes,
+                             uint8_t* scales, float* rotated,
+                             cudaStream_t s, bool oas) {
+  const uint32_t sign_key = stream_key(sign_seed, 1);
+  const RngKey key = make_key(sr_seed, 0);
+  return oas ? rht_dispatch<true>(x, bf16, rows, cols, sign_key, key, sr, codes, scales,
+                                  rotated, s)
+             : rht_dispatch<false>(x, bf16, rows, cols, sign_key, key, sr, codes, scales,
+                                   rotated, s);
 }
 
 }  // namespace mxfp4

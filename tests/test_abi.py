@@ -76,6 +76,19 @@ def test_quantize_oas_rejects_bad_arguments():
     assert L.mxfp4_quantize_oas(PODD, 1, 64, 64, 0, 0, 0, P, P, NUL) == ALIGN
 
 
+def test_overflow_aware_double_and_rotation_reject_bad_arguments():
+    L = m.lib()
+    assert L.mxfp4_double_quantize_oas(P, 2, 64, 64, 0, P, P, P, P, NUL) == ENUM
+    assert L.mxfp4_double_quantize_oas(P, 1, 64, 48, 0, P, P, P, P, NUL) == SHAPE
+    assert L.mxfp4_double_quantize_oas(P, 1, 48, 64, 0, P, P, P, P, NUL) == SHAPE
+    assert L.mxfp4_double_quantize_oas(P, 1, 64, 64, 0, P, NUL, P, P, NUL) == NULL
+    assert L.mxfp4_double_quantize_oas(PODD, 1, 64, 64, 0, P, P, P, P, NUL) == ALIGN
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 40, 0, 0, 0, P, P, NUL, NUL) == SHAPE
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 3, 0, P, P, NUL, NUL) == ENUM
+    assert L.mxfp4_rht_quantize_oas(NUL, 1, 64, 64, 0, 0, 0, P, P, NUL, NUL) == NULL
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 0, 0, P, P, PODD, NUL) == ALIGN
+
+
 def test_other_entry_points_reject_bad_arguments():
     L = m.lib()
     assert L.mxfp4_dequantize(P, P, 64, 64, 0, P, 3, NUL) == ENUM
