@@ -531,25 +531,37 @@ def run_ours(args):
                                   "launches": args.steps}
         del qw, qe, qout
 
-        # the overflow-aware scale rule on the sweep (ROWS, RNE)
+        # the overflow-aware scale rule on the sweep: rows RNE, double
+        # quantization, rotation + SR (the step's ops with the other rule)
+        def timed_alone(fn):
+            for _ in range(args.warmup):
+                fn()
+            tev = []
+            for _ in range(args.steps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                tev.append((a, b))
+            torch.cuda.synchronize(dev)
+            return reduce_max(statistics.mean(a.elapsed_time(b) for a, b in tev) * 1e-3,
+                              world, dev)
+
         oout = (u8(R, C // 2), u8(R, C // 32))
-        for _ in range(args.warmup):
-            m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)
-        oev = []
-        for _ in range(args.steps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)
-            b.record(stream)
-            oev.append((a, b))
-        torch.cuda.synchronize(dev)
-        d = statistics.mean(a.elapsed_time(b) for a, b in oev) * 1e-3
-        d = reduce_max(d, world, dev)
-        nbytes = BYTES_PER_ELEM["quant_rows_rne"] * R * C
-        next_ops["quant_rows_rne_oas"] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9,
-                                          "bytes": nbytes, "shape": [R, C],
-                                          "launches": args.steps}
-        del oout
+        dout = (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32))
+        for name, step_op, fn in (
+                ("quant_rows_rne_oas", "quant_rows_rne",
+                 lambda: m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)),
+                ("double_quant_oas", "double_quant",
+                 lambda: m.double_quantize(buf0["x"], SEED, out=dout, oas=True)),
+                ("rht_quant_sr_oas", "rht_quant_sr",
+                 lambda: m.rht_quantize(buf0["x"], 2, m.SR, SEED, out=oout + (None,),
+                                        oas=True))):
+            d = timed_alone(fn)
+            nbytes = BYTES_PER_ELEM[step_op] * R * C
+            next_ops[name] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9, "bytes": nbytes,
+                              "shape": [R, C], "launches": args.steps}
+        del oout, dout
 
         # MXFP4 GEMM on the block-scaled tensor cores, consuming the step's
         # ROWS codes of the sweep as the activation operand
