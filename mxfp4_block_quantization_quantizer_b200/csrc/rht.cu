@@ -33,8 +33,9 @@ constexpr int kRhtRowsY = 32;   // rows per CTA step
 // fp32 nearest to 1/sqrt(32).
 constexpr float kInvSqrt32 = 0.17677669529663687f;
 
-template <bool BF16, bool SR, bool ROT, bool OAS>
-__global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
+// fp32 inputs (bf16 inputs take the tensor-core kernel below).
+template <bool SR, bool ROT, bool OAS>
+__global__ void __launch_bounds__(kRhtThreads, 2)
     k_rht_quant(const void* __restrict__ x, int64_t rows, int64_t cols,
                 uint32_t sign_key, RngKey key, uint8_t* __restrict__ codes,
                 uint8_t* __restrict__ scales, float* __restrict__ rotated) {
@@ -55,35 +56,14 @@ __global__ void __launch_bounds__(kRhtThreads, BF16 ? 4 : 2)
   if (k >= n_cgroups) return;
   const uint32_t neg = sign_bits[kk];
   // XOR masks that flip the sign bit of the elements whose column sign is -1
-  uint32_t flip[BF16 ? 16 : 32];
-  if (BF16) {
+  uint32_t flip[32];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      flip[i] = ((neg >> (2 * i)) & 1u) << 15 | ((neg >> (2 * i + 1)) & 1u) << 31;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) flip[i] = ((neg >> i) & 1u) << 31;
-  }
+  for (int i = 0; i < 32; ++i) flip[i] = ((neg >> i) & 1u) << 31;
   for (int64_t r = int64_t(blockIdx.y) * kRhtRowsY + rr; r < rows;
        r += int64_t(gridDim.y) * kRhtRowsY) {
     const int64_t e0 = r * cols + k * 32;  // first element of the group
     float y[32];
-    if (BF16) {
-      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + e0);
-      uint4 q[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) q[i] = ld_l1(p + i);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t w4[4] = {q[i].x ^ flip[4 * i], q[i].y ^ flip[4 * i + 1],
-                                q[i].z ^ flip[4 * i + 2], q[i].w ^ flip[4 * i + 3]};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          y[8 * i + 2 * j] = bf16_lo(w4[j]);
-          y[8 * i + 2 * j + 1] = bf16_hi(w4[j]);
-        }
-      }
-    } else {
+    {
       const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(x) + e0);
       uint4 q[8];
 #pragma unroll
@@ -529,11 +509,11 @@ cudaError_t rht_tc_impl(const CUtensorMap& mx, int64_t rows, int64_t cols,
   return cudaGetLastError();
 }
 
-template <bool BF16, bool SR, bool ROT, bool OAS>
+template <bool SR, bool ROT, bool OAS>
 cudaError_t rht_impl(const void* x, int64_t rows, int64_t cols,
                      uint32_t sign_key, RngKey key, uint8_t* codes,
                      uint8_t* scales, float* rotated, cudaStream_t s) {
-  auto kern = k_rht_quant<BF16, SR, ROT, OAS>;
+  auto kern = k_rht_quant<SR, ROT, OAS>;
   const int64_t gx = (cols / 32 + kRhtGroupsX - 1) / kRhtGroupsX;
   const int64_t row_blocks = (rows + kRhtRowsY - 1) / kRhtRowsY;
   const int target = persistent_grid(reinterpret_cast<const void*>(kern),
@@ -571,13 +551,13 @@ static cudaError_t rht_dispatch(const void* x, bool bf16, int64_t rows, int64_t 
                                                       scales, rotated, s);
   }
   if (sr)
-    return rot ? rht_impl<false, true, true, OAS>(x, rows, cols, sign_key, key, codes,
+    return rot ? rht_impl<true, true, OAS>(x, rows, cols, sign_key, key, codes,
                                                   scales, rotated, s)
-               : rht_impl<false, true, false, OAS>(x, rows, cols, sign_key, key, codes,
+               : rht_impl<true, false, OAS>(x, rows, cols, sign_key, key, codes,
                                                    scales, rotated, s);
-  return rot ? rht_impl<false, false, true, OAS>(x, rows, cols, sign_key, key, codes, scales,
+  return rot ? rht_impl<false, true, OAS>(x, rows, cols, sign_key, key, codes, scales,
                                                  rotated, s)
-             : rht_impl<false, false, false, OAS>(x, rows, cols, sign_key, key, codes, scales,
+             : rht_impl<false, false, OAS>(x, rows, cols, sign_key, key, codes, scales,
                                                   rotated, s);
 }
 
