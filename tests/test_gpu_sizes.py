@@ -51,6 +51,25 @@ def test_llm_weight_rht_sr_sampled_rows():
     assert n_near <= 20  # boundary cases are rare
 
 
+@pytest.mark.parametrize("rnd", [O.RNE, O.SR])
+def test_llm_weight_rht_without_rotated_output(rnd):
+    """The benchmark's form (no rotated output; nearest rounding stages its
+    codes for whole-row stores): on the 4096x14336 weight every CTA runs
+    several tiles across column blocks; the codes and scales equal those of
+    the call that also writes the rotated values, which are checked against
+    the oracle on sampled rows."""
+    x = W.llm_w(seed=2)
+    xd = to_dev(x)
+    codes, scales, rot = m.rht_quantize(xd, 2, rnd, 2, want_rotated=True)
+    c2, s2, none = m.rht_quantize(xd, 2, rnd, 2)
+    assert none is None
+    assert torch.equal(c2, codes) and torch.equal(s2, scales)
+    codes, scales, rot = to_np(codes), to_np(scales), to_np(rot)
+    for r in (0, 127, 128, 2048, 4095):
+        check_rht(x[r:r + 1], 2, rnd, 2, codes[r:r + 1], scales[r:r + 1],
+                  rot[r:r + 1], row0=r)
+
+
 def test_osc_weight_200_steps_sampled_bands():
     w_np = W.osc_w(seed=3)  # 4096 x 4096
     w = to_dev(w_np)
