@@ -360,7 +360,16 @@ __device__ __forceinline__ void load_tile(const void* __restrict__ x,
 // Stage one [128 x kCols] tile of a tensor whose rows are 16-byte aligned
 // and whose cols are a whole number of 16-byte chunks, with asynchronous
 // copies (zero-filled outside the tensor), and commit them as one group.
-template <bool BF16>
+// Tiles wholly inside the tensor skip the per-chunk range checks.
+// SWZ (bf16 only): chunk ch of tile row r lands in slot
+// ch ^ dq_swizzle(ch >> 2, r) of that row, so that the double quantizer's
+// row pass, where four consecutive threads read the four 64-byte groups of
+// a row chunk by chunk, hits 32 distinct banks per 8-thread phase.
+__device__ __forceinline__ int dq_swizzle(int group, int row) {
+  return (group & 2) | (row & 1);
+}
+
+template <bool BF16, bool SWZ = false>
 __device__ __forceinline__ void stage_tile_async(const void* __restrict__ x,
                                                  int64_t rows, int64_t cols,
                                                  int64_t tile_r, int64_t tile_c,
@@ -375,10 +384,17 @@ __device__ __forceinline__ void stage_tile_async(const void* __restrict__ x,
   const bool col_ok = gc < cols;
   const char* src = static_cast<const char*>(x) + ((tile_r + r0) * cols + gc) * T::kElemBytes;
   const int64_t step = int64_t(kRowStep) * cols * T::kElemBytes;
+  static_assert(!SWZ || (BF16 && kRowStep % 2 == 0), "swizzle: bf16 tiles, even row step");
+  uint4* dst = tile + r0 * T::kChunksPerRow + (SWZ ? ch ^ dq_swizzle(ch >> 2, r0) : ch);
+  if (tile_r + kTileRows <= rows && tile_c + T::kCols <= cols) {
 #pragma unroll
-  for (int k = 0; k < kPer; ++k, src += step) {
-    const bool ok = col_ok && tile_r + r0 + k * kRowStep < rows;
-    cp_async16(tile + k * T::kThreads + threadIdx.x, ok ? src : x, ok);
+    for (int k = 0; k < kPer; ++k, src += step) cp_async16(dst + k * T::kThreads, src, true);
+  } else {
+#pragma unroll
+    for (int k = 0; k < kPer; ++k, src += step) {
+      const bool ok = col_ok && tile_r + r0 + k * kRowStep < rows;
+      cp_async16(dst + k * T::kThreads, ok ? src : x, ok);
+    }
   }
   cp_async_commit();
 }
@@ -659,28 +675,51 @@ __global__ void __launch_bounds__(kDqThreads)
   }
 }
 
-// Row pass of one 1x32 group quarter (8 values of tile row tr, chunk ch):
-// writes the row codes and scale to global memory (when in range) and stages
-// the codes and the scale value 2^e in shared memory for the column pass.
+// Row pass of one whole 1x32 group: group g of the staged raw tile row
+// `row` (tile row tr; chunks swizzled as the staging placed them). Writes
+// the 32 row codes and the scale byte to global memory (when in range) and
+// stages the codes and the scale value 2^e in shared memory for the column
+// pass.
 template <bool OAS>
-__device__ __forceinline__ void dq_row_chunk(float (&v)[8], uint32_t amax, bool ok,
-                                             int tr, int ch, uint8_t* __restrict__ rc,
-                                             uint8_t* __restrict__ rs, uint32_t* s_codes,
-                                             float* s_scales) {
-  amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-  amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+__device__ __forceinline__ void dq_row_group(const uint4* row, int g, int tr, bool ok,
+                                             uint8_t* __restrict__ rc,
+                                             uint8_t* __restrict__ rs, uint4* s_code,
+                                             float* s_scale) {
+  uint32_t w[16];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 q = row[4 * g + (c ^ dq_swizzle(g, tr))];
+    w[4 * c] = q.x, w[4 * c + 1] = q.y, w[4 * c + 2] = q.z, w[4 * c + 3] = q.w;
+  }
+  uint32_t m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = bf16x2_absmax_nan(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+  for (int n = 4; n >= 1; n /= 2)
+#pragma unroll
+    for (int i = 0; i < n; ++i) m[i] = bf16x2_absmax_nan(m[i], m[i + n]);
+  const uint32_t mm = m[0] & 0x7FFF7FFFu;
+  const uint32_t amax = max(mm << 16, mm & 0xFFFF0000u);
   const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
   const float mul = inv_scale(sb);
+  uint32_t word[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] *= mul;
-  uint32_t word = e2m1x8_rn(v);
-  if (sb == 0xFFu) word = 0;
-  if (ok) {
-    *reinterpret_cast<uint32_t*>(rc) = word;
-    if ((ch & 3) == 0) *rs = uint8_t(sb);
+  for (int c = 0; c < 4; ++c) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = bf16_lo(w[4 * c + j]) * mul;
+      v[2 * j + 1] = bf16_hi(w[4 * c + j]) * mul;
+    }
+    word[c] = sb == 0xFFu ? 0u : e2m1x8_rn(v);
   }
-  s_codes[tr * (kDqCols / 8) + ch] = word;
-  if ((ch & 3) == 0) s_scales[tr * (kDqCols / 32) + ch / 4] = scale_value(sb);
+  const uint4 out = make_uint4(word[0], word[1], word[2], word[3]);
+  if (ok) {
+    *reinterpret_cast<uint4*>(rc) = out;
+    *rs = uint8_t(sb);
+  }
+  *s_code = out;
+  *s_scale = scale_value(sb);
 }
 
 // Column pass of the double quantizer over the staged Q_D(X) codes: decode
@@ -748,39 +787,36 @@ __global__ void __launch_bounds__(kDqThreads, 3)
   float* s_scales = reinterpret_cast<float*>(s_codes + kTileRows * (kDqCols / 8));
   const int64_t tiles_c = (cols + kDqCols - 1) / kDqCols;
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
-  const int ch = threadIdx.x & 15, rr = threadIdx.x >> 4;
-  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  const int g = threadIdx.x & 3, tr = threadIdx.x >> 2;  // row pass
+  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;  // column pass
   int64_t t = blockIdx.x;
   if (t >= n_tiles) return;
   TileWalk cur(t, gridDim.x, tiles_c), nxt = cur;
   nxt.next();
-  stage_tile_async<true>(x, rows, cols, cur.r * kTileRows, cur.c * kDqCols, smem);
+  stage_tile_async<true, true>(x, rows, cols, cur.r * kTileRows, cur.c * kDqCols, smem);
   for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
     const int64_t tn = t + gridDim.x;
     if (tn < n_tiles)
-      stage_tile_async<true>(x, rows, cols, nxt.r * kTileRows, nxt.c * kDqCols,
-                             smem + (buf ^ 1) * kChunks);
+      stage_tile_async<true, true>(x, rows, cols, nxt.r * kTileRows, nxt.c * kDqCols,
+                                   smem + (buf ^ 1) * kChunks);
     else
       cp_async_commit();
     cp_async_wait<1>();
     __syncthreads();
     const int64_t tile_r = cur.r * kTileRows;
     const int64_t tile_c = cur.c * kDqCols;
-    const int64_t gc = tile_c + 8 * ch;
     const uint4* raw = smem + buf * kChunks;
-    // this thread's row outputs: rows tile_r + rr + 16k, columns gc .. gc+7
-    uint8_t* rc = row_codes + (tile_r + rr) * (cols / 2) + gc / 2;
-    uint8_t* rs = row_scales + (tile_r + rr) * (cols / 32) + gc / 32;
-    const int64_t rc_step = 16 * (cols / 2), rs_step = 16 * (cols / 32);
-    const bool col_ok = gc < cols;
-#pragma unroll 2
-    for (int k = 0; k < kTileRows / 16; ++k, rc += rc_step, rs += rs_step) {
-      const int tr = rr + 16 * k;
-      const uint4 w = raw[tr * (kDqCols / 8) + ch];
-      float v[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                    bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-      dq_row_chunk<OAS>(v, bf16x8_absmax(w), col_ok && tile_r + tr < rows, tr, ch, rc,
-                        rs, s_codes, s_scales);
+    // this thread's row outputs: group g of tile rows tr and tr + 64
+    uint8_t* rc = row_codes + (tile_r + tr) * (cols / 2) + (tile_c + 32 * g) / 2;
+    uint8_t* rs = row_scales + (tile_r + tr) * (cols / 32) + (tile_c + 32 * g) / 32;
+    const bool g_ok = tile_c + 32 * g < cols;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int r = tr + 64 * k;
+      dq_row_group<OAS>(raw + r * (kDqCols / 8), g, r, g_ok && tile_r + r < rows,
+                        rc + k * 64 * (cols / 2), rs + k * 64 * (cols / 32),
+                        reinterpret_cast<uint4*>(s_codes) + r * (kDqCols / 32) + g,
+                        s_scales + r * (kDqCols / 32) + g);
     }
     __syncthreads();
     static_assert(ColStage<kDqCols>::kBytes <= kChunks * 16, "stage fits a tile");
