@@ -470,14 +470,13 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
   nxt.next();
   stage_tile_async<BF16>(x, rows, cols, cur.r * kTileRows, cur.c * T::kCols, smem);
   for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
-    const int64_t tn = t + gridDim.x;
-    if (tn < n_tiles)
+    // this tile's copies are done and visible, and every thread has left the
+    // previous tile (whose buffer and column stage are reused below)
+    cp_async_wait<0>();
+    __syncthreads();
+    if (t + gridDim.x < n_tiles)
       stage_tile_async<BF16>(x, rows, cols, nxt.r * kTileRows, nxt.c * T::kCols,
                              smem + (buf ^ 1) * kChunks);
-    else
-      cp_async_commit();  // keep one group per iteration
-    cp_async_wait<1>();   // this tile's copies (the older group) are done
-    __syncthreads();
     const int64_t tile_r = cur.r * kTileRows;
     const int64_t tile_c = cur.c * T::kCols;
     if (tile_r + 32 * rg < rows)
@@ -488,9 +487,7 @@ __global__ void __launch_bounds__(ColTile<BF16>::kThreads, 3)
     __syncthreads();
     store_staged_columns<T::kCols, T::kThreads>(s_col, s_sc, tile_r, tile_c,
                                                 rows, cols, codes, scales);
-    __syncthreads();  // the next copies and stage writes reuse the buffers
   }
-  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -562,6 +559,11 @@ __global__ void __launch_bounds__(kRowThreads)
 
 constexpr int kDqThreads = 256;
 constexpr int kDqCols = 128;
+// Staged row-group scale values of the pipelined double quantizer, group
+// major: value (row r, group g) at g * kDqScaleStride + r. The column pass
+// reads four consecutive rows in one 16-byte load; the padding (8 words)
+// spreads the row pass's stores (8 rows x 4 groups per warp) over 32 banks.
+constexpr int kDqScaleStride = kTileRows + 8;
 
 template <bool BF16, bool BIG, bool OAS>
 __global__ void __launch_bounds__(kDqThreads)
@@ -744,12 +746,13 @@ __device__ __forceinline__ ColPair dq_column_pass(
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     uint32_t w4 = 0;
-    float sv[4];
+    const float4 sv4 = *reinterpret_cast<const float4*>(
+        s_scales + (cp / 16) * kDqScaleStride + 32 * rg + 4 * q);
+    const float sv[4] = {sv4.x, sv4.y, sv4.z, sv4.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = 32 * rg + 4 * q + i;
       w4 |= uint32_t(sc[r * (kDqCols / 2) + cp]) << (8 * i);
-      sv[i] = s_scales[r * (kDqCols / 32) + cp / 16];
     }
     float f[8];
     e2m1x8_decode(w4, f);
@@ -795,14 +798,13 @@ __global__ void __launch_bounds__(kDqThreads, 3)
   nxt.next();
   stage_tile_async<true, true>(x, rows, cols, cur.r * kTileRows, cur.c * kDqCols, smem);
   for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
-    const int64_t tn = t + gridDim.x;
-    if (tn < n_tiles)
+    // this tile's copies are done and visible, and every thread has left the
+    // previous tile (whose buffer the next copies overwrite)
+    cp_async_wait<0>();
+    __syncthreads();
+    if (t + gridDim.x < n_tiles)
       stage_tile_async<true, true>(x, rows, cols, nxt.r * kTileRows, nxt.c * kDqCols,
                                    smem + (buf ^ 1) * kChunks);
-    else
-      cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
     const int64_t tile_r = cur.r * kTileRows;
     const int64_t tile_c = cur.c * kDqCols;
     const uint4* raw = smem + buf * kChunks;
@@ -816,7 +818,7 @@ __global__ void __launch_bounds__(kDqThreads, 3)
       dq_row_group<OAS>(raw + r * (kDqCols / 8), g, r, g_ok && tile_r + r < rows,
                         rc + k * 64 * (cols / 2), rs + k * 64 * (cols / 32),
                         reinterpret_cast<uint4*>(s_codes) + r * (kDqCols / 32) + g,
-                        s_scales + r * (kDqCols / 32) + g);
+                        s_scales + g * kDqScaleStride + r);
     }
     __syncthreads();
     static_assert(ColStage<kDqCols>::kBytes <= kChunks * 16, "stage fits a tile");
@@ -829,9 +831,7 @@ __global__ void __launch_bounds__(kDqThreads, 3)
     __syncthreads();
     store_staged_columns<kDqCols, kDqThreads>(s_col, s_sc, tile_r, tile_c,
                                               rows, cols, col_codes, col_scales);
-    __syncthreads();  // the next copies overwrite this buffer
   }
-  cp_async_wait<0>();
 }
 
 }  // namespace
@@ -988,7 +988,7 @@ static cudaError_t double_quant_impl(const void* x, bool bf16, int64_t rows,
     auto kern = big ? k_double_quant_pipe<true, OAS> : k_double_quant_pipe<false, OAS>;
     constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) +
                             kTileRows * (kDqCols / 8) * 4 +
-                            kTileRows * (kDqCols / 32) * sizeof(float);
+                            (kDqCols / 32) * kDqScaleStride * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(
         reinterpret_cast<const void*>(kern),
         cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
