@@ -119,6 +119,35 @@ __device__ __forceinline__ float inv_scale(uint32_t sb) {
   return __uint_as_float((254u - b) << 23);
 }
 
+// The double quantizer carries its decoded row groups at half their size,
+// G[m] 2^(e-1), so that the largest, 6 2^126 under the overflow-aware rule,
+// stays finite (exact: at least 0.5 2^-128). half_scale_value(sb) = 2^(e-1)
+// (sb 0 and 1: the subnormals 2^-128, 2^-127; sb 0xFF: +inf), and the
+// column scale bytes of such halved values: scale_byte / scale_byte_oas of
+// twice the maximum, from the fp32 bit pattern of the halved maximum (one
+// exponent step down; below 2^-125 the OCP byte is 0 either way).
+__device__ __forceinline__ float half_scale_value(uint32_t sb) {
+  return __uint_as_float(sb == 0xFFu ? 0x7F800000u
+                                     : (sb >= 2u ? (sb - 1u) << 23 : 0x00200000u << sb));
+}
+__device__ __forceinline__ uint32_t scale_byte_of_double(uint32_t half_bits) {
+  const uint32_t E = half_bits >> 23;
+  return half_bits >= 0x7F800000u ? 0xFFu : (E > 1u ? E - 1u : 0u);
+}
+__device__ __forceinline__ uint32_t scale_byte_oas_of_double(uint32_t half_bits) {
+  const bool up = half_bits >= (1u << 23) && half_bits < 0x7F800000u &&
+                  (half_bits & 0x7FFFFFu) > 0x400000u;
+  return scale_byte_of_double(half_bits) + (up ? 1u : 0u);
+}
+
+// 2^(e-1) and 6 2^e as fp32 for byte sb = e + 127 in [2, 252].
+__device__ __forceinline__ float scale_half(uint32_t sb) {
+  return __uint_as_float((sb - 1u) << 23);
+}
+__device__ __forceinline__ float scale_six(uint32_t sb) {
+  return __uint_as_float(((sb + 2u) << 23) | 0x400000u);
+}
+
 // 2^e as fp32 for byte sb (sb = 0 gives the subnormal 2^-127, whose pattern
 // 0x00400000 lies below every normal one; sb = 0xFF gives +inf).
 __device__ __forceinline__ float scale_value(uint32_t sb) {
@@ -179,6 +208,21 @@ __device__ __forceinline__ void sr_noise64_pair(uint32_t g, uint32_t& n_even,
   n_odd = sr_noise64(hi);
 }
 
+// The same noise for a value left unscaled by 2^-e, e = sb - 127, and its
+// pair form: with y the rounding operand of v 2^-e (normal) and y' = 2^e y
+// that of v (normal when e >= -125), bits(y) = bits(y') - e 2^23, so
+// 64 bits(y) + sr_noise64(r) = 64 bits(y') + (r * 0xFFFFF000 + base).
+__device__ __forceinline__ uint32_t sr_noise64_base(uint32_t sb) {
+  return 0x4FFFF7C0u - ((sb - 127u) << 29);
+}
+__device__ __forceinline__ void sr_noise64_pair_based(uint32_t g, uint32_t base_even,
+                                                      uint32_t base_odd, uint32_t& n_even,
+                                                      uint32_t& n_odd) {
+  const uint32_t hi = g >> 16;
+  n_even = ((g ^ hi) & 0xFFFFu) * 0xFFFFF000u + base_even;
+  n_odd = hi * 0xFFFFF000u + base_odd;
+}
+
 // The stochastic code of v in bits 28..31 (sign in bit 31; the bits below
 // are not part of it). SAT = false leaves out the saturation, for callers
 // whose |v| never exceeds 6.
@@ -189,6 +233,23 @@ __device__ __forceinline__ uint32_t e2m1_sr_top(float v, uint32_t noise64) {
   if (SAT) y = fminf(y, 6.0f);  // |v| >= 6 saturates to 6
   return (__float_as_uint(y) * 64u + noise64) |
          (__float_as_uint(v) & 0x80000000u);
+}
+
+// e2m1_sr_top of v 2^-e computed on the unscaled v, for scale bytes
+// sb = e + 127 in [2, 252]: half = 2^(e-1), sat = 6 2^e (scale_half,
+// scale_six), noise from sr_noise64_pair_based with base
+// sr_noise64_base(sb). Every step is the unscaled one times 2^e, and each
+// result is normal (y' >= 2^(e-1) >= 2^-126), so the rounding up and the
+// comparisons are those of the scaled value; a value whose scaled form
+// would underflow is below 2^-126 and gives the same code (the carry needs
+// a scaled value of at least 33 2^-23).
+template <bool SAT>
+__device__ __forceinline__ uint32_t e2m1_sr_top_scaled(float v, float half, float sat,
+                                                      uint32_t noise) {
+  const float a = fabsf(v);
+  float y = fmaxf(a, __fmaf_ru(a, 0.5f, half));
+  if (SAT) y = fminf(y, sat);
+  return (__float_as_uint(y) * 64u + noise) | (__float_as_uint(v) & 0x80000000u);
 }
 
 // Shift a packed code word up by one nibble and append the code held in the

@@ -160,30 +160,75 @@ struct ColPair {
   uint32_t sa, sb;
 };
 
+// The multiplier that scales a value v held at half its size (HALF) by
+// 2^-e, e = sb - 127, in one or two exact steps: 2^(1-e) for sb >= 1, and
+// 2 then 2^127 for sb = 0 (where 2^128 is not an fp32 value).
+struct HalfScale {
+  float m1, m2;
+  __device__ __forceinline__ explicit HalfScale(uint32_t sb) {
+    m1 = sb == 0u ? 2.0f : 1.0f;
+    m2 = __uint_as_float((sb == 0u ? 254u : 255u - min(sb, 254u)) << 23);
+  }
+  __device__ __forceinline__ float operator()(float v) const { return (v * m1) * m2; }
+};
+
 // Quantize the two adjacent columns c0, c0+1 over the 32 rows r0 .. r0+31.
 // get(j) returns the values of row r0+j (x: column c0, y: column c0+1); ma
 // and mb are the fp32 bit patterns of the two columns' absolute maxima.
+// HALF: get() returns every value at half its size (see half_scale_value),
+// and ma, mb are the halved maxima.
 template <bool SR, bool EVEN, bool BIG, bool SAT = true, bool OAS = false,
-          typename Get>
+          bool HALF = false, typename Get>
 __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
                                                      uint32_t mb, int64_t r0,
                                                      int64_t c0, int64_t cols,
                                                      RngKey key) {
   ColPair o;
-  o.sa = OAS ? scale_byte_oas(ma) : scale_byte(ma);
-  o.sb = OAS ? scale_byte_oas(mb) : scale_byte(mb);
+  if (HALF) {
+    o.sa = OAS ? scale_byte_oas_of_double(ma) : scale_byte_of_double(ma);
+    o.sb = OAS ? scale_byte_oas_of_double(mb) : scale_byte_of_double(mb);
+  } else {
+    o.sa = OAS ? scale_byte_oas(ma) : scale_byte(ma);
+    o.sb = OAS ? scale_byte_oas(mb) : scale_byte(mb);
+  }
   const float mula = inv_scale(o.sa), mulb = inv_scale(o.sb);
+  const HalfScale hsa(o.sa), hsb(o.sb);
+  auto scale_a = [&](float v) { return HALF ? hsa(v) : v * mula; };
+  auto scale_b = [&](float v) { return HALF ? hsb(v) : v * mulb; };
+  // the scale byte of the values as get() returns them
+  constexpr uint32_t kHeld = HALF ? 1u : 0u;
 #pragma unroll
   for (int q = 0; q < 4; ++q) o.wa[q] = o.wb[q] = 0;
-  if (SR) {
+  if (SR && EVEN && !BIG && o.sa >= 2u + kHeld && o.sb >= 2u + kHeld && o.sa != 0xFFu &&
+      o.sb != 0xFFu) {
+    // Scales of at least 2^-125 (for the values as held): the power of two
+    // rides on the rounding (e2m1_sr_top_scaled) instead of a multiply per
+    // element. Overflow-aware scales never leave a value above 6, so they
+    // skip the saturation.
+    constexpr bool kSat = SAT && !OAS;
+    const uint32_t ua = o.sa - kHeld, ub = o.sb - kHeld;
+    const float ha = scale_half(ua), hb = scale_half(ub);
+    const float xa = kSat ? scale_six(ua) : 0.0f, xb = kSat ? scale_six(ub) : 0.0f;
+    const uint32_t ka = sr_noise64_base(ua), kb = sr_noise64_base(ub);
+    const uint32_t p0 = key.k0 + uint32_t((uint64_t(r0) * uint64_t(cols) + uint64_t(c0)) >> 1);
+    const uint32_t hc = uint32_t(uint64_t(cols) >> 1);
+#pragma unroll
+    for (int j = 31; j >= 0; --j) {  // push_code fills nibbles 7 .. 0
+      uint32_t na, nb;
+      sr_noise64_pair_based(mix32_pre(p0 + uint32_t(j) * hc), ka, kb, na, nb);
+      const float2 v = get(j);
+      o.wa[j >> 3] = push_code(o.wa[j >> 3], e2m1_sr_top_scaled<kSat>(v.x, ha, xa, na));
+      o.wb[j >> 3] = push_code(o.wb[j >> 3], e2m1_sr_top_scaled<kSat>(v.y, hb, xb, nb));
+    }
+  } else if (SR) {
     const uint64_t i0 = uint64_t(r0) * uint64_t(cols) + uint64_t(c0);
 #pragma unroll
     for (int j = 31; j >= 0; --j) {  // push_code fills nibbles 7 .. 0
       uint32_t na, nb;
       column_noise<EVEN, BIG>(key, i0, cols, j, na, nb);
       const float2 v = get(j);
-      o.wa[j >> 3] = push_code(o.wa[j >> 3], e2m1_sr_top<SAT>(v.x * mula, na));
-      o.wb[j >> 3] = push_code(o.wb[j >> 3], e2m1_sr_top<SAT>(v.y * mulb, nb));
+      o.wa[j >> 3] = push_code(o.wa[j >> 3], e2m1_sr_top<SAT>(scale_a(v.x), na));
+      o.wb[j >> 3] = push_code(o.wb[j >> 3], e2m1_sr_top<SAT>(scale_b(v.y), nb));
     }
   } else {
 #pragma unroll
@@ -192,8 +237,8 @@ __device__ __forceinline__ ColPair column_pair_codes(Get get, uint32_t ma,
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float2 v = get(8 * q + j);
-        va[j] = v.x * mula;
-        vb[j] = v.y * mulb;
+        va[j] = scale_a(v.x);
+        vb[j] = scale_b(v.y);
       }
       o.wa[q] = e2m1x8_rn(va);
       o.wb[q] = e2m1x8_rn(vb);
@@ -639,9 +684,9 @@ __global__ void __launch_bounds__(kDqThreads)
       if ((ch & 3) == 0) s_scales[(rr + 16 * k) * (kDqCols / 32) + ch / 4] = uint8_t(sb);
     }
     __syncthreads();
-    // Column pass: decode Q_D(X) for columns 2cp, 2cp+1 over 32 rows (one
-    // shared byte per row holds both codes), then stochastic rounding along
-    // the 32x1 groups. A row group of scale 0xFF decodes to NaN (0 x inf).
+    // Column pass: decode Q_D(X) / 2 for columns 2cp, 2cp+1 over 32 rows
+    // (one shared byte per row holds both codes), then stochastic rounding
+    // along the 32x1 groups. A row group of scale 0xFF decodes to NaN (0 x inf).
     const int64_t r0 = tile_r + 32 * rg;
     if (r0 < rows) {
       const uint8_t* sc = reinterpret_cast<const uint8_t*>(s_codes);
@@ -655,7 +700,7 @@ __global__ void __launch_bounds__(kDqThreads)
         for (int i = 0; i < 4; ++i) {
           const int r = 32 * rg + 4 * q + i;
           w4 |= uint32_t(sc[r * (kDqCols / 2) + cp]) << (8 * i);
-          sv[i] = scale_value(s_scales[r * (kDqCols / 32) + cp / 16]);
+          sv[i] = half_scale_value(s_scales[r * (kDqCols / 32) + cp / 16]);
         }
         float f[8];
         e2m1x8_decode(w4, f);
@@ -668,7 +713,7 @@ __global__ void __launch_bounds__(kDqThreads)
         }
       }
       // cols is a multiple of 32 here, so every pair index is even-aligned
-      store_column_pair(column_pair_codes<true, true, BIG, true, OAS>(
+      store_column_pair(column_pair_codes<true, true, BIG, true, OAS, true>(
                             [&](int j) { return make_float2(a[j], b[j]); }, ma,
                             mb, r0, tile_c + 2 * cp, cols, key),
                         r0, tile_c + 2 * cp, rows, cols, col_codes, col_scales);
@@ -680,8 +725,8 @@ __global__ void __launch_bounds__(kDqThreads)
 // Row pass of one whole 1x32 group: group g of the staged raw tile row
 // `row` (tile row tr; chunks swizzled as the staging placed them). Writes
 // the 32 row codes and the scale byte to global memory (when in range) and
-// stages the codes and the scale value 2^e in shared memory for the column
-// pass.
+// stages the codes and the halved scale value 2^(e-1) (half_scale_value) in
+// shared memory for the column pass.
 template <bool OAS>
 __device__ __forceinline__ void dq_row_group(const uint4* row, int g, int tr, bool ok,
                                              uint8_t* __restrict__ rc,
@@ -721,16 +766,17 @@ __device__ __forceinline__ void dq_row_group(const uint4* row, int g, int tr, bo
     *rs = uint8_t(sb);
   }
   *s_code = out;
-  *s_scale = scale_value(sb);
+  *s_scale = half_scale_value(sb);
 }
 
 // Column pass of the double quantizer over the staged Q_D(X) codes: decode
 // columns 2cp, 2cp+1 of rows 32rg.. (one shared byte per row holds both
-// codes) and multiply by the row groups' staged scale values (a row group of
-// scale 0xFF has the value +inf and codes 0, so it decodes to NaN, and the
-// NaN-propagating maximum carries it into the column scale), then
-// stochastic rounding along the 32x1 groups. The caller checks that the row
-// group lies inside the tensor.
+// codes) and multiply by the row groups' staged halved scale values, which
+// gives Q_D(X) / 2 exactly (a row group of scale 0xFF has the value +inf and
+// codes 0, so it decodes to NaN, and the NaN-propagating maximum carries it
+// into the column scale), then stochastic rounding along the 32x1 groups
+// (column_pair_codes with HALF). The caller checks that the row group lies
+// inside the tensor.
 //
 // No saturation is needed: every decoded value is G[m] 2^k, two significant
 // bits, and the column scale puts the column maximum in [4, 8), so a scaled
@@ -768,7 +814,7 @@ __device__ __forceinline__ ColPair dq_column_pass(
     }
   }
   // cols is a multiple of 32 here, so every pair index is even-aligned
-  return column_pair_codes<true, true, BIG, false, OAS>(
+  return column_pair_codes<true, true, BIG, false, OAS, true>(
       [&](int j) { return make_float2(a[j], b[j]); }, __float_as_uint(ma),
       __float_as_uint(mb), r0, tile_c + 2 * cp, cols, key);
 }

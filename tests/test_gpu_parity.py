@@ -155,6 +155,62 @@ def test_edge_groups(dtype, rnd):
 
 
 # ---------------------------------------------------------------------------
+# Column stochastic rounding at extreme scales: scale bytes 2 .. 252 round
+# the unscaled value (the power of two folded into the rounding), bytes 0
+# and 1 scale first; both must give the oracle's codes.
+# ---------------------------------------------------------------------------
+
+EXTREME_PEAKS = [(1.5 * 2.0 ** -124, 1), (1.5 * 2.0 ** -123, 2), (1.5 * 2.0 ** -122, 3),
+                 (1.5 * 2.0 ** -121, 4), (7.875 * 2.0 ** 125, 252)]
+
+
+def extreme_scale_columns(dtype, seed, rows=128, per_band=64):
+    """rows x (5 * per_band): one band of columns per peak of EXTREME_PEAKS,
+    each 32x1 group uniform in [-peak, peak] with its peak present, plus
+    subnormal, tiny and signed-zero entries."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    bands = []
+    for peak, _ in EXTREME_PEAKS:
+        b = g.uniform(-1.0, 1.0, (rows, per_band)) * peak
+        b[g.integers(0, 32, per_band) + 32 * g.integers(0, rows // 32, per_band),
+          np.arange(per_band)] = peak * np.where(np.arange(per_band) % 2, 1.0, -1.0)
+        tiny = [2.0 ** -133, -2.0 ** -140, 2.0 ** -126, -0.0, 0.0] + (
+            [2.0 ** -149, -2.0 ** -145] if dtype == "f32" else [])
+        for k, t in enumerate(tiny):
+            b[(7 * k + 3) % rows, (5 * k + 1) % per_band :: 3] = t
+        bands.append(b)
+    x = np.concatenate(bands, axis=1).astype(np.float32)
+    # the band peaks survive the rounding to bf16 (all are bf16 values)
+    return x.astype(BF16) if dtype == "bf16" else x
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("oas", [False, True])
+def test_column_sr_extreme_scales(dtype, oas):
+    x = extreme_scale_columns(dtype, 11)
+    c, s = m.quantize(to_dev(x), m.COLS, m.SR, 6, oas=oas)
+    oc, os_ = O.quantize(x, O.COLS, O.SR, 6, oas=oas)
+    if not oas:  # every band sits at its intended scale byte
+        for i, (_, sb) in enumerate(EXTREME_PEAKS):
+            assert (os_[64 * i:64 * (i + 1)] == sb).all()
+    assert_bits_equal(to_np(c), oc, "extreme-scale column codes")
+    assert_bits_equal(to_np(s), os_, "extreme-scale column scales")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("oas", [False, True])
+def test_double_quant_extreme_scales(oas, dtype):
+    # overflow-aware row scales reach 2^126 here, where Q_D(X) holds 4 2^126
+    # and 6 2^126: above the largest fp32 value, exact in the oracle
+    x = extreme_scale_columns(dtype, 12)
+    got = m.double_quantize(to_dev(x), seed=7, oas=oas)
+    want = O.double_quantize(x, 7, oas=oas)
+    assert set(np.unique(want[3])) >= {1, 2, 3}
+    for g_, w, name in zip(got, want, ("row codes", "row scales", "col codes", "col scales")):
+        assert_bits_equal(to_np(g_), w, "extreme-scale double quant " + name)
+
+
+# ---------------------------------------------------------------------------
 # Dequantize
 # ---------------------------------------------------------------------------
 
