@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     int64_t cb = t_begin / n_rt, rt = t_begin % n_rt;
     for (int64_t t = t_begin; t < t_end; ++t, rt = rt + 1 == n_rt ? 0 : rt + 1,
                  cb += rt == 0 ? 1 : 0) {
-      if (!wait_parity(&sm.empty[s], ph ^ 1u)) {
+      if (!wait_parity_sleep(&sm.empty[s], ph ^ 1u)) {  // runs ahead of the epilogue
         atomicExch(&sm.failed, 1);
         break;
       }
@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                          kHk = (2 * 32 * 16) >> 4;
       uint32_t s = 0, ph = 0, b = 0, bph = 0;
       for (int64_t t = t_begin; t < t_end; ++t) {
-        if (!wait_parity(&sm.full[s], ph) || !wait_parity(&sm.acc_empty[b], bph ^ 1u)) {
+        if (!wait_parity_sleep(&sm.full[s], ph) ||
+            !wait_parity_sleep(&sm.acc_empty[b], bph ^ 1u)) {
           atomicExch(&sm.failed, 1);
           break;
         }

@@ -62,6 +62,28 @@ __device__ __forceinline__ bool wait_parity(unsigned long long* bar,
   return false;
 }
 
+// wait_parity for threads off the critical path (a producer that runs
+// ahead of a slower consumer): between failed polls the thread sleeps, so
+// its polls do not take issue slots from the warps doing the work.
+constexpr unsigned kPollSleepNs = 128;
+__device__ __forceinline__ bool wait_parity_sleep(unsigned long long* bar,
+                                                  uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (long long i = 0; i < kWaitLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    __nanosleep(kPollSleepNs);
+  }
+  return false;
+}
+
 __device__ __forceinline__ void expect_tx(unsigned long long* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
