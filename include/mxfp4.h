@@ -146,7 +146,10 @@ mxfp4_status mxfp4_double_quantize(const void* x, int dtype, int64_t rows,
  * in both passes. The row pass moves where a group maximum would scale above
  * 6; the column pass then sees decoded values with two significant bits,
  * whose maxima never scale above 6, so its scales follow the OCP rule as
- * well. Same arguments, layouts and statuses as mxfp4_double_quantize.
+ * well. A row scale of 2^126 gives Q_D(X) values of 4 * 2^126 and 6 * 2^126,
+ * beyond the fp32 range; the column pass still quantizes them exactly (to
+ * codes 4 and 6 at column scale 2^126). Same arguments, layouts and statuses
+ * as mxfp4_double_quantize.
  * Source: "Unveiling the Potential of Quantization with MXFP4", abstract
  * (overflow-aware scaling), with the double quantization above.
  */
