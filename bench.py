@@ -550,6 +550,8 @@ def run_ours(args):
         oout = (u8(R, C // 2), u8(R, C // 32))
         dout = (u8(R, C // 2), u8(R, C // 32), u8(C, R // 2), u8(C, R // 32))
         for name, step_op, fn in (
+                ("quant_rows_sr", "quant_rows_rne",
+                 lambda: m.quantize(buf0["x"], m.ROWS, m.SR, SEED, out=oout)),
                 ("quant_rows_rne_oas", "quant_rows_rne",
                  lambda: m.quantize(buf0["x"], m.ROWS, m.RNE, out=oout, oas=True)),
                 ("double_quant_oas", "double_quant",

@@ -252,6 +252,12 @@ __device__ __forceinline__ uint32_t e2m1_sr_top_scaled(float v, float half, floa
   return (__float_as_uint(y) * 64u + noise) | (__float_as_uint(v) & 0x80000000u);
 }
 
+// e2m1x8_sr on 8 unscaled values (e2m1_sr_top_scaled; scale byte in
+// [2, 252], or up to 253 with SAT = false).
+template <bool SAT>
+__device__ __forceinline__ uint32_t e2m1x8_sr_scaled(const float* v, const uint32_t* g,
+                                                    float half, float sat, uint32_t base);
+
 // Shift a packed code word up by one nibble and append the code held in the
 // top nibble of t: codes pushed in the order 7, 6, .., 0 land in nibbles
 // 7 .. 0.
@@ -271,6 +277,20 @@ __device__ __forceinline__ uint32_t e2m1x8_sr(const float* v,
     sr_noise64_pair(g[k], ne, no);
     out = push_code(out, e2m1_sr_top(v[2 * k + 1], no));
     out = push_code(out, e2m1_sr_top(v[2 * k], ne));
+  }
+  return out;
+}
+
+template <bool SAT>
+__device__ __forceinline__ uint32_t e2m1x8_sr_scaled(const float* v, const uint32_t* g,
+                                                    float half, float sat, uint32_t base) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 3; k >= 0; --k) {
+    uint32_t ne, no;
+    sr_noise64_pair_based(g[k], base, base, ne, no);
+    out = push_code(out, e2m1_sr_top_scaled<SAT>(v[2 * k + 1], half, sat, no));
+    out = push_code(out, e2m1_sr_top_scaled<SAT>(v[2 * k], half, sat, ne));
   }
   return out;
 }

@@ -34,10 +34,13 @@ namespace {
 
 constexpr int kRowThreads = 256;
 
+// Nearest rounding (SR = false; stochastic rounding along rows is
+// k_quant_rows_sr below).
 template <bool BF16, bool SR, int U, bool OAS = false>
 __global__ void __launch_bounds__(kRowThreads)
-    k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey key,
+    k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey,
                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  static_assert(!SR, "stochastic rounding along rows is k_quant_rows_sr");
   const int lane = threadIdx.x & 31;
   const int sub = lane & 3;
   const int64_t warp = (int64_t(blockIdx.x) * kRowThreads + threadIdx.x) >> 5;
@@ -88,22 +91,106 @@ __global__ void __launch_bounds__(kRowThreads)
       const float mul = inv_scale(sb);
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[u][j] *= mul;
-      uint32_t word;
-      if (SR) {
-        const uint64_t p0 = uint64_t(g) * 16 + uint64_t(sub) * 4;
-        const uint32_t kh = inner_key(key, uint32_t(p0 >> 32));
-        uint32_t h[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) h[k] = mix32_pre(kh + uint32_t(p0) + k);
-        word = e2m1x8_sr(v[u], h);
-      } else {
-        word = e2m1x8_rn(v[u]);
-      }
+      uint32_t word = e2m1x8_rn(v[u]);
       if (sb == 0xFFu) word = 0;
       if (ok[u]) {
         reinterpret_cast<uint32_t*>(codes)[g * 4 + sub] = word;
         if (sub == 0) scales[g] = static_cast<uint8_t>(sb);
       }
+    }
+  }
+}
+
+// Row groups with stochastic rounding: one thread per whole 1x32 group.
+// The counter hash and the exact rounding decision make this path bound by
+// instruction issue, so the group's maximum and scale are computed once, by
+// the thread that rounds all 32 values, rather than by four threads with
+// shuffles. Consecutive threads take consecutive groups; a group's 64 (bf16)
+// or 128 (fp32) bytes arrive as 16-byte L1-allocating loads, which together
+// cover whole sectors, U groups in flight per thread.
+template <bool BF16, bool OAS, int U>
+__global__ void __launch_bounds__(kRowThreads)
+    k_quant_rows_sr(const void* __restrict__ x, int64_t n_groups, RngKey key,
+                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  constexpr int kLoads = BF16 ? 4 : 8;  // 16-byte pieces per group
+  const int64_t stride = int64_t(gridDim.x) * kRowThreads;
+  for (int64_t base = int64_t(blockIdx.x) * kRowThreads + threadIdx.x; base < n_groups;
+       base += stride * U) {
+    uint4 w[U][kLoads];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * stride;
+      const uint4* p = reinterpret_cast<const uint4*>(static_cast<const char*>(x) +
+                                                      g * (BF16 ? 64 : 128));
+#pragma unroll
+      for (int k = 0; k < kLoads; ++k)
+        w[u][k] = g < n_groups ? ld_l1(p + k) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t g = base + u * stride;
+      if (g >= n_groups) break;
+      float v[32];
+      uint32_t amax;
+      if (BF16) {
+        uint32_t m[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 q = w[u][k];
+          v[8 * k] = bf16_lo(q.x), v[8 * k + 1] = bf16_hi(q.x);
+          v[8 * k + 2] = bf16_lo(q.y), v[8 * k + 3] = bf16_hi(q.y);
+          v[8 * k + 4] = bf16_lo(q.z), v[8 * k + 5] = bf16_hi(q.z);
+          v[8 * k + 6] = bf16_lo(q.w), v[8 * k + 7] = bf16_hi(q.w);
+          m[2 * k] = bf16x2_absmax_nan(q.x, q.y);
+          m[2 * k + 1] = bf16x2_absmax_nan(q.z, q.w);
+        }
+#pragma unroll
+        for (int n = 4; n >= 1; n /= 2)
+#pragma unroll
+          for (int i = 0; i < n; ++i) m[i] = bf16x2_absmax_nan(m[i], m[i + n]);
+        const uint32_t mm = m[0] & 0x7FFF7FFFu;
+        amax = max(mm << 16, mm & 0xFFFF0000u);
+      } else {
+        amax = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 q = w[u][k];
+          v[4 * k] = __uint_as_float(q.x), v[4 * k + 1] = __uint_as_float(q.y);
+          v[4 * k + 2] = __uint_as_float(q.z), v[4 * k + 3] = __uint_as_float(q.w);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) amax = max(amax, __float_as_uint(v[j]) & 0x7FFFFFFFu);
+      }
+      const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
+      // the group's 16 pairs start at a multiple of 16: one inner key
+      const uint64_t p0 = uint64_t(g) * 16;
+      const uint32_t kh = inner_key(key, uint32_t(p0 >> 32)) + uint32_t(p0);
+      uint32_t word[4];
+      if (sb >= 2u && sb != 0xFFu) {
+        // the power of two rides on the rounding (e2m1_sr_top_scaled)
+        const float half = scale_half(sb), sat = OAS ? 0.0f : scale_six(sb);
+        const uint32_t nb = sr_noise64_base(sb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t h[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) h[k] = mix32_pre(kh + uint32_t(4 * q + k));
+          word[q] = e2m1x8_sr_scaled<!OAS>(v + 8 * q, h, half, sat, nb);
+        }
+      } else {
+        const float mul = inv_scale(sb);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= mul;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t h[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) h[k] = mix32_pre(kh + uint32_t(4 * q + k));
+          word[q] = sb == 0xFFu ? 0u : e2m1x8_sr(v + 8 * q, h);
+        }
+      }
+      reinterpret_cast<uint4*>(codes)[g] = make_uint4(word[0], word[1], word[2], word[3]);
+      scales[g] = static_cast<uint8_t>(sb);
     }
   }
 }
@@ -904,15 +991,23 @@ template <bool BF16, bool SR, bool OAS>
 static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
-  constexpr int U = BF16 ? 4 : 2;  // 8 lowers occupancy and runs slower
-  auto kern = k_quant_rows<BF16, SR, U, OAS>;
-  const int64_t groups_per_block = (kRowThreads / 4) * U;
-  const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
-                                   kRowThreads, 0,
-                                   (n_groups + groups_per_block - 1) /
-                                       groups_per_block);
-  kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
-  return cudaGetLastError();
+  if constexpr (SR) {
+    constexpr int U = BF16 ? 2 : 1;
+    auto kern = k_quant_rows_sr<BF16, OAS, U>;
+    const int64_t groups_per_block = int64_t(kRowThreads) * U;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRowThreads, 0,
+                                     (n_groups + groups_per_block - 1) / groups_per_block);
+    kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
+    return cudaGetLastError();
+  } else {
+    constexpr int U = BF16 ? 4 : 2;  // 8 lowers occupancy and runs slower
+    auto kern = k_quant_rows<BF16, SR, U, OAS>;
+    const int64_t groups_per_block = (kRowThreads / 4) * U;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRowThreads, 0,
+                                     (n_groups + groups_per_block - 1) / groups_per_block);
+    kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
+    return cudaGetLastError();
+  }
 }
 
 template <bool OAS>

@@ -210,6 +210,22 @@ def test_double_quant_extreme_scales(oas, dtype):
         assert_bits_equal(to_np(g_), w, "extreme-scale double quant " + name)
 
 
+@pytest.mark.parametrize("oas", [False, True])
+def test_column_kernels_multi_tile_ragged(oas):
+    """2080 x 4000: 17 x 32 tiles of 128 x 128 with a ragged last row and
+    column tile, more tiles than resident blocks (each block walks several,
+    interior tiles on the unchecked staging path), compared in full."""
+    x = rand_tensor((2080, 4000), "bf16", 21, spread=12)
+    c, s = m.quantize(to_dev(x), m.COLS, m.SR, 13, oas=oas)
+    oc, os_ = O.quantize(x, O.COLS, O.SR, 13, oas=oas)
+    assert_bits_equal(to_np(c), oc, "multi-tile column codes")
+    assert_bits_equal(to_np(s), os_, "multi-tile column scales")
+    got = m.double_quantize(to_dev(x), seed=13, oas=oas)
+    want = O.double_quantize(x, 13, oas=oas)
+    for g_, w, name in zip(got, want, ("row codes", "row scales", "col codes", "col scales")):
+        assert_bits_equal(to_np(g_), w, "multi-tile double quant " + name)
+
+
 # ---------------------------------------------------------------------------
 # Dequantize
 # ---------------------------------------------------------------------------
