@@ -8,12 +8,13 @@
 // backward GEMM).
 //
 // Row groups: a [rows, cols] tensor with cols % 32 == 0 is a flat array of
-// rows*cols/32 groups, so the row kernel is a grid-stride loop over groups.
-// Four threads share a group (8 elements, one 16-byte load per thread for
-// bf16), the absmax is reduced with two quad shuffles, and each thread
-// writes the 4 code bytes of its 8 elements; a warp covers 8 consecutive
-// groups per load, so loads and code stores are fully coalesced. U groups
-// per quad are loaded before any arithmetic to keep enough bytes in flight.
+// rows*cols/32 groups, so the row kernel is a grid-stride loop over groups,
+// one thread per group: its 16-byte loads of a group (L1-allocating, so the
+// warp's loads together read whole sectors) are all issued, for U groups,
+// before any arithmetic; the maximum and the scale are computed once per
+// group and its 32 codes leave in one 16-byte store. (A form with four
+// threads per group, one 16-byte load each and quad shuffles, ran 12%
+// slower for nearest rounding and 22% slower for stochastic rounding.)
 //
 // Column groups: a CTA stages a 128-row tile (128 bf16 or 64 fp32 columns)
 // in shared memory, then each thread reduces two adjacent columns over 32
@@ -34,84 +35,16 @@ namespace {
 
 constexpr int kRowThreads = 256;
 
-// Nearest rounding (SR = false; stochastic rounding along rows is
-// k_quant_rows_sr below).
+// One thread per whole 1x32 group: the group's maximum and scale are
+// computed once, by the thread that rounds all 32 values, with no shuffles.
+// Consecutive threads take consecutive groups; a group's 64 (bf16) or 128
+// (fp32) bytes arrive as 16-byte L1-allocating loads, which together cover
+// whole sectors, U groups in flight per thread; each group leaves as one
+// 16-byte code store and its scale byte.
 template <bool BF16, bool SR, int U, bool OAS = false>
 __global__ void __launch_bounds__(kRowThreads)
-    k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey,
+    k_quant_rows(const void* __restrict__ x, int64_t n_groups, RngKey key,
                  uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
-  static_assert(!SR, "stochastic rounding along rows is k_quant_rows_sr");
-  const int lane = threadIdx.x & 31;
-  const int sub = lane & 3;
-  const int64_t warp = (int64_t(blockIdx.x) * kRowThreads + threadIdx.x) >> 5;
-  const int64_t chunk = (int64_t(gridDim.x) * kRowThreads) >> 2;  // quads
-  const int64_t my = warp * 8 + (lane >> 2);
-
-  for (int64_t base = 0; base < n_groups; base += chunk * U) {
-    float v[U][8];
-    uint32_t pmax[U];
-    bool ok[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t g = base + u * chunk + my;
-      ok[u] = g < n_groups;
-      if (BF16) {
-        uint4 w = ok[u] ? ld_stream(static_cast<const uint16_t*>(x) + g * 32 +
-                                    sub * 8)
-                        : make_uint4(0, 0, 0, 0);
-        pmax[u] = bf16x8_absmax(w);
-        v[u][0] = bf16_lo(w.x), v[u][1] = bf16_hi(w.x);
-        v[u][2] = bf16_lo(w.y), v[u][3] = bf16_hi(w.y);
-        v[u][4] = bf16_lo(w.z), v[u][5] = bf16_hi(w.z);
-        v[u][6] = bf16_lo(w.w), v[u][7] = bf16_hi(w.w);
-      } else {
-        const float* p = static_cast<const float*>(x) + g * 32 + sub * 8;
-        uint4 a = ok[u] ? ld_stream(p) : make_uint4(0, 0, 0, 0);
-        uint4 b = ok[u] ? ld_stream(p + 4) : make_uint4(0, 0, 0, 0);
-        v[u][0] = __uint_as_float(a.x), v[u][1] = __uint_as_float(a.y);
-        v[u][2] = __uint_as_float(a.z), v[u][3] = __uint_as_float(a.w);
-        v[u][4] = __uint_as_float(b.x), v[u][5] = __uint_as_float(b.y);
-        v[u][6] = __uint_as_float(b.z), v[u][7] = __uint_as_float(b.w);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int64_t g = base + u * chunk + my;
-      uint32_t amax = 0;
-      if (BF16) {
-        amax = pmax[u];
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          amax = max(amax, __float_as_uint(v[u][j]) & 0x7FFFFFFFu);
-      }
-      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-      amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-      const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
-      const float mul = inv_scale(sb);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[u][j] *= mul;
-      uint32_t word = e2m1x8_rn(v[u]);
-      if (sb == 0xFFu) word = 0;
-      if (ok[u]) {
-        reinterpret_cast<uint32_t*>(codes)[g * 4 + sub] = word;
-        if (sub == 0) scales[g] = static_cast<uint8_t>(sb);
-      }
-    }
-  }
-}
-
-// Row groups with stochastic rounding: one thread per whole 1x32 group.
-// The counter hash and the exact rounding decision make this path bound by
-// instruction issue, so the group's maximum and scale are computed once, by
-// the thread that rounds all 32 values, rather than by four threads with
-// shuffles. Consecutive threads take consecutive groups; a group's 64 (bf16)
-// or 128 (fp32) bytes arrive as 16-byte L1-allocating loads, which together
-// cover whole sectors, U groups in flight per thread.
-template <bool BF16, bool OAS, int U>
-__global__ void __launch_bounds__(kRowThreads)
-    k_quant_rows_sr(const void* __restrict__ x, int64_t n_groups, RngKey key,
-                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   constexpr int kLoads = BF16 ? 4 : 8;  // 16-byte pieces per group
   const int64_t stride = int64_t(gridDim.x) * kRowThreads;
   for (int64_t base = int64_t(blockIdx.x) * kRowThreads + threadIdx.x; base < n_groups;
@@ -166,7 +99,13 @@ __global__ void __launch_bounds__(kRowThreads)
       const uint64_t p0 = uint64_t(g) * 16;
       const uint32_t kh = inner_key(key, uint32_t(p0 >> 32)) + uint32_t(p0);
       uint32_t word[4];
-      if (sb >= 2u && sb != 0xFFu) {
+      if (!SR) {
+        const float mul = inv_scale(sb);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= mul;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) word[q] = sb == 0xFFu ? 0u : e2m1x8_rn(v + 8 * q);
+      } else if (sb >= 2u && sb != 0xFFu) {
         // the power of two rides on the rounding (e2m1_sr_top_scaled)
         const float half = scale_half(sb), sat = OAS ? 0.0f : scale_six(sb);
         const uint32_t nb = sr_noise64_base(sb);
@@ -991,23 +930,13 @@ template <bool BF16, bool SR, bool OAS>
 static cudaError_t quant_rows_impl(const void* x, int64_t n_groups,
                                    RngKey key, uint8_t* codes,
                                    uint8_t* scales, cudaStream_t s) {
-  if constexpr (SR) {
-    constexpr int U = BF16 ? 2 : 1;
-    auto kern = k_quant_rows_sr<BF16, OAS, U>;
-    const int64_t groups_per_block = int64_t(kRowThreads) * U;
-    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRowThreads, 0,
-                                     (n_groups + groups_per_block - 1) / groups_per_block);
-    kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
-    return cudaGetLastError();
-  } else {
-    constexpr int U = BF16 ? 4 : 2;  // 8 lowers occupancy and runs slower
-    auto kern = k_quant_rows<BF16, SR, U, OAS>;
-    const int64_t groups_per_block = (kRowThreads / 4) * U;
-    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRowThreads, 0,
-                                     (n_groups + groups_per_block - 1) / groups_per_block);
-    kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
-    return cudaGetLastError();
-  }
+  constexpr int U = BF16 ? 2 : 1;
+  auto kern = k_quant_rows<BF16, SR, U, OAS>;
+  const int64_t groups_per_block = int64_t(kRowThreads) * U;
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRowThreads, 0,
+                                   (n_groups + groups_per_block - 1) / groups_per_block);
+  kern<<<grid, kRowThreads, 0, s>>>(x, n_groups, key, codes, scales);
+  return cudaGetLastError();
 }
 
 template <bool OAS>
