@@ -198,6 +198,22 @@ def test_column_sr_extreme_scales(dtype, oas):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("rnd", [O.RNE, O.SR])
+@pytest.mark.parametrize("oas", [False, True])
+def test_row_quant_extreme_scales(dtype, rnd, oas):
+    # the same groups along rows: the row kernel folds the scale into
+    # stochastic rounding for bytes 2..252 and multiplies otherwise
+    x = np.ascontiguousarray(extreme_scale_columns(dtype, 14).T)
+    c, s = m.quantize(to_dev(x), m.ROWS, rnd, 8, oas=oas)
+    oc, os_ = O.quantize(x, O.ROWS, rnd, 8, oas=oas)
+    if not oas:
+        for i, (_, sb) in enumerate(EXTREME_PEAKS):
+            assert (os_[64 * i:64 * (i + 1)] == sb).all()
+    assert_bits_equal(to_np(c), oc, "extreme-scale row codes")
+    assert_bits_equal(to_np(s), os_, "extreme-scale row scales")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("oas", [False, True])
 def test_double_quant_extreme_scales(oas, dtype):
     # overflow-aware row scales reach 2^126 here, where Q_D(X) holds 4 2^126
