@@ -95,11 +95,37 @@ def _dtype_code(t):
     raise TypeError("expected a bfloat16 or float32 tensor, got %s" % t.dtype)
 
 
-def _cuda2d(t, name):
+def _on_device(t, name, device=None):
+    """t is a CUDA tensor (on `device` when one is given)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def _cuda2d(t, name):
+    if not isinstance(t, torch.Tensor):
         raise TypeError("%s must be a CUDA tensor" % name)
     if t.dim() != 2 or not t.is_contiguous():
         raise ValueError("%s must be a contiguous 2-D tensor" % name)
+    _on_device(t, name)
+    return t
+
+
+def _buffer(t, name, dtype, numel, device):
+    """Check a buffer before its pointer reaches the C ABI, which cannot see
+    sizes: the library reads and writes exactly the bytes the header states
+    for the given shape, so a smaller, strided, mistyped or foreign-device
+    buffer would be read or written out of bounds. Raises before any launch."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a tensor" % name)
+    if t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.numel() != numel:
+        raise ValueError("%s must hold %d elements, got %d" % (name, numel, t.numel()))
+    _on_device(t, name, device)
     return t
 
 
@@ -128,6 +154,8 @@ def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None,
         shape_s = (R, C // 32) if axis == ROWS else (C, R // 32)
         out = (_empty_u8(shape_c, x.device), _empty_u8(shape_s, x.device))
     codes, scales = out
+    _buffer(codes, "codes", torch.uint8, R * C // 2, x.device)
+    _buffer(scales, "scales", torch.uint8, R * C // 32, x.device)
     fn = lib().mxfp4_quantize_oas if oas else lib().mxfp4_quantize
     _check(fn(_ptr(x), _dtype_code(x), R, C, axis, rounding, seed, _ptr(codes),
               _ptr(scales), _stream(x.device, stream)), "mxfp4_quantize")
@@ -137,11 +165,15 @@ def quantize(x, axis=ROWS, rounding=RNE, seed=0, out=None, stream=None,
 def dequantize(codes, scales, rows, cols, axis=ROWS, out_dtype=torch.bfloat16,
                out=None, stream=None):
     """mxfp4_dequantize: values [rows, cols] (ROWS) or [cols, rows] (COLS)."""
-    if not codes.is_cuda or not scales.is_cuda:
-        raise TypeError("codes and scales must be CUDA tensors")
+    _on_device(codes, "codes")
+    n = int(rows) * int(cols)
+    _buffer(codes, "codes", torch.uint8, n // 2, codes.device)
+    _buffer(scales, "scales", torch.uint8, n // 32, codes.device)
     if out is None:
         shape = (rows, cols) if axis == ROWS else (cols, rows)
         out = torch.empty(shape, dtype=out_dtype, device=codes.device)
+    _dtype_code(out)
+    _buffer(out, "out", out.dtype, n, codes.device)
     _check(lib().mxfp4_dequantize(_ptr(codes), _ptr(scales), rows, cols, axis,
                                   _ptr(out), _dtype_code(out),
                                   _stream(codes.device, stream)),
@@ -159,6 +191,9 @@ def double_quantize(x, seed=0, out=None, stream=None, oas=False):
         out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d),
                _empty_u8((C, R // 2), d), _empty_u8((C, R // 32), d))
     rc, rs, cc, cs = out
+    for t, nm, n in ((rc, "row_codes", R * C // 2), (rs, "row_scales", R * C // 32),
+                     (cc, "col_codes", R * C // 2), (cs, "col_scales", R * C // 32)):
+        _buffer(t, nm, torch.uint8, n, x.device)
     name = "mxfp4_double_quantize_oas" if oas else "mxfp4_double_quantize"
     _check(getattr(lib(), name)(_ptr(x), _dtype_code(x), R, C, seed, _ptr(rc),
                                 _ptr(rs), _ptr(cc), _ptr(cs),
@@ -178,6 +213,10 @@ def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
         rot = torch.empty((R, C), dtype=torch.float32, device=d) if want_rotated else None
         out = (_empty_u8((R, C // 2), d), _empty_u8((R, C // 32), d), rot)
     codes, scales, rot = out
+    _buffer(codes, "codes", torch.uint8, R * C // 2, x.device)
+    _buffer(scales, "scales", torch.uint8, R * C // 32, x.device)
+    if rot is not None:
+        _buffer(rot, "rotated", torch.float32, R * C, x.device)
     name = "mxfp4_rht_quantize_oas" if oas else "mxfp4_rht_quantize"
     _check(getattr(lib(), name)(_ptr(x), _dtype_code(x), R, C, sign_seed, rounding,
                                 sr_seed, _ptr(codes), _ptr(scales), _ptr(rot),
@@ -194,9 +233,10 @@ def osc_step(w, w_snap, d_w, d_q, window_end=False, threshold=4.0,
         _cuda2d(t, name)
         if t.dtype != torch.float32 or t.shape != w.shape:
             raise TypeError("%s must be float32 with the shape of w" % name)
-    if n_flagged is not None and (not n_flagged.is_cuda
-                                  or n_flagged.dtype not in (torch.int64, torch.uint64)):
-        raise TypeError("n_flagged must be a CUDA int64 tensor")
+        _on_device(t, name, w.device)
+    if n_flagged is not None:
+        _buffer(n_flagged, "n_flagged", torch.int64 if n_flagged.dtype != torch.uint64
+                else torch.uint64, 1, w.device)
     R, C = w.shape
     _check(lib().mxfp4_osc_step(_ptr(w), _ptr(w_snap), _ptr(d_w), _ptr(d_q),
                                 R, C, int(bool(window_end)), threshold,
@@ -222,10 +262,13 @@ def qema_quantize(w, w_ema, beta=0.998, out=None, stream=None):
         _cuda2d(t, name)
         if t.dtype != torch.float32 or t.shape != w.shape:
             raise TypeError("%s must be float32 with the shape of w" % name)
+    _on_device(w_ema, "w_ema", w.device)
     R, C = w.shape
     if out is None:
         out = (_empty_u8((R, C // 2), w.device), _empty_u8((R, C // 32), w.device))
     codes, scales = out
+    _buffer(codes, "codes", torch.uint8, R * C // 2, w.device)
+    _buffer(scales, "scales", torch.uint8, R * C // 32, w.device)
     _check(lib().mxfp4_qema_quantize(_ptr(w), _ptr(w_ema), R, C, beta,
                                      _ptr(codes), _ptr(scales),
                                      _stream(w.device, stream)),
@@ -244,6 +287,8 @@ def scales_to_blocked(scales, out=None, stream=None):
     if out is None:
         out = _empty_u8((-(-rows // 128) * 128, -(-groups // 4) * 4),
                         scales.device)
+    _buffer(out, "out", torch.uint8, -(-rows // 128) * 128 * (-(-groups // 4) * 4),
+            scales.device)
     _check(lib().mxfp4_scales_to_blocked(_ptr(scales), rows, groups, _ptr(out),
                                          _stream(scales.device, stream)),
            "mxfp4_scales_to_blocked")
@@ -265,8 +310,12 @@ def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None):
         need = -(-rows // 128) * 128 * (-(-k // 128) * 4)
         if t.numel() != need:
             raise ValueError("%s must hold %d bytes" % (name, need))
+    for name, t in (("a_blocked", a_blocked), ("b_codes", b_codes),
+                    ("b_blocked", b_blocked)):
+        _on_device(t, name, a_codes.device)
     if out is None:
         out = torch.empty((m, n), dtype=torch.float32, device=a_codes.device)
+    _buffer(out, "out", torch.float32, m * n, a_codes.device)
     _check(lib().mxfp4_gemm(_ptr(a_codes), _ptr(a_blocked), _ptr(b_codes),
                             _ptr(b_blocked), m, n, k, _ptr(out),
                             _stream(a_codes.device, stream)), "mxfp4_gemm")
