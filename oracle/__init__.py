@@ -78,6 +78,8 @@ def _declare(L):
                               _u8p, _fp], i32),
         "orc_rht_quantize_oas": ([vp, i32, i64, i64, i64, u64, i32, u64, _u8p,
                                   _u8p, _fp], i32),
+        "orc_qramp_step": ([_fp, _fp, _fp, _fp, _fp, _fp, _u8p, i64, i64, i64, i64,
+                            ctypes.c_float, i64], i64),
         "orc_osc_step": ([_fp, _fp, _fp, _fp, i64, i64, i32, ctypes.c_float],
                          i64),
         "orc_osc_synthetic_update": ([_fp, i64, i64, i64, u64, u32,
@@ -222,6 +224,22 @@ class Oracle:
                                 R, C, int(bool(window_end)), threshold)
         if n < 0:
             raise ValueError("bad shape for the oracle tracker")
+        return int(n)
+
+    def qramp_step(self, w, delta, w_snap, d_w, d_q, acc, flag, it, track_iters=30,
+                   k1=16.0, k2=5):
+        """One Q-Ramping iteration on fp32 arrays (flag: uint8), in place;
+        returns the number of weights flagged at this iteration."""
+        for a in (w, delta, w_snap, d_w, d_q, acc):
+            if a.dtype != np.float32 or not a.flags.c_contiguous or a.shape != w.shape:
+                raise TypeError("Q-Ramping state must be contiguous float32 of w's shape")
+        if flag.dtype != np.uint8 or not flag.flags.c_contiguous or flag.shape != w.shape:
+            raise TypeError("flag must be contiguous uint8 of w's shape")
+        R, C = w.shape
+        n = self.L.orc_qramp_step(_f32(w), _f32(delta), _f32(w_snap), _f32(d_w), _f32(d_q),
+                                  _f32(acc), _u8(flag), R, C, it, track_iters, k1, k2)
+        if n < 0:
+            raise ValueError("bad arguments for the oracle Q-Ramping step")
         return int(n)
 
     def osc_synthetic_update(self, w, seed, step, rel_step=1e-4, row0=0):

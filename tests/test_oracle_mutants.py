@@ -19,6 +19,18 @@ SRC = os.path.join(os.path.dirname(O.__file__), "mxfp4_oracle.c")
 
 # (name, original text, mutated text, pins that must fail)
 MUTANTS = [
+    ("Q-Ramping flag test inclusive", "flag[i] = d_q[i] > limit ? 1 : 0;",
+     "flag[i] = d_q[i] >= limit ? 1 : 0;",
+     ["test_qramp_flags_the_worked_oscillation_and_not_the_drift"]),
+    ("Q-Ramping gathered update every iteration", "if (iter % k2 == k2 - 1) {",
+     "if (1) {", ["test_qramp_flagged_weight_updates_every_k2th_iteration"]),
+    ("Q-Ramping held updates dropped at the epoch start",
+     "if (flag[i]) w[i] = (float)((double)w[i] + (double)acc[i]);", "",
+     ["test_qramp_flagged_weight_updates_every_k2th_iteration"]),
+    ("Q-Ramping window without the absolute value",
+     "float moved_q = (float)fabs(qw[i] - qs[i]);",
+     "float moved_q = (float)(qw[i] - qs[i]);",
+     ["test_qramp_window_accumulates_like_the_tracker"]),
     ("overflow-aware bound inclusive", "ldexp(absmax, -e) > 6.0",
      "ldexp(absmax, -e) >= 6.0",
      ["test_oas_scale_is_the_smallest_non_saturating_exponent",

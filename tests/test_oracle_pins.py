@@ -546,6 +546,124 @@ def test_osc_synthetic_update_magnitude_and_signs():
 
 
 # --------------------------------------------------------------------------
+# Q-Ramping (TetraJet rebuttal, Weakness 2 and the hyper-parameter answers:
+# track the first iterations of an epoch, detection factor k1, update
+# frequency factor k2). The rule is a reading; the pins check it against
+# plain fp32 update loops, the tracker's own (pinned) accumulators and the
+# page's worked ratio.
+# --------------------------------------------------------------------------
+
+def _qramp_state(w0):
+    w = w0.copy()
+    z = np.zeros_like(w)
+    return w, w.copy(), z.copy(), z.copy(), z.copy(), np.zeros(w.shape, np.uint8)
+
+
+def test_qramp_without_flags_is_the_plain_update():
+    g = np.random.Generator(np.random.PCG64(41))
+    w0 = g.normal(0, 0.02, size=(4, 64)).astype(np.float32)
+    deltas = [(g.normal(0, 1e-3, size=w0.shape)).astype(np.float32) for _ in range(12)]
+    for track in (0, 3):  # no window, and a window whose flags stay clear
+        w, ws, dw, dq, acc, fl = _qramp_state(w0)
+        ref = w0.copy()
+        for it, d in enumerate(deltas):
+            n = O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=track,
+                             k1=1e30, k2=5)
+            ref = (ref + d).astype(np.float32)  # one fp32 add per iteration
+            assert n == 0
+        assert np.array_equal(w, ref) and not fl.any() and not acc.any()
+
+
+def test_qramp_k2_one_is_the_plain_update_even_when_flagged():
+    g = np.random.Generator(np.random.PCG64(42))
+    w0 = g.normal(0, 0.02, size=(2, 32)).astype(np.float32)
+    w, ws, dw, dq, acc, fl = _qramp_state(w0)
+    ref = w0.copy()
+    for it in range(10):
+        d = g.normal(0, 1e-3, size=w0.shape).astype(np.float32)
+        O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=2, k1=-1.0, k2=1)
+        ref = (ref + d).astype(np.float32)
+    assert fl.all()  # k1 = -1 flags every weight that moved
+    assert np.array_equal(w, ref)
+
+
+def test_qramp_window_accumulates_like_the_tracker():
+    """Inside the window the Q-Ramping accumulators are the ALTO tracker's on
+    the same weights (the tracker is pinned by the page's worked example)."""
+    from mxfp4_block_quantization_quantizer_b200 import workloads as W
+    w0 = W.osc_w(seed=3, rows=8, cols=128)
+    w, ws, dw, dq, acc, fl = _qramp_state(w0)
+    tw, tws, tdw, tdq = w0.copy(), w0.copy(), np.zeros_like(w0), np.zeros_like(w0)
+    g = np.random.Generator(np.random.PCG64(43))
+    for it in range(6):
+        d = (np.where(g.random(w0.shape) < 0.5, -1.0, 1.0) * 1e-4 * np.abs(w)).astype(np.float32)
+        O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=30)
+        tw = (tw + d).astype(np.float32)
+        O.osc_step(tw, tws, tdw, tdq, window_end=False)
+        assert np.array_equal(w, tw) and np.array_equal(ws, tws)
+        assert np.array_equal(dw, tdw) and np.array_equal(dq, tdq)
+
+
+def test_qramp_flags_the_worked_oscillation_and_not_the_drift():
+    ex = load("osc_worked_example.json")
+    k1 = 16.0  # the detection factor the page recommends
+    for case in ex["cases"]:
+        assert (case["ratio"] > k1) == case["flagged"]  # 75 flagged, 0.83 not
+    # an element oscillating across the 0.625 edge (bins 0.5 / 0.75) and one
+    # drifting across it once, in one 32-group whose scale is fixed by a 3.0
+    base = np.zeros((1, 32), np.float32)
+    base[0, 0] = 3.0
+    base[0, 1] = 0.624
+    base[0, 2] = 0.55
+    w, ws, dw, dq, acc, fl = _qramp_state(base)
+    T = 30
+    flagged = None
+    for it in range(T):
+        d = np.zeros_like(base)
+        d[0, 1] = np.float32(0.002) if it % 2 == 0 else np.float32(-0.002)
+        d[0, 2] = np.float32(0.005)
+        flagged = O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=T, k1=k1, k2=5)
+    assert flagged == 1 and fl[0, 1] == 1 and fl[0, 2] == 0 and fl[0, 0] == 0
+    assert not dw.any() and not dq.any()  # reset at the window end
+
+
+def test_qramp_flagged_weight_updates_every_k2th_iteration():
+    base = np.zeros((1, 32), np.float32)
+    base[0, 0] = 3.0
+    base[0, 1] = 0.624
+    w, ws, dw, dq, acc, fl = _qramp_state(base)
+    T, k2 = 4, 3
+    for it in range(T):  # oscillate inside the window: flagged at its end
+        d = np.zeros_like(base)
+        d[0, 1] = np.float32(0.002) if it % 2 == 0 else np.float32(-0.002)
+        O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=T, k1=16.0, k2=k2)
+    assert fl[0, 1] == 1
+    w_start = w[0, 1]
+    steps = [2.0 ** -10, 2.0 ** -11, 2.0 ** -12, 2.0 ** -9, 2.0 ** -13]  # exact sums
+    f = np.float32
+    # iterations 4..8 with k2 = 3: the gathered updates land at 5 (steps 0, 1)
+    # and at 8 (steps 2, 3, 4); in between the weight stays put
+    want = {4: w_start, 5: f(w_start + f(steps[0] + steps[1])),
+            6: f(w_start + f(steps[0] + steps[1])), 7: f(w_start + f(steps[0] + steps[1]))}
+    want[8] = f(want[7] + f(f(steps[2] + steps[3]) + steps[4]))
+    for i, v in enumerate(steps):
+        it = T + i
+        d = np.zeros_like(base)
+        d[0, 1] = v
+        O.qramp_step(w, d, ws, dw, dq, acc, fl, it, track_iters=T, k1=16.0, k2=k2)
+        assert w[0, 1] == want[it], (it, w[0, 1], want[it])
+        assert (acc[0, 1] == 0) == (it % k2 == k2 - 1)
+    # the next epoch starts by applying what is still held and clearing flags
+    d = np.zeros_like(base)
+    d[0, 1] = 2.0 ** -14
+    acc[0, 1] = np.float32(2.0 ** -8)
+    before = w[0, 1]
+    O.qramp_step(w, d, ws, dw, dq, acc, fl, 0, track_iters=T, k1=16.0, k2=k2)
+    assert fl[0, 1] == 0 and acc[0, 1] == 0
+    assert w[0, 1] == np.float32(np.float32(before + np.float32(2.0 ** -8)) + np.float32(2.0 ** -14))
+
+
+# --------------------------------------------------------------------------
 # Q-EMA (TetraJet rebuttal, Question 4: quantize an EMA of the weight)
 # --------------------------------------------------------------------------
 
