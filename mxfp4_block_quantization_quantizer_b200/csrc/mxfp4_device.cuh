@@ -448,6 +448,140 @@ __device__ __forceinline__ uint4 ld_l1(const void* p) {
   return r;
 }
 
+// ---------------------------------------------------------------------------
+// Stochastic rounding of bf16 inputs with few integer-logic instructions.
+//
+// On sm_100a the integer-logic pipe (logic ops, shifts, byte permutes,
+// minimum/maximum, the E2M1 conversions) issues at half the rate of the FMA
+// pipes and bounds the stochastic-rounding kernels, so these helpers move
+// work onto the FMA pipes: a bf16 value is widened and scaled by 2^-e in
+// one exact mixed-precision product, the saturation runs on packed bf16
+// pairs, two codes share one byte-merge, and the signs are gathered from
+// the input words by byte permutes, eight codes at a time.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+// (a & c) | (b & ~c)
+__device__ __forceinline__ uint32_t bitsel(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// (a & b) | c
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// a * b + c on the multiply pipe (an integer add there would take a logic
+// pipe slot)
+__device__ __forceinline__ uint32_t mad_u32(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// Per half: the sign of w with magnitude min(|w|, sat), sat >= 0 (the
+// saturation at 6 2^e, a bf16 value, applied to two inputs at once).
+__device__ __forceinline__ uint32_t bf16x2_clamp_abs(uint32_t w, uint32_t sat2) {
+  uint32_t d;
+  asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(w), "r"(sat2));
+  return d;
+}
+// The low / high bf16 half of w times s16 (a bf16 power of two), as fp32:
+// one exact mixed-precision product on the FMA pipe (both factors have at
+// most 8 significant bits; no flush of subnormals).
+__device__ __forceinline__ float bf16lo_mul(uint32_t w, unsigned short s16) {
+  float d;
+  asm("{.reg .b16 l, h; mov.b32 {l, h}, %1;\n\t"
+      "fma.rn.f32.bf16 %0, l, %2, %3;}" : "=f"(d) : "r"(w), "h"(s16), "f"(-0.0f));
+  return d;
+}
+__device__ __forceinline__ float bf16hi_mul(uint32_t w, unsigned short s16) {
+  float d;
+  asm("{.reg .b16 l, h; mov.b32 {l, h}, %1;\n\t"
+      "fma.rn.f32.bf16 %0, h, %2, %3;}" : "=f"(d) : "r"(w), "h"(s16), "f"(-0.0f));
+  return d;
+}
+// 2^-e as bf16 bits for scale byte sb = e + 127 in [0, 253].
+__device__ __forceinline__ unsigned short bf16_inv_scale(uint32_t sb) {
+  return static_cast<unsigned short>((254u - sb) << 7);
+}
+// 6 2^e as bf16 bits in both halves (sb in [0, 252]).
+__device__ __forceinline__ uint32_t bf16x2_six_scale(uint32_t sb) {
+  return (((sb + 2u) << 7) | 0x40u) * 0x10001u;
+}
+
+// The rounding operand y of the carry test (e2m1_sr_top) of a scaled value
+// v, without saturation (callers clamp beforehand) and without the sign.
+__device__ __forceinline__ uint32_t sr_operand(float v) {
+  const float a = fabsf(v);
+  return __float_as_uint(fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f)));
+}
+// The same for v held unscaled, half = 2^(e-1) (e2m1_sr_top_scaled).
+__device__ __forceinline__ uint32_t sr_operand_scaled(float v, float half) {
+  const float a = fabsf(v);
+  return __float_as_uint(fmaxf(a, __fmaf_ru(a, 0.5f, half)));
+}
+
+// Two forms of the carry test's sum for scaled values: x64 (the sum times
+// 64, magnitude index in bits 28..30, the bits below are not part of it) =
+// y * 64 + r * 0xFFFFF000 + kSrBase64, and x4 (the sum times 4: index in
+// bits 24..26, bits 27..31 zero, since the sum is below 2^25) = y * 4 +
+// r * 0xFFFFFF00 + kSrBase4; r the element's 16-bit random number.
+constexpr uint32_t kSrBase64 = 64u * (0x400000u - 33u) - (0x3F000000u << 6);
+constexpr uint32_t kSrBase4 = 4u * (0x400000u - 33u) - (0x3F000000u << 2);
+// The bases for operands held unscaled by 2^e, e = u - 127 (see
+// sr_noise64_base): the sum is the same integer.
+__device__ __forceinline__ uint32_t sr_base64(uint32_t u) {
+  return 64u * (0x400000u - 33u) - ((0x3F000000u + ((u - 127u) << 23)) << 6);
+}
+__device__ __forceinline__ uint32_t sr_base4(uint32_t u) {
+  return 4u * (0x400000u - 33u) - ((0x3F000000u + ((u - 127u) << 23)) << 2);
+}
+
+// The byte of a pair of codes, in bits 24..31 (the bits below are not part
+// of it): the odd element's x64 sum over the even element's x4 sum, whose
+// bits above its index are zero; signs are added afterwards.
+__device__ __forceinline__ uint32_t pair_byte(uint32_t t_odd64, uint32_t t_even4) {
+  return and_or(t_odd64, 0xF0000000u, t_even4);
+}
+// Four pair bytes (pairs 0..3 of eight consecutive codes) into one code word.
+__device__ __forceinline__ uint32_t pack_pair_bytes(uint32_t b0, uint32_t b1, uint32_t b2,
+                                                    uint32_t b3) {
+  return prmt(prmt(b0, b1, 0x0073u), prmt(b2, b3, 0x7300u), 0x7610u);
+}
+
+// Sign bits (bit 4i+3) of the codes of 8 bf16 values held in 4 words,
+// element 2k in the low half of word k: byte permutes replicate each sign
+// over a byte, a bit select merges the even and odd elements' bytes.
+__device__ __forceinline__ uint32_t sign_nibbles_rows(uint32_t w0, uint32_t w1, uint32_t w2,
+                                                      uint32_t w3) {
+  const uint32_t p01 = prmt(w0, w1, 0xFDB9u), p23 = prmt(w2, w3, 0xFDB9u);
+  const uint32_t e = prmt(p01, p23, 0x6420u), o = prmt(p01, p23, 0x7531u);
+  return bitsel(e, o, 0x0F0F0F0Fu) & 0x88888888u;
+}
+// The same for two columns over 8 rows: word w[j] of row j holds column a
+// in its low half and column b in its high half (bf16 or f16); ta, tb get
+// the sign of row i in bit 4i+3.
+__device__ __forceinline__ void sign_nibbles_cols(const uint32_t* w, uint32_t& ta, uint32_t& tb) {
+  const uint32_t qlo = prmt(w[0], w[2], 0xFBD9u), rlo = prmt(w[1], w[3], 0xFBD9u);
+  const uint32_t qhi = prmt(w[4], w[6], 0xFBD9u), rhi = prmt(w[5], w[7], 0xFBD9u);
+  const uint32_t mlo = bitsel(qlo, rlo, 0x0F0F0F0Fu), mhi = bitsel(qhi, rhi, 0x0F0F0F0Fu);
+  ta = prmt(mlo, mhi, 0x5410u) & 0x88888888u;
+  tb = prmt(mlo, mhi, 0x7632u) & 0x88888888u;
+}
+
+// The two 16-bit random numbers of a pair whose hash has mix32_pre g (low
+// half, after the finalizer's last xorshift, for the even element).
+__device__ __forceinline__ void pair_randoms(uint32_t g, uint32_t& r_even, uint32_t& r_odd) {
+  r_odd = g >> 16;
+  r_even = (g ^ r_odd) & 0xFFFFu;
+}
+
 constexpr uint32_t kNaNbf16x2 = 0x7FC07FC0u;
 constexpr uint32_t kNaNf32 = 0x7FC00000u;
 

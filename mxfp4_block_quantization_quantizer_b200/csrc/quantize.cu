@@ -105,6 +105,31 @@ __global__ void __launch_bounds__(kRowThreads)
         for (int j = 0; j < 32; ++j) v[j] *= mul;
 #pragma unroll
         for (int q = 0; q < 4; ++q) word[q] = sb == 0xFFu ? 0u : e2m1x8_rn(v + 8 * q);
+      } else if (BF16 && sb != 0xFFu) {
+        // bf16: each value is widened and scaled by 2^-e in one exact
+        // mixed-precision product, after the packed pairs are saturated at
+        // 6 2^e (the overflow-aware rule never exceeds 6); the codes of a
+        // pair share one byte merge, the signs come from the input words
+        const unsigned short s16 = bf16_inv_scale(sb);
+        const uint32_t sat2 = bf16x2_six_scale(sb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t* wq = reinterpret_cast<const uint32_t*>(&w[u][q]);
+          uint32_t pb[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t ws = OAS ? wq[k] : bf16x2_clamp_abs(wq[k], sat2);
+            uint32_t re, ro;
+            pair_randoms(mix32_pre(mad_u32(uint32_t(4 * q + k), 1u, kh)), re, ro);
+            const uint32_t te = mad_u32(sr_operand(bf16lo_mul(ws, s16)), 4u,
+                                        mad_u32(re, 0xFFFFFF00u, kSrBase4));
+            const uint32_t to = mad_u32(sr_operand(bf16hi_mul(ws, s16)), 64u,
+                                        mad_u32(ro, 0xFFFFF000u, kSrBase64));
+            pb[k] = pair_byte(to, te);
+          }
+          word[q] = pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) |
+                    sign_nibbles_rows(wq[0], wq[1], wq[2], wq[3]);
+        }
       } else if (sb >= 2u && sb != 0xFFu) {
         // the power of two rides on the rounding (e2m1_sr_top_scaled)
         const float half = scale_half(sb), sat = OAS ? 0.0f : scale_six(sb);
@@ -361,15 +386,64 @@ __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
   uint32_t ma = 0, mb = 0;
   if (BF16) {
     const uint32_t* s = reinterpret_cast<const uint32_t*>(tile) + 32 * rg * (kcols / 2) + cp;
-    uint32_t m = 0;
+    uint32_t m = 0, wr[32];  // the column pair's 32 rows, kept for the codes
 #pragma unroll
-    for (int j = 0; j < 32; ++j) m = bf16x2_absmax_nan(m, s[j * (kcols / 2)]);
+    for (int j = 0; j < 32; ++j) {
+      wr[j] = s[j * (kcols / 2)];
+      m = bf16x2_absmax_nan(m, wr[j]);
+    }
     m &= 0x7FFF7FFFu;
     ma = m << 16;
     mb = m & 0xFFFF0000u;
+    if (SR && EVEN && !BIG) {
+      const uint32_t sa = OAS ? scale_byte_oas(ma) : scale_byte(ma);
+      const uint32_t sb = OAS ? scale_byte_oas(mb) : scale_byte(mb);
+      if (sa != 0xFFu && sb != 0xFFu) {
+        // as the bf16 row kernel: one exact mixed-precision product per
+        // value (each column its own 2^-e), packed saturation, the codes of
+        // rows 2k (x4 sum) and 2k+1 (x64 sum) merged into one byte per
+        // column, signs gathered from the rows' words
+        ColPair o;
+        o.sa = sa;
+        o.sb = sb;
+        const unsigned short s16a = bf16_inv_scale(sa), s16b = bf16_inv_scale(sb);
+        const uint32_t sat2 = bitsel(bf16x2_six_scale(sa), bf16x2_six_scale(sb), 0xFFFFu);
+        const int64_t c0 = tile_c + 2 * cp;
+        const uint32_t kp0 =
+            key.k0 + uint32_t((uint64_t(r0) * uint64_t(cols) + uint64_t(c0)) >> 1);
+        const uint32_t hc = uint32_t(uint64_t(cols) >> 1);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pa[4], pb[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint32_t t[2][2];
+#pragma unroll
+            for (int par = 0; par < 2; ++par) {  // row 8q+2k+par
+              const int j = 8 * q + 2 * k + par;
+              uint32_t re, ro;
+              pair_randoms(mix32_pre(mad_u32(uint32_t(j), hc, kp0)), re, ro);
+              const uint32_t ws = OAS ? wr[j] : bf16x2_clamp_abs(wr[j], sat2);
+              const uint32_t mul = par ? 64u : 4u;
+              const uint32_t nm = par ? 0xFFFFF000u : 0xFFFFFF00u;
+              const uint32_t nbase = par ? kSrBase64 : kSrBase4;
+              t[par][0] = mad_u32(sr_operand(bf16lo_mul(ws, s16a)), mul, mad_u32(re, nm, nbase));
+              t[par][1] = mad_u32(sr_operand(bf16hi_mul(ws, s16b)), mul, mad_u32(ro, nm, nbase));
+            }
+            pa[k] = pair_byte(t[1][0], t[0][0]);
+            pb[k] = pair_byte(t[1][1], t[0][1]);
+          }
+          uint32_t ta, tb;
+          sign_nibbles_cols(wr + 8 * q, ta, tb);
+          o.wa[q] = pack_pair_bytes(pa[0], pa[1], pa[2], pa[3]) | ta;
+          o.wb[q] = pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) | tb;
+        }
+        return o;
+      }
+    }
     return column_pair_codes<SR, EVEN, BIG, true, OAS>(
         [&](int j) {
-          const uint32_t w = s[j * (kcols / 2)];
+          const uint32_t w = wr[j];
           return make_float2(bf16_lo(w), bf16_hi(w));
         },
         ma, mb, r0, tile_c + 2 * cp, cols, key);

@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kRhtThreads, 2)
         const uint32_t p0 = uint32_t(pg) + 4 * q;
         uint32_t h[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + p0 + t);
+        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(mad_u32(uint32_t(t), 1u, kh + p0));
         wq[q] = e2m1x8_sr(v, h);
       } else {
         wq[q] = e2m1x8_rn(v);
@@ -255,7 +255,7 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
       const uint32_t p0 = uint32_t(pg) + 4 * q;
       uint32_t h[4];
 #pragma unroll
-      for (int t = 0; t < 4; ++t) h[t] = mix32_pre(kh + p0 + t);
+      for (int t = 0; t < 4; ++t) h[t] = mix32_pre(mad_u32(uint32_t(t), 1u, kh + p0));
       wq[q] = e2m1x8_sr(v, h);
     } else {
       wq[q] = e2m1x8_rn(v);
