@@ -213,6 +213,42 @@ mxfp4_status mxfp4_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                             void* stream);
 
 /*
+ * One iteration of Q-Ramping: oscillation detection in a short tracking
+ * window at the start of each epoch, then k2-times-slower updates for the
+ * weights it flags. Source: "Oscillation-Reduced MXFP4 Training for Vision
+ * Transformers", rebuttal, Weakness 2 (oscillations are tracked only in the
+ * first 30 of about 2500 iterations of an epoch) and the hyper-parameter
+ * answers (oscillation detection factor k1, 16 recommended; weight update
+ * frequency factor k2, 3 to 5, 5 by default). The page gives no formula;
+ * this is the reading the library implements (parity against the page
+ * unpinned). Per element, in fp32 with no fused multiply-add, at iteration
+ * `iter` of the epoch (0-based):
+ *   iter == 0:  if flag: w += acc;  acc = 0; flag = 0;
+ *               w_snap = w; d_w = d_q = 0          (the window starts)
+ *   update:     if flag: acc += delta, and when iter % k2 == k2 - 1:
+ *               w += acc, acc = 0;   else: w += delta
+ *   iter < track_iters (the window), on the updated w:
+ *               d_w += |w - w_snap|; d_q += |DQ(w) - DQ(w_snap)|; w_snap = w
+ *               (DQ = 1x32 RNE quantize-dequantize, as mxfp4_osc_step)
+ *   iter == track_iters - 1 (the window's end):
+ *               flag = d_q > k1 * d_w; d_w = d_q = 0; the number of flagged
+ *               elements is ADDED to *n_flagged (if not NULL).
+ * Outside the window w_snap, d_w and d_q are neither read nor written.
+ *   w, w_snap, d_w, d_q, acc  device fp32 [rows][cols], read and written
+ *   delta                     device fp32 [rows][cols], the iteration's
+ *                             optimizer update (read only)
+ *   flag                      device uint8 [rows][cols] (0 or 1)
+ *   n_flagged                 device, or NULL
+ * cols must be a multiple of 32; every array 16-byte aligned.
+ * MXFP4_ERR_SHAPE also for iter < 0, track_iters < 0 or k2 < 1.
+ */
+mxfp4_status mxfp4_qramp_step(float* w, const float* delta, float* w_snap,
+                              float* d_w, float* d_q, float* acc, uint8_t* flag,
+                              int64_t rows, int64_t cols, int64_t iter,
+                              int64_t track_iters, float k1, int64_t k2,
+                              unsigned long long* n_flagged, void* stream);
+
+/*
  * Synthetic optimizer update that drives the oscillation workload (a stand-in
  * for the AdamW step that the tracker follows; not part of the method):
  * w = w + s * (rel_step * |w|) in fp32 (separate multiply and add), where

@@ -7,7 +7,7 @@ from ._binding import (  # noqa: F401
     BF16, COLS, F32, RNE, ROWS, SR, SYMBOLS, Mxfp4Error, dequantize,
     double_quantize, gemm, lib, mxfp4_dequantize, mxfp4_double_quantize,
     mxfp4_gemm,
-    mxfp4_osc_step, mxfp4_osc_synthetic_update, mxfp4_qema_quantize,
+    mxfp4_osc_step, mxfp4_osc_synthetic_update, mxfp4_qema_quantize, mxfp4_qramp_step,
     mxfp4_quantize, mxfp4_quantize_oas, mxfp4_rht_quantize, mxfp4_scales_to_blocked,
     mxfp4_status_string, osc_step, osc_synthetic_update, qema_quantize,
-    quantize, rht_quantize, scales_to_blocked, status_string)
+    qramp_step, quantize, rht_quantize, scales_to_blocked, status_string)

@@ -22,7 +22,7 @@ RNE, SR = 0, 1
 SYMBOLS = ("mxfp4_quantize", "mxfp4_quantize_oas", "mxfp4_dequantize",
            "mxfp4_double_quantize", "mxfp4_double_quantize_oas",
            "mxfp4_rht_quantize", "mxfp4_rht_quantize_oas", "mxfp4_osc_step",
-           "mxfp4_osc_synthetic_update", "mxfp4_qema_quantize",
+           "mxfp4_osc_synthetic_update", "mxfp4_qramp_step", "mxfp4_qema_quantize",
            "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_status_string")
 
 
@@ -66,6 +66,8 @@ def lib():
                                            ctypes.c_float, vp],
             "mxfp4_qema_quantize": [vp, vp, i64, i64, ctypes.c_float, vp, vp,
                                     vp],
+            "mxfp4_qramp_step": [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                 ctypes.c_float, i64, vp, vp],
             "mxfp4_scales_to_blocked": [vp, i64, i64, vp, vp],
             "mxfp4_gemm": [vp, vp, vp, vp, i64, i64, i64, vp, vp],
         }
@@ -244,6 +246,29 @@ def osc_step(w, w_snap, d_w, d_q, window_end=False, threshold=4.0,
            "mxfp4_osc_step")
 
 
+def qramp_step(w, delta, w_snap, d_w, d_q, acc, flag, it, track_iters=30, k1=16.0,
+               k2=5, n_flagged=None, stream=None):
+    """mxfp4_qramp_step: one Q-Ramping iteration, in place. w, delta,
+    w_snap, d_w, d_q, acc: fp32 CUDA tensors of one shape; flag: uint8 of
+    that shape; n_flagged: optional int64 CUDA tensor of one element."""
+    _cuda2d(w, "w")
+    if w.dtype != torch.float32:
+        raise TypeError("w must be float32")
+    for name, t in (("delta", delta), ("w_snap", w_snap), ("d_w", d_w), ("d_q", d_q),
+                    ("acc", acc)):
+        _buffer(t, name, torch.float32, w.numel(), w.device)
+    _buffer(flag, "flag", torch.uint8, w.numel(), w.device)
+    if n_flagged is not None:
+        _buffer(n_flagged, "n_flagged", torch.int64 if n_flagged.dtype != torch.uint64
+                else torch.uint64, 1, w.device)
+    R, C = w.shape
+    _check(lib().mxfp4_qramp_step(_ptr(w), _ptr(delta), _ptr(w_snap), _ptr(d_w), _ptr(d_q),
+                                  _ptr(acc), _ptr(flag), R, C, int(it), int(track_iters),
+                                  float(k1), int(k2), _ptr(n_flagged),
+                                  _stream(w.device, stream)),
+           "mxfp4_qramp_step")
+
+
 def osc_synthetic_update(w, seed, step, rel_step=1e-4, stream=None):
     """mxfp4_osc_synthetic_update on an fp32 CUDA tensor, in place."""
     _cuda2d(w, "w")
@@ -335,6 +360,7 @@ mxfp4_double_quantize = double_quantize
 mxfp4_rht_quantize = rht_quantize
 mxfp4_osc_step = osc_step
 mxfp4_osc_synthetic_update = osc_synthetic_update
+mxfp4_qramp_step = qramp_step
 mxfp4_qema_quantize = qema_quantize
 mxfp4_scales_to_blocked = scales_to_blocked
 mxfp4_gemm = gemm

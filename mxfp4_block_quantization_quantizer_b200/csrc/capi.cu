@@ -169,6 +169,22 @@ mxfp4_status mxfp4_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                                           n_flagged, as_stream(stream)));
 }
 
+mxfp4_status mxfp4_qramp_step(float* w, const float* delta, float* w_snap,
+                              float* d_w, float* d_q, float* acc, uint8_t* flag,
+                              int64_t rows, int64_t cols, int64_t iter,
+                              int64_t track_iters, float k1, int64_t k2,
+                              unsigned long long* n_flagged, void* stream) {
+  if (!w || !delta || !w_snap || !d_w || !d_q || !acc || !flag) return MXFP4_ERR_NULL;
+  if (!dims_ok(rows, cols) || cols % 32) return MXFP4_ERR_SHAPE;
+  if (iter < 0 || track_iters < 0 || k2 < 1) return MXFP4_ERR_SHAPE;
+  if (!aligned16(w) || !aligned16(delta) || !aligned16(w_snap) || !aligned16(d_w) ||
+      !aligned16(d_q) || !aligned16(acc) || !aligned16(flag))
+    return MXFP4_ERR_ALIGN;
+  return from_cuda(mxfp4::launch_qramp_step(w, delta, w_snap, d_w, d_q, acc, flag, rows,
+                                            cols, iter, track_iters, k1, k2, n_flagged,
+                                            as_stream(stream)));
+}
+
 mxfp4_status mxfp4_osc_synthetic_update(float* w, int64_t rows, int64_t cols,
                                         uint64_t seed, uint32_t step,
                                         float rel_step, void* stream) {

@@ -47,6 +47,12 @@ cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                             float threshold, unsigned long long* n_flagged,
                             cudaStream_t s);
 
+// One Q-Ramping iteration (see mxfp4_qramp_step).
+cudaError_t launch_qramp_step(float* w, const float* delta, float* w_snap, float* d_w,
+                              float* d_q, float* acc, uint8_t* flag, int64_t rows,
+                              int64_t cols, int64_t iter, int64_t track_iters, float k1,
+                              int64_t k2, unsigned long long* n_flagged, cudaStream_t s);
+
 cudaError_t launch_qema_quant(const float* w, float* w_ema, int64_t rows,
                               int64_t cols, float beta, uint8_t* codes,
                               uint8_t* scales, cudaStream_t s);

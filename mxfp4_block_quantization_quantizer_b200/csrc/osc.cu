@@ -108,6 +108,116 @@ __global__ void __launch_bounds__(kOscThreads)
   }
 }
 
+// Q-Ramping ("Oscillation-Reduced MXFP4 Training for Vision Transformers",
+// rebuttal, Weakness 2 and the hyper-parameter answers): one iteration.
+// FLUSH (iteration 0 of an epoch): a flagged weight takes what it still
+// holds, flags clear and the tracking window starts. Then the update: an
+// unflagged weight takes delta at once, a flagged one gathers it and takes
+// the gathered sum when APPLY (iteration % k2 == k2 - 1). TRACK (inside the
+// window): the tracker's accumulation on the updated weight; WEND (the
+// window's last iteration): flag d_q > k1 * d_w, reset the distances. Four
+// threads per 1x32 group (the group maxima of DQ come from quad shuffles);
+// every update is one fp32 operation with explicit rounding.
+template <bool FLUSH, bool TRACK, bool WEND, bool APPLY>
+__global__ void __launch_bounds__(kOscThreads)
+    k_qramp_step(float* __restrict__ w, const float* __restrict__ delta,
+                 float* __restrict__ w_snap, float* __restrict__ d_w,
+                 float* __restrict__ d_q, float* __restrict__ acc,
+                 uint8_t* __restrict__ flag, int64_t n_groups, float k1,
+                 unsigned long long* __restrict__ n_flagged) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 3;
+  const int64_t warp = (int64_t(blockIdx.x) * kOscThreads + threadIdx.x) >> 5;
+  const int64_t chunk = (int64_t(gridDim.x) * kOscThreads) >> 2;
+  const int64_t my = warp * 8 + (lane >> 2);
+  unsigned count = 0;
+  for (int64_t base = 0; base < n_groups; base += chunk) {
+    const int64_t g = base + my;
+    const bool ok = g < n_groups;
+    const int64_t e = (ok ? g : 0) * 32 + sub * 8;
+    float vw[8], dv[8], va[8];
+    load8(w + e, vw);
+    load8(delta + e, dv);
+    load8(acc + e, va);
+    const uint2 f8 = *reinterpret_cast<const uint2*>(flag + e);
+    uint8_t fl[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      fl[j] = uint8_t(f8.x >> (8 * j));
+      fl[4 + j] = uint8_t(f8.y >> (8 * j));
+    }
+    float vs[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (FLUSH) {
+        if (fl[j]) vw[j] = __fadd_rn(vw[j], va[j]);
+        va[j] = 0.0f;
+        fl[j] = 0;
+        vs[j] = vw[j];
+      }
+      if (fl[j]) {
+        va[j] = __fadd_rn(va[j], dv[j]);
+        if (APPLY) {
+          vw[j] = __fadd_rn(vw[j], va[j]);
+          va[j] = 0.0f;
+        }
+      } else {
+        vw[j] = __fadd_rn(vw[j], dv[j]);
+      }
+    }
+    if (TRACK) {
+      float dw[8], dq[8], qw[8], qs[8];
+      if (FLUSH) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dw[j] = dq[j] = 0.0f;
+      } else {
+        load8(w_snap + e, vs);
+        load8(d_w + e, dw);
+        load8(d_q + e, dq);
+      }
+      dq8(vw, qw);
+      dq8(vs, qs);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        dw[j] = __fadd_rn(dw[j], fabsf(__fsub_rn(vw[j], vs[j])));
+        dq[j] = __fadd_rn(dq[j], fabsf(__fsub_rn(qw[j], qs[j])));
+        if (WEND) {
+          fl[j] = dq[j] > __fmul_rn(k1, dw[j]) ? 1 : 0;
+          count += fl[j];
+          dw[j] = dq[j] = 0.0f;
+        }
+      }
+      if (ok) {
+        store8(w_snap + e, vw);
+        store8(d_w + e, dw);
+        store8(d_q + e, dq);
+      }
+    } else if (FLUSH && ok) {
+      const float z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      store8(w_snap + e, vs);  // the window starts from the pre-update
+      store8(d_w + e, z);      // weight, but no window runs
+      store8(d_q + e, z);
+    }
+    if (!ok) continue;
+    store8(w + e, vw);
+    store8(acc + e, va);
+    uint2 o;
+    o.x = uint32_t(fl[0]) | (uint32_t(fl[1]) << 8) | (uint32_t(fl[2]) << 16) | (uint32_t(fl[3]) << 24);
+    o.y = uint32_t(fl[4]) | (uint32_t(fl[5]) << 8) | (uint32_t(fl[6]) << 16) | (uint32_t(fl[7]) << 24);
+    *reinterpret_cast<uint2*>(flag + e) = o;
+  }
+  if (WEND && n_flagged != nullptr) {
+    __shared__ unsigned block_count;
+    if (threadIdx.x == 0) block_count = 0;
+    __syncthreads();
+    count = __reduce_add_sync(0xFFFFFFFFu, count);
+    if (lane == 0 && count) atomicAdd(&block_count, count);
+    __syncthreads();
+    if (threadIdx.x == 0 && block_count)
+      atomicAdd(n_flagged, static_cast<unsigned long long>(block_count));
+  }
+}
+
 // w += s * (rel_step * |w|), s = -1 iff bit 31 of the element's hash is set.
 __global__ void __launch_bounds__(kOscThreads)
     k_osc_update(float* __restrict__ w, int64_t n, RngKey key, float rel_step) {
@@ -157,6 +267,54 @@ cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                                       n_flagged);
   }
   return cudaGetLastError();
+}
+
+template <bool FLUSH, bool TRACK, bool WEND, bool APPLY>
+static cudaError_t qramp_impl(float* w, const float* delta, float* w_snap, float* d_w,
+                              float* d_q, float* acc, uint8_t* flag, int64_t n_groups,
+                              float k1, unsigned long long* n_flagged, cudaStream_t s) {
+  auto kern = k_qramp_step<FLUSH, TRACK, WEND, APPLY>;
+  const int64_t blocks = (n_groups + kOscThreads / 4 - 1) / (kOscThreads / 4);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kOscThreads, 0, blocks);
+  kern<<<grid, kOscThreads, 0, s>>>(w, delta, w_snap, d_w, d_q, acc, flag, n_groups, k1,
+                                    n_flagged);
+  return cudaGetLastError();
+}
+
+template <bool FLUSH, bool TRACK, bool WEND>
+static cudaError_t qramp_apply(bool apply, float* w, const float* delta, float* w_snap,
+                               float* d_w, float* d_q, float* acc, uint8_t* flag,
+                               int64_t n_groups, float k1, unsigned long long* n_flagged,
+                               cudaStream_t s) {
+  return apply ? qramp_impl<FLUSH, TRACK, WEND, true>(w, delta, w_snap, d_w, d_q, acc, flag,
+                                                      n_groups, k1, n_flagged, s)
+               : qramp_impl<FLUSH, TRACK, WEND, false>(w, delta, w_snap, d_w, d_q, acc, flag,
+                                                       n_groups, k1, n_flagged, s);
+}
+
+cudaError_t launch_qramp_step(float* w, const float* delta, float* w_snap, float* d_w,
+                              float* d_q, float* acc, uint8_t* flag, int64_t rows,
+                              int64_t cols, int64_t iter, int64_t track_iters, float k1,
+                              int64_t k2, unsigned long long* n_flagged, cudaStream_t s) {
+  const int64_t n_groups = rows * cols / kGroup;
+  const bool flush = iter == 0, track = iter < track_iters;
+  const bool wend = iter == track_iters - 1, apply = iter % k2 == k2 - 1;
+  if (flush) {
+    if (!track)
+      return qramp_apply<true, false, false>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                             n_groups, k1, n_flagged, s);
+    return wend ? qramp_apply<true, true, true>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                                n_groups, k1, n_flagged, s)
+                : qramp_apply<true, true, false>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                                 n_groups, k1, n_flagged, s);
+  }
+  if (!track)
+    return qramp_apply<false, false, false>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                            n_groups, k1, n_flagged, s);
+  return wend ? qramp_apply<false, true, true>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                               n_groups, k1, n_flagged, s)
+              : qramp_apply<false, true, false>(apply, w, delta, w_snap, d_w, d_q, acc, flag,
+                                                n_groups, k1, n_flagged, s);
 }
 
 cudaError_t launch_osc_update(float* w, int64_t n, uint64_t seed,

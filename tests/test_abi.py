@@ -107,6 +107,13 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_osc_step(P, PODD, P, P, 64, 64, 0, 4.0, NUL, NUL) == ALIGN
     assert L.mxfp4_osc_synthetic_update(NUL, 4, 4, 0, 0, 1e-4, NUL) == NULL
     assert L.mxfp4_osc_synthetic_update(P, 0, 4, 0, 0, 1e-4, NUL) == SHAPE
+    q = (P, P, P, P, P, P, P)
+    assert L.mxfp4_qramp_step(P, P, P, P, P, P, NUL, 64, 64, 0, 30, 16.0, 5, NUL, NUL) == NULL
+    assert L.mxfp4_qramp_step(*q, 64, 48, 0, 30, 16.0, 5, NUL, NUL) == SHAPE
+    assert L.mxfp4_qramp_step(*q, 64, 64, -1, 30, 16.0, 5, NUL, NUL) == SHAPE
+    assert L.mxfp4_qramp_step(*q, 64, 64, 0, -1, 16.0, 5, NUL, NUL) == SHAPE
+    assert L.mxfp4_qramp_step(*q, 64, 64, 0, 30, 16.0, 0, NUL, NUL) == SHAPE
+    assert L.mxfp4_qramp_step(P, P, P, P, P, P, PODD, 64, 64, 0, 30, 16.0, 5, NUL, NUL) == ALIGN
     assert L.mxfp4_qema_quantize(P, NUL, 64, 64, 0.998, P, P, NUL) == NULL
     assert L.mxfp4_qema_quantize(P, P, 64, 48, 0.998, P, P, NUL) == SHAPE
     assert L.mxfp4_qema_quantize(P, PODD, 64, 64, 0.998, P, P, NUL) == ALIGN

@@ -123,7 +123,15 @@ def test_qema_blocked_gemm_and_tracker_reject_bad_buffers(fake):
     with pytest.raises(ValueError):
         B.osc_step(w, w.clone(), w.clone(), w.clone(),
                    n_flagged=torch.zeros(2, dtype=torch.int64))
+    with pytest.raises(ValueError):
+        B.qramp_step(w, w.clone(), w.clone(), w.clone(), w.clone(), w.clone(),
+                     u8(32, 63), 0)
+    with pytest.raises(ValueError):
+        B.qramp_step(w, w.clone()[:, :32], w.clone(), w.clone(), w.clone(), w.clone(),
+                     u8(32, 64), 0)
     assert fake.calls == []
+    B.qramp_step(w, w.clone(), w.clone(), w.clone(), w.clone(), w.clone(), u8(32, 64), 0)
+    fake.calls.clear()
     B.scales_to_blocked(u8(130, 5), out=u8(256, 8))
     B.gemm(a, ab, a, ab, 128, out=torch.zeros((128, 128)))
     assert fake.calls == ["mxfp4_scales_to_blocked", "mxfp4_gemm"]

@@ -453,6 +453,49 @@ def test_osc_mid_window_state():
     assert np.any(odq > 0)
 
 
+def qramp_deltas(w0, n, seed):
+    """Seeded updates of the tracker workload: +-1e-4 |w0| with random signs,
+    and a quarter of the weights alternating sign every iteration (they sit
+    near a rounding edge, so these oscillate)."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    osc = g.random(w0.shape) < 0.25
+    mag = (np.float32(1e-4) * np.abs(w0)).astype(np.float32)
+    out = []
+    for t in range(n):
+        s = np.where(osc, 1.0 if t % 2 == 0 else -1.0,
+                     np.where(g.random(w0.shape) < 0.5, -1.0, 1.0))
+        out.append((s * mag).astype(np.float32))
+    return out
+
+
+@pytest.mark.parametrize("track,k2", [(5, 3), (6, 1), (0, 4)])
+def test_qramp_epochs(track, k2):
+    """Three epochs of 9 iterations: every array bit for bit, and the flag
+    counts, after every iteration."""
+    w_np = W.osc_w(seed=5, rows=64, cols=256)
+    deltas = qramp_deltas(w_np, 27, 11)
+    z = np.zeros_like(w_np)
+    ref = [w_np.copy(), z.copy(), z.copy(), z.copy(), z.copy(), np.zeros(w_np.shape, np.uint8)]
+    dev = [to_dev(a.copy()) for a in ref]
+    nflag = torch.zeros(1, dtype=torch.int64, device="cuda")
+    total = 0
+    for t, d in enumerate(deltas):
+        it = t % 9
+        dd = to_dev(d)
+        m.qramp_step(dev[0], dd, dev[1], dev[2], dev[3], dev[4], dev[5], it,
+                     track_iters=track, k1=16.0, k2=k2, n_flagged=nflag)
+        total += O.qramp_step(ref[0], d, ref[1], ref[2], ref[3], ref[4], ref[5], it,
+                              track_iters=track, k1=16.0, k2=k2)
+        for g, r, name in zip(dev, ref, ("w", "w_snap", "d_w", "d_q", "acc", "flag")):
+            if name == "flag":
+                assert_bits_equal(to_np(g), r, "flag at %d" % t)
+            else:
+                assert_f32_equal_or_both_nan(to_np(g), r, "%s at %d" % (name, t))
+    assert int(nflag.item()) == total
+    if track:
+        assert total > 0
+
+
 def test_osc_update_alone_and_ragged_length():
     g = np.random.Generator(np.random.PCG64(2))
     w_np = g.normal(0, 0.02, size=(7, 13)).astype(np.float32)  # 91 elements
