@@ -43,6 +43,13 @@ BYTES_PER_ELEM = {
     "osc_update": 8,
     "osc_step": 28,
 }
+# ... of which read (the rest is written): the DRAM read counter of a kernel
+# compares with these (a ratio above 1 means re-reads); writes can still sit
+# in L2 when a kernel ends, so the write counter reads low.
+READ_BYTES_PER_ELEM = {
+    "quant_rows_rne": 2, "quant_cols_sr": 2, "double_quant": 2,
+    "dequant_rows": 0.5 + 1 / 32, "rht_quant_sr": 2, "osc_update": 4, "osc_step": 16,
+}
 OP_ELEMS = {k: SWEEP[0] * SWEEP[1] for k in BYTES_PER_ELEM}
 OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
 
@@ -107,8 +114,9 @@ def kernel_source_digest(op):
 
 
 def measured_traffic(op):
-    """ncu dram read+write bytes per full launch of op, from
-    profiles/dram_traffic.txt, or None when the kernels changed since."""
+    """(dram read bytes, dram write bytes) of one full-size launch of op from
+    profiles/dram_traffic.txt (an ncu capture of that launch), or None when
+    the op's kernel sources changed since the capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     try:
         lines = open(path).read().splitlines()
@@ -117,8 +125,8 @@ def measured_traffic(op):
     digest = kernel_source_digest(op)
     for line in lines:
         parts = line.split()
-        if len(parts) >= 3 and parts[0] == op and parts[2] == "src=" + digest:
-            return float(parts[1])
+        if len(parts) >= 4 and parts[0] == op and parts[3] == "src=" + digest:
+            return float(parts[1]), float(parts[2])
     return None
 
 
@@ -565,6 +573,40 @@ def run_ours(args):
                               "shape": [R, C], "launches": args.steps}
         del oout, dout
 
+        # the tracker's window-end step (flag, snap, reset: k_osc_step with
+        # the window end) on the tracker workload, on copies of its state
+        ow, ows = buf0["w"].clone(), ws.clone()
+        odw, odq = dwt.clone(), dqt.clone()
+        nfl = torch.zeros(1, dtype=torch.int64, device=dev)
+        d = timed_alone(lambda: m.osc_step(ow, ows, odw, odq, window_end=True, n_flagged=nfl))
+        nbytes = (BYTES_PER_ELEM["osc_step"] + 4) * OSC[0] * OSC[1]  # w is written too
+        next_ops["osc_step_window_end"] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9,
+                                           "bytes": nbytes, "shape": list(OSC),
+                                           "launches": args.steps}
+        # Q-Ramping on the tracker workload: an iteration inside the tracking
+        # window (46 B/element) and one outside it (22 B/element)
+        qd = (ow * 1e-4).contiguous()
+        qacc = torch.zeros_like(ow)
+        qfl = torch.zeros(OSC, dtype=torch.uint8, device=dev)
+        for name, it, per in (("qramp_step_tracking", 5, 46), ("qramp_step", 35, 22)):
+            d = timed_alone(lambda: m.qramp_step(ow, qd, ows, odw, odq, qacc, qfl, it,
+                                                 track_iters=30, k1=16.0, k2=5))
+            nbytes = per * OSC[0] * OSC[1]
+            next_ops[name] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9, "bytes": nbytes,
+                              "shape": list(OSC), "launches": args.steps}
+        del ow, ows, odw, odq, nfl, qd, qacc, qfl
+        # the rotation of fp32 inputs (the in-register butterfly kernel) on
+        # the fp32 master weight, rounding SR
+        fR, fC = NEXT_OPS["qema_quant"][1]
+        fw = torch.from_numpy(W.master_w(seed=7 + rank, rows=fR, cols=fC)).to(dev)
+        fout = (u8(fR, fC // 2), u8(fR, fC // 32), None)
+        d = timed_alone(lambda: m.rht_quantize(fw, 2, m.SR, SEED, out=fout))
+        nbytes = (4 + 0.5 + 1 / 32) * fR * fC
+        next_ops["rht_quant_sr_f32"] = {"us": d * 1e6, "GB_s": nbytes / d / 1e9,
+                                        "bytes": nbytes, "shape": [fR, fC],
+                                        "launches": args.steps}
+        del fw, fout
+
         # MXFP4 GEMM on the block-scaled tensor cores, consuming the step's
         # ROWS codes of the sweep as the activation operand
         gM, gN, gK = NEXT_OPS["gemm_mxf4"][1]
@@ -672,7 +714,10 @@ def run_ours(args):
         dom = max(per_op, key=lambda k: per_op[k]["us"])
         step_s = elapsed_ms * 1e-3 / args.steps
         value = job_gbs(world, STEP_BYTES, args.steps, elapsed_ms)
-        traffic = measured_traffic(dom)
+        measured = measured_traffic(dom)
+        traffic = None if measured is None else measured[0] + measured[1]
+        read_ratio = (None if measured is None else
+                      measured[0] / (READ_BYTES_PER_ELEM[dom] * OP_ELEMS[dom]))
         line = {
             "metric": "MXFP4 quantize GB/s (bytes in+out)",
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -685,7 +730,8 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "kernel": dom,
                          "achieved": per_op[dom]["GB_s"], "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": per_op[dom]["frac"], "traffic": traffic},
+                         "frac": per_op[dom]["frac"], "traffic": traffic,
+                         "dram_read_over_alg_read": read_ratio},
             "ops": per_op,
             "e2e": {"value": job_gbs(world, STEP_BYTES, args.e2e_steps, e2e_ms),
                     "unit": "GB/s", "h2d_bytes_per_step": h2d,
