@@ -409,6 +409,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return d;
 }
 
+// Shared-state-space address of a generic pointer into shared memory.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
 // 16-byte load of read-once data: no L1 allocation.
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
@@ -580,6 +585,30 @@ __device__ __forceinline__ void sign_nibbles_cols(const uint32_t* w, uint32_t& t
 __device__ __forceinline__ void pair_randoms(uint32_t g, uint32_t& r_even, uint32_t& r_odd) {
   r_odd = g >> 16;
   r_even = (g ^ r_odd) & 0xFFFFu;
+}
+
+// f16 halves as fp32 by an exact mixed-precision product with one (f16 1.0)
+// on the FMA pipe.
+__device__ __forceinline__ float f16lo_f32(uint32_t h, unsigned short one) {
+  float d;
+  asm("{.reg .b16 l, u; mov.b32 {l, u}, %1;\n\t"
+      "fma.rn.f32.f16 %0, l, %2, %3;}" : "=f"(d) : "r"(h), "h"(one), "f"(-0.0f));
+  return d;
+}
+__device__ __forceinline__ float f16hi_f32(uint32_t h, unsigned short one) {
+  float d;
+  asm("{.reg .b16 l, u; mov.b32 {l, u}, %1;\n\t"
+      "fma.rn.f32.f16 %0, u, %2, %3;}" : "=f"(d) : "r"(h), "h"(one), "f"(-0.0f));
+  return d;
+}
+// The 4 bytes of w as 4 f16x2 words of E2M1 values (byte i's low nibble in
+// the low half of h[i]). Decode only words loaded from memory (see
+// e2m1x8_decode).
+__device__ __forceinline__ void e2m1x4_decode_rows(uint32_t w, uint32_t* h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(w));
 }
 
 constexpr uint32_t kNaNbf16x2 = 0x7FC07FC0u;

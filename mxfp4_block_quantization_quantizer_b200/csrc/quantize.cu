@@ -371,6 +371,55 @@ __device__ __forceinline__ void store_staged_columns(
   }
 }
 
+// Stochastic 32x1 codes of two adjacent columns from their 32 row words
+// wr[j] (bf16 pairs, the even column in the low half), the columns' scale
+// bytes sa, sb (not 0xFF) and the pair counter of row 0, kp0 (key.k0 plus
+// the pair index; row j adds j * hc), for tensors below 2^33 elements. As
+// the bf16 row kernel: one exact mixed-precision product per value (each
+// column its own power of two), saturation on the packed pairs when SAT,
+// the codes of rows 2k (x4 sum) and 2k+1 (x64 sum) merged into one byte per
+// column, signs gathered from the row words. HELD: the words hold half of
+// the values (the double quantizer's Q_D(X) / 2), so the power of two is
+// 2^(1-e) and sa, sb must be at least 1.
+template <bool SAT, bool HELD>
+__device__ __forceinline__ ColPair column_pair_sr_bf16(const uint32_t* wr, uint32_t sa,
+                                                       uint32_t sb, uint32_t kp0,
+                                                       uint32_t hc) {
+  ColPair o;
+  o.sa = sa;
+  o.sb = sb;
+  const unsigned short s16a = bf16_inv_scale(HELD ? sa - 1u : sa);
+  const unsigned short s16b = bf16_inv_scale(HELD ? sb - 1u : sb);
+  const uint32_t sat2 = SAT ? bitsel(bf16x2_six_scale(sa), bf16x2_six_scale(sb), 0xFFFFu) : 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t pa[4], pb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t t[2][2];
+#pragma unroll
+      for (int par = 0; par < 2; ++par) {  // row 8q+2k+par
+        const int j = 8 * q + 2 * k + par;
+        uint32_t re, ro;
+        pair_randoms(mix32_pre(mad_u32(uint32_t(j), hc, kp0)), re, ro);
+        const uint32_t ws = SAT ? bf16x2_clamp_abs(wr[j], sat2) : wr[j];
+        const uint32_t mul = par ? 64u : 4u;
+        const uint32_t nm = par ? 0xFFFFF000u : 0xFFFFFF00u;
+        const uint32_t nbase = par ? kSrBase64 : kSrBase4;
+        t[par][0] = mad_u32(sr_operand(bf16lo_mul(ws, s16a)), mul, mad_u32(re, nm, nbase));
+        t[par][1] = mad_u32(sr_operand(bf16hi_mul(ws, s16b)), mul, mad_u32(ro, nm, nbase));
+      }
+      pa[k] = pair_byte(t[1][0], t[0][0]);
+      pb[k] = pair_byte(t[1][1], t[0][1]);
+    }
+    uint32_t ta, tb;
+    sign_nibbles_cols(wr + 8 * q, ta, tb);
+    o.wa[q] = pack_pair_bytes(pa[0], pa[1], pa[2], pa[3]) | ta;
+    o.wb[q] = pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) | tb;
+  }
+  return o;
+}
+
 // Column pass over a staged tile: thread (rg, cp) quantizes the columns
 // 2cp, 2cp+1 over tile rows 32rg .. 32rg+31 (rows below the tensor's end:
 // the caller checks tile_r + 32rg < rows). The tile is read twice (maxima,
@@ -399,46 +448,11 @@ __device__ __forceinline__ ColPair column_tile_pass(const uint4* tile,
       const uint32_t sa = OAS ? scale_byte_oas(ma) : scale_byte(ma);
       const uint32_t sb = OAS ? scale_byte_oas(mb) : scale_byte(mb);
       if (sa != 0xFFu && sb != 0xFFu) {
-        // as the bf16 row kernel: one exact mixed-precision product per
-        // value (each column its own 2^-e), packed saturation, the codes of
-        // rows 2k (x4 sum) and 2k+1 (x64 sum) merged into one byte per
-        // column, signs gathered from the rows' words
-        ColPair o;
-        o.sa = sa;
-        o.sb = sb;
-        const unsigned short s16a = bf16_inv_scale(sa), s16b = bf16_inv_scale(sb);
-        const uint32_t sat2 = bitsel(bf16x2_six_scale(sa), bf16x2_six_scale(sb), 0xFFFFu);
         const int64_t c0 = tile_c + 2 * cp;
-        const uint32_t kp0 =
-            key.k0 + uint32_t((uint64_t(r0) * uint64_t(cols) + uint64_t(c0)) >> 1);
-        const uint32_t hc = uint32_t(uint64_t(cols) >> 1);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t pa[4], pb[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            uint32_t t[2][2];
-#pragma unroll
-            for (int par = 0; par < 2; ++par) {  // row 8q+2k+par
-              const int j = 8 * q + 2 * k + par;
-              uint32_t re, ro;
-              pair_randoms(mix32_pre(mad_u32(uint32_t(j), hc, kp0)), re, ro);
-              const uint32_t ws = OAS ? wr[j] : bf16x2_clamp_abs(wr[j], sat2);
-              const uint32_t mul = par ? 64u : 4u;
-              const uint32_t nm = par ? 0xFFFFF000u : 0xFFFFFF00u;
-              const uint32_t nbase = par ? kSrBase64 : kSrBase4;
-              t[par][0] = mad_u32(sr_operand(bf16lo_mul(ws, s16a)), mul, mad_u32(re, nm, nbase));
-              t[par][1] = mad_u32(sr_operand(bf16hi_mul(ws, s16b)), mul, mad_u32(ro, nm, nbase));
-            }
-            pa[k] = pair_byte(t[1][0], t[0][0]);
-            pb[k] = pair_byte(t[1][1], t[0][1]);
-          }
-          uint32_t ta, tb;
-          sign_nibbles_cols(wr + 8 * q, ta, tb);
-          o.wa[q] = pack_pair_bytes(pa[0], pa[1], pa[2], pa[3]) | ta;
-          o.wb[q] = pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) | tb;
-        }
-        return o;
+        return column_pair_sr_bf16<!OAS, false>(
+            wr, sa, sb,
+            key.k0 + uint32_t((uint64_t(r0) * uint64_t(cols) + uint64_t(c0)) >> 1),
+            uint32_t(uint64_t(cols) >> 1));
       }
     }
     return column_pair_codes<SR, EVEN, BIG, true, OAS>(
@@ -980,6 +994,154 @@ __global__ void __launch_bounds__(kDqThreads, 3)
   }
 }
 
+// Fused double quantization of bf16 X, second form. The row pass writes,
+// in place of each 1x32 group it read from the staged tile, the group's
+// Q_D(X) / 2 as bf16 (exact: a decoded value has two significant bits and
+// an exponent of at least -130), decoded from the codes it stores (through
+// shared memory: codes are only decoded from memory). The column pass then
+// runs the bf16 column kernel's stochastic rounding on those words (no
+// saturation: a decoded value never scales past 6). X is read once.
+constexpr int kDq3StageBytes = ColStage<kDqCols>::kBytes;
+
+template <bool OAS>
+__device__ __forceinline__ void dq3_row_group(uint4* row, int g, int tr, bool ok,
+                                              uint8_t* __restrict__ rc,
+                                              uint8_t* __restrict__ rs, uint4* s_code) {
+  uint32_t w[16];
+  const int sw = dq_swizzle(g, tr);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 q = row[4 * g + (c ^ sw)];
+    w[4 * c] = q.x, w[4 * c + 1] = q.y, w[4 * c + 2] = q.z, w[4 * c + 3] = q.w;
+  }
+  uint32_t m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = bf16x2_absmax_nan(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+  for (int n = 4; n >= 1; n /= 2)
+#pragma unroll
+    for (int i = 0; i < n; ++i) m[i] = bf16x2_absmax_nan(m[i], m[i + n]);
+  const uint32_t mm = m[0] & 0x7FFF7FFFu;
+  const uint32_t amax = max(mm << 16, mm & 0xFFFF0000u);
+  const uint32_t sb = OAS ? scale_byte_oas(amax) : scale_byte(amax);
+  const unsigned short s16 = bf16_inv_scale(min(sb, 253u));
+  uint32_t word[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = bf16lo_mul(w[4 * c + j], s16);
+      v[2 * j + 1] = bf16hi_mul(w[4 * c + j], s16);
+    }
+    word[c] = sb == 0xFFu ? 0u : e2m1x8_rn(v);
+  }
+  const uint4 out = make_uint4(word[0], word[1], word[2], word[3]);
+  if (ok) {
+    *reinterpret_cast<uint4*>(rc) = out;
+    *rs = uint8_t(sb);
+  }
+  // decode from shared memory: Q_D(X) / 2 = G[m] 2^(e-1) (a group of scale
+  // 0xFF has codes 0 and the value +inf: it decodes to NaN)
+  *s_code = out;
+  uint32_t wb[4];  // a load the compiler cannot replace by the stored registers
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(wb[0]), "=r"(wb[1]), "=r"(wb[2]), "=r"(wb[3])
+               : "r"(smem_addr(s_code))
+               : "memory");
+  const float sv = half_scale_value(sb);
+  const unsigned short one = 0x3C00;  // 1.0 as f16
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t h[4];
+    e2m1x4_decode_rows(wb[c], h);  // elements 8c+2i, 8c+2i+1 in h[i]
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = prmt(__float_as_uint(f16lo_f32(h[i], one) * sv),
+                  __float_as_uint(f16hi_f32(h[i], one) * sv), 0x7632u);
+    row[4 * g + (c ^ sw)] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <bool OAS>
+__global__ void __launch_bounds__(kDqThreads, 3)
+    k_double_quant_pipe3(const void* __restrict__ x, int64_t rows, int64_t cols,
+                         RngKey key, uint8_t* __restrict__ row_codes,
+                         uint8_t* __restrict__ row_scales,
+                         uint8_t* __restrict__ col_codes,
+                         uint8_t* __restrict__ col_scales) {
+  constexpr int kChunks = kTileRows * (kDqCols / 8);
+  extern __shared__ uint4 smem[];  // two raw tiles, then the codes / column stage
+  uint4* s_codes = smem + 2 * kChunks;
+  uint4* s_col = s_codes;  // the column stage reuses the codes' space
+  uint8_t* s_sc = reinterpret_cast<uint8_t*>(s_col + ColStage<kDqCols>::kChunks);
+  const int64_t tiles_c = (cols + kDqCols - 1) / kDqCols;
+  const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) * tiles_c;
+  const int g = threadIdx.x & 3, tr = threadIdx.x >> 2;    // row pass
+  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;  // column pass
+  // the column pass's word offsets within a row (the chunk slot depends on
+  // the row's parity through the staging swizzle)
+  const int chunk = cp >> 2, cg = chunk >> 2;
+  const int off_even = ((chunk ^ dq_swizzle(cg, 0)) << 2) + (cp & 3);
+  const int off_odd = ((chunk ^ dq_swizzle(cg, 1)) << 2) + (cp & 3);
+  const uint32_t hc = uint32_t(uint64_t(cols) >> 1);
+  int64_t t = blockIdx.x;
+  if (t >= n_tiles) return;
+  TileWalk cur(t, gridDim.x, tiles_c), nxt = cur;
+  nxt.next();
+  stage_tile_async<true, true>(x, rows, cols, cur.r * kTileRows, cur.c * kDqCols, smem);
+  for (int buf = 0; t < n_tiles; t += gridDim.x, buf ^= 1, cur = nxt, nxt.next()) {
+    cp_async_wait<0>();
+    __syncthreads();
+    if (t + gridDim.x < n_tiles)
+      stage_tile_async<true, true>(x, rows, cols, nxt.r * kTileRows, nxt.c * kDqCols,
+                                   smem + (buf ^ 1) * kChunks);
+    const int64_t tile_r = cur.r * kTileRows;
+    const int64_t tile_c = cur.c * kDqCols;
+    uint4* raw = smem + buf * kChunks;
+    uint8_t* rc = row_codes + (tile_r + tr) * (cols / 2) + (tile_c + 32 * g) / 2;
+    uint8_t* rs = row_scales + (tile_r + tr) * (cols / 32) + (tile_c + 32 * g) / 32;
+    const bool g_ok = tile_c + 32 * g < cols;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int r = tr + 64 * k;
+      dq3_row_group<OAS>(raw + r * (kDqCols / 8), g, r, g_ok && tile_r + r < rows,
+                         rc + k * 64 * (cols / 2), rs + k * 64 * (cols / 32),
+                         s_codes + r * (kDqCols / 32) + g);
+    }
+    __syncthreads();
+    if (tile_r + 32 * rg < rows) {
+      const uint32_t* s = reinterpret_cast<const uint32_t*>(raw) + 32 * rg * (kDqCols / 2);
+      uint32_t m = 0, wr[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        wr[j] = s[j * (kDqCols / 2) + ((j & 1) ? off_odd : off_even)];
+        m = bf16x2_absmax_nan(m, wr[j]);
+      }
+      m &= 0x7FFF7FFFu;
+      const uint32_t ma = m << 16, mb = m & 0xFFFF0000u;
+      const uint32_t sa = OAS ? scale_byte_oas_of_double(ma) : scale_byte_of_double(ma);
+      const uint32_t sb = OAS ? scale_byte_oas_of_double(mb) : scale_byte_of_double(mb);
+      const int64_t r0 = tile_r + 32 * rg, c0 = tile_c + 2 * cp;
+      ColPair o;
+      if (sa >= 1u && sb >= 1u && sa != 0xFFu && sb != 0xFFu) {
+        o = column_pair_sr_bf16<false, true>(
+            wr, sa, sb,
+            key.k0 + uint32_t((uint64_t(r0) * uint64_t(cols) + uint64_t(c0)) >> 1), hc);
+      } else {
+        o = column_pair_codes<true, true, false, false, OAS, true>(
+            [&](int j) { return make_float2(bf16_lo(wr[j]), bf16_hi(wr[j])); }, ma, mb, r0,
+            c0, cols, key);
+      }
+      stage_column_pair(o, cp, rg, s_col, s_sc);
+    }
+    __syncthreads();
+    store_staged_columns<kDqCols, kDqThreads>(s_col, s_sc, tile_r, tile_c,
+                                              rows, cols, col_codes, col_scales);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -1128,6 +1290,20 @@ static cudaError_t double_quant_impl(const void* x, bool bf16, int64_t rows,
   const int64_t n_tiles = ((rows + kTileRows - 1) / kTileRows) *
                           ((cols + kDqCols - 1) / kDqCols);
   const bool big = big_tensor(rows, cols);
+  if (bf16 && !big) {
+    auto kern = k_double_quant_pipe3<OAS>;
+    constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) + kDq3StageBytes;
+    static_assert(kDq3StageBytes >= kTileRows * (kDqCols / 8) * 4, "codes fit the stage");
+    cudaError_t e = cudaFuncSetAttribute(
+        reinterpret_cast<const void*>(kern),
+        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern),
+                                     kDqThreads, smem, n_tiles);
+    kern<<<grid, kDqThreads, smem, s>>>(x, rows, cols, key, row_codes,
+                                        row_scales, col_codes, col_scales);
+    return cudaGetLastError();
+  }
   if (bf16) {
     auto kern = big ? k_double_quant_pipe<true, OAS> : k_double_quant_pipe<false, OAS>;
     constexpr size_t smem = 2 * kTileRows * (kDqCols / 8) * sizeof(uint4) +
