@@ -52,16 +52,23 @@ READ_BYTES_PER_ELEM = {
 }
 OP_ELEMS = {k: SWEEP[0] * SWEEP[1] for k in BYTES_PER_ELEM}
 OP_ELEMS["osc_update"] = OP_ELEMS["osc_step"] = OSC[0] * OSC[1]
+# Kernels outside the step that --only can still run inside it, alone, for
+# a profiler capture (rows SR quantization of the sweep).
+PROFILE_ONLY_OPS = {"quant_rows_sr": 2 + 0.5 + 1 / 32}
 
 
 # Further operations built beyond the step (Q-EMA), timed on their own.
 NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336)),
             # Y = Q_D(X) Q_D(W)^T: X the sweep, W a second 8192-row tensor
-            "gemm_mxf4": (None, (8192, 8192, 28672))}
+            "gemm_mxf4": (None, (8192, 8192, 28672)),
+            # the same with X quantized in the GEMM's load stage, against
+            # quantize + blocked scales + GEMM, for W's first N rows
+            "gemm_quant_a": (None, (256, 1024, 8192))}
 
 
 def alg_bytes(op):
-    return BYTES_PER_ELEM[op] * OP_ELEMS[op]
+    per = BYTES_PER_ELEM[op] if op in BYTES_PER_ELEM else PROFILE_ONLY_OPS[op]
+    return per * OP_ELEMS.get(op, SWEEP[0] * SWEEP[1])
 
 
 STEP_BYTES = sum(alg_bytes(op) for op in BYTES_PER_ELEM)
@@ -165,6 +172,9 @@ def parse_args():
     ap.add_argument("--gemm", default="",
                     help="M,N,K: time only the MXFP4 GEMM at that shape "
                          "(profiling); prints one line")
+    ap.add_argument("--gemm-fused", action="store_true",
+                    help="with --gemm: the GEMM that quantizes bf16 A in its "
+                         "load stage (mxfp4_gemm_quantize_a)")
     return ap.parse_args()
 
 
@@ -180,24 +190,31 @@ def run_gemm_only(args):
     M, N, K = (int(v) for v in args.gemm.split(","))
     dev = torch.device("cuda", 0)
     to = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
-    ac, as_ = m.quantize(to(W.normal_bf16(M, K, 11)), m.ROWS, m.RNE)
+    xa = to(W.normal_bf16(M, K, 11))
+    ac, as_ = m.quantize(xa, m.ROWS, m.RNE)
     bc, bs = m.quantize(to(W.normal_bf16(N, K, 12)), m.ROWS, m.RNE)
     ab, bb = m.scales_to_blocked(as_), m.scales_to_blocked(bs)
     out = torch.empty(M, N, dtype=torch.float32, device=dev)
+    if args.gemm_fused:
+        run = lambda: m.gemm_quantize_a(xa, bc, bb, out=out)  # noqa: E731
+    else:
+        run = lambda: m.gemm(ac, ab, bc, bb, K, out=out)  # noqa: E731
     for _ in range(args.warmup):
-        m.gemm(ac, ab, bc, bb, K, out=out)
+        run()
     evs = []
     for _ in range(args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        m.gemm(ac, ab, bc, bb, K, out=out)
+        run()
         b.record()
         evs.append((a, b))
     torch.cuda.synchronize(dev)
     d = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e-3
     peak, kind = measured_fp4_peak()
     tf = 2.0 * M * N * K / d / 1e12
-    print(json.dumps({"profile_run": True, "op": "gemm_mxf4", "shape": [M, N, K],
+    print(json.dumps({"profile_run": True,
+                      "op": "gemm_quant_a" if args.gemm_fused else "gemm_mxf4",
+                      "shape": [M, N, K],
                       "us": d * 1e6, "TFLOP_s": tf, "frac": tf / peak,
                       "peak_kind": kind}), flush=True)
 
@@ -453,6 +470,7 @@ def run_ours(args):
     ws, dwt, dqt = buf0["w"].clone(), torch.zeros_like(buf0["w"]), torch.zeros_like(buf0["w"])
 
     ops = [o for o in BYTES_PER_ELEM if not args.only or o in args.only.split(",")]
+    ops += [o for o in PROFILE_ONLY_OPS if o in args.only.split(",")]
     if (R, C) != SWEEP:
         for o in ops:
             if o not in ("osc_update", "osc_step"):
@@ -481,6 +499,7 @@ def run_ours(args):
 
         x, w = b["x"], b["w"]
         timed("quant_rows_rne", lambda: m.quantize(x, m.ROWS, m.RNE, 0, out=b["rows"]))
+        timed("quant_rows_sr", lambda: m.quantize(x, m.ROWS, m.SR, SEED, out=b["rows"]))
         timed("quant_cols_sr", lambda: m.quantize(x, m.COLS, m.SR, SEED, out=b["cols"]))
         timed("double_quant", lambda: m.double_quantize(x, SEED, out=b["dq"]))
         timed("dequant_rows", lambda: m.dequantize(b["rows"][0], b["rows"][1], R, C, out=b["y"]))
@@ -637,6 +656,30 @@ def run_ours(args):
                                      "launches": args.steps, "peak_TFLOP_s": peak,
                                      "peak_kind": kind,
                                      "frac": flops / d / 1e12 / peak}
+            # the activation quantized inside the GEMM (one launch) against
+            # quantize + blocked scales + GEMM (three), for W's first N rows
+            qout = (u8(gM, gK // 2), u8(gM, gK // 32))
+            qblk = u8(-(-gM // 128) * 128, -(-(gK // 32) // 4) * 4)
+            for nn in NEXT_OPS["gemm_quant_a"][1]:
+                bcn = bc[:nn]
+                bbn = m.scales_to_blocked(bs[:nn])
+                outn = torch.empty(gM, nn, dtype=torch.float32, device=dev)
+                d_fused = timed_alone(lambda: m.gemm_quantize_a(buf0["x"], bcn, bbn, out=outn))
+
+                def two_step():
+                    m.quantize(buf0["x"], m.ROWS, m.RNE, out=qout)
+                    m.scales_to_blocked(qout[1], out=qblk)
+                    m.gemm(qout[0], qblk, bcn, bbn, gK, out=outn)
+                d_two = timed_alone(two_step)
+                flops = 2.0 * gM * nn * gK
+                next_ops["gemm_quant_a_n%d" % nn] = {
+                    "us": d_fused * 1e6, "two_step_us": d_two * 1e6,
+                    "speedup_vs_two_step": d_two / d_fused,
+                    "TFLOP_s": flops / d_fused / 1e12, "shape": [gM, nn, gK],
+                    "launches": args.steps,
+                    "x_read_GB_s": 2.0 * gM * gK / d_fused / 1e9}
+                del bcn, bbn, outn
+            del qout, qblk
             del ac, as_, bc, bs, ab, bb, gout
 
     # end to end: pinned host input -> device -> kernels -> host results

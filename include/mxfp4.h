@@ -63,7 +63,8 @@ typedef enum mxfp4_status {
   MXFP4_ERR_NULL = 1,  /* a required pointer is NULL */
   MXFP4_ERR_SHAPE = 2, /* rows or cols <= 0, a group axis that is not a
                           multiple of 32, or a size past the stated limit */
-  MXFP4_ERR_ALIGN = 3, /* a tensor pointer is not 16-byte aligned */
+  MXFP4_ERR_ALIGN = 3, /* a tensor pointer is not 16-byte aligned (a
+                          status word: not 4-byte aligned) */
   MXFP4_ERR_ENUM = 4,  /* dtype, axis or rounding out of range */
   MXFP4_ERR_CUDA = 5   /* the launch failed (cudaGetLastError); faults of a
                           kernel that launched surface on the stream */
@@ -76,6 +77,22 @@ typedef enum mxfp4_rounding { MXFP4_RNE = 0, MXFP4_SR = 1 } mxfp4_rounding;
 /* Largest rows and largest cols accepted (each); rows*cols must also stay
  * below 2^46 elements. */
 #define MXFP4_MAX_DIM ((int64_t)1 << 31)
+
+/*
+ * Device status word of the tensor-core entry points (mxfp4_rht_quantize,
+ * mxfp4_rht_quantize_oas, mxfp4_gemm, mxfp4_gemm_quantize_a). Their kernels wait on mbarriers for
+ * copies and tensor-core work inside the CTA; every such wait is bounded.
+ * When one runs out, the CTA stops waiting, lets its own copies and MMAs in
+ * flight finish (again with bounded waits), frees its tensor memory, writes
+ * the poison values the entry point states for the tiles it did not
+ * complete, and ORs MXFP4_STATUS_WAIT_TIMEOUT into the caller's status word
+ * (an int in device memory, 4-byte aligned; NULL: not reported). The bit is
+ * never cleared by the library: zero the word before the call and read it
+ * once the stream has passed the call. A set bit means the outputs are
+ * incomplete; it does not mean the CUDA context is damaged. The paper has no
+ * counterpart: this is the library's own error channel.
+ */
+#define MXFP4_STATUS_WAIT_TIMEOUT 1
 
 /*
  * Block quantize X [rows, cols] (bf16 or fp32) into MXFP4 codes and E8M0
@@ -173,12 +190,16 @@ mxfp4_status mxfp4_double_quantize_oas(const void* x, int dtype, int64_t rows,
  *   x        device, [rows][cols] of dtype; cols a multiple of 32
  *   codes, scales  device, ROWS layout
  *   rotated  device fp32 [rows][cols] receiving y, or NULL to skip it
+ *   status   device int or NULL (MXFP4_STATUS_WAIT_TIMEOUT above); bf16
+ *            inputs only (the fp32 path never waits). A group whose
+ *            rotation was not read out gets scale byte 0xFF, zero codes and
+ *            NaN in `rotated`.
  */
 mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
                                 int64_t cols, uint64_t sign_seed,
                                 int rounding, uint64_t sr_seed,
                                 uint8_t* codes, uint8_t* scales,
-                                float* rotated, void* stream);
+                                float* rotated, int* status, void* stream);
 
 /*
  * mxfp4_rht_quantize with the overflow-aware scale (as mxfp4_quantize_oas)
@@ -188,7 +209,7 @@ mxfp4_status mxfp4_rht_quantize_oas(const void* x, int dtype, int64_t rows,
                                     int64_t cols, uint64_t sign_seed,
                                     int rounding, uint64_t sr_seed,
                                     uint8_t* codes, uint8_t* scales,
-                                    float* rotated, void* stream);
+                                    float* rotated, int* status, void* stream);
 
 /*
  * One step of the weight-oscillation tracker on fp32 master weights w.
@@ -320,15 +341,44 @@ mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
  *             aligned
  *   b_codes, b_scales  the same for B with n rows
  *   c         device fp32 [m][n], written (every element)
+ *   status    device int or NULL (MXFP4_STATUS_WAIT_TIMEOUT above)
  * k must be a multiple of 32; m, n, k > 0 within the size limit. The result
  * equals the exact sum of the products up to fp32 accumulation rounding (the
- * order of the additions is the hardware's). A tile whose tensor-core work
- * does not complete within a bounded wait is written as NaN.
+ * order of the additions is the hardware's). When a bounded wait runs out,
+ * the tile it served and the CTA's later tiles are written as NaN.
  */
 mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                         const uint8_t* b_codes, const uint8_t* b_scales,
                         int64_t m, int64_t n, int64_t k, float* c,
-                        void* stream);
+                        int* status, void* stream);
+
+/*
+ * Forward GEMM with the activation quantized in the GEMM's load stage:
+ *   C[m][n] = sum_k Q_D(X)[m][k] * B[n][k]      (fp32 accumulate, fp32 out)
+ * Q_D(X) is the 1x32 nearest-even quantization of X along k (ROWS), the
+ * one mxfp4_quantize(x, MXFP4_BF16, m, k, MXFP4_ROWS, MXFP4_RNE, ...)
+ * computes; B is given as in mxfp4_gemm (the pre-quantized weight). The
+ * result equals that quantization followed by mxfp4_scales_to_blocked and
+ * mxfp4_gemm, bit for bit, but Q_D(X) never passes through global memory:
+ * bf16 X tiles are quantized in shared memory into the tensor cores'
+ * operand layout. Source: "Oscillation-Reduced MXFP4 Training for Vision
+ * Transformers", rebuttal Question 2 (the forward GEMM Q_D(X) Q_D(W)^T).
+ *   x         device bf16 [m][k], 16-byte aligned, read only
+ *   b_codes, b_scales  as in mxfp4_gemm, n rows
+ *   c         device fp32 [m][n], written (every element)
+ *   a_codes   device [m][k/2], 16-byte aligned, or NULL: receives the codes
+ *             of Q_D(X) in the ROWS layout
+ *   a_scales  device [m][k/32], or NULL; given exactly when a_codes is
+ *   status    device int or NULL, as in mxfp4_gemm
+ * k must be a multiple of 256; m, n > 0 within the size limit. X is read
+ * and quantized once per 256 columns of C (tiles that run together share
+ * it through L2), so the fusion pays where n is small; for large n the
+ * separate quantize + mxfp4_gemm is faster.
+ */
+mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t k,
+                                   const uint8_t* b_codes, const uint8_t* b_scales,
+                                   float* c, uint8_t* a_codes, uint8_t* a_scales,
+                                   int* status, void* stream);
 
 /* Static text for a status code; never NULL. */
 const char* mxfp4_status_string(int status);

@@ -17,13 +17,16 @@ LIB_PATH = os.path.join(_PKG, "libmxfp4.so")
 F32, BF16 = 0, 1
 ROWS, COLS = 0, 1
 RNE, SR = 0, 1
+# Bit of the tensor-core entry points' status word: a bounded wait ran out.
+STATUS_WAIT_TIMEOUT = 1
 
 # Every symbol include/mxfp4.h declares.
 SYMBOLS = ("mxfp4_quantize", "mxfp4_quantize_oas", "mxfp4_dequantize",
            "mxfp4_double_quantize", "mxfp4_double_quantize_oas",
            "mxfp4_rht_quantize", "mxfp4_rht_quantize_oas", "mxfp4_osc_step",
            "mxfp4_osc_synthetic_update", "mxfp4_qramp_step", "mxfp4_qema_quantize",
-           "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_status_string")
+           "mxfp4_scales_to_blocked", "mxfp4_gemm", "mxfp4_gemm_quantize_a",
+           "mxfp4_status_string")
 
 
 class Mxfp4Error(RuntimeError):
@@ -57,9 +60,9 @@ def lib():
             "mxfp4_double_quantize_oas": [vp, i32, i64, i64, u64, vp, vp, vp,
                                           vp, vp],
             "mxfp4_rht_quantize": [vp, i32, i64, i64, u64, i32, u64, vp, vp,
-                                   vp, vp],
+                                   vp, vp, vp],
             "mxfp4_rht_quantize_oas": [vp, i32, i64, i64, u64, i32, u64, vp,
-                                       vp, vp, vp],
+                                       vp, vp, vp, vp],
             "mxfp4_osc_step": [vp, vp, vp, vp, i64, i64, i32, ctypes.c_float,
                                vp, vp],
             "mxfp4_osc_synthetic_update": [vp, i64, i64, u64, u32,
@@ -69,7 +72,9 @@ def lib():
             "mxfp4_qramp_step": [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
                                  ctypes.c_float, i64, vp, vp],
             "mxfp4_scales_to_blocked": [vp, i64, i64, vp, vp],
-            "mxfp4_gemm": [vp, vp, vp, vp, i64, i64, i64, vp, vp],
+            "mxfp4_gemm": [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp],
+            "mxfp4_gemm_quantize_a": [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp,
+                                      vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -204,10 +209,20 @@ def double_quantize(x, seed=0, out=None, stream=None, oas=False):
     return out
 
 
+def _status_word(status, device):
+    """The optional device status word of the tensor-core entry points: an
+    int32 tensor of one element on `device` (the kernels OR
+    MXFP4_STATUS_WAIT_TIMEOUT = 1 into it; the caller zeroes it)."""
+    if status is not None:
+        _buffer(status, "status", torch.int32, 1, device)
+    return _ptr(status)
+
+
 def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
-                 out=None, stream=None, oas=False):
+                 out=None, stream=None, oas=False, status=None):
     """mxfp4_rht_quantize (mxfp4_rht_quantize_oas when oas): (codes, scales,
-    rotated or None), ROWS layout."""
+    rotated or None), ROWS layout. status: optional int32 CUDA tensor of one
+    element, the timeout status word."""
     _cuda2d(x, "x")
     R, C = x.shape
     if out is None:
@@ -219,9 +234,10 @@ def rht_quantize(x, sign_seed=0, rounding=RNE, sr_seed=0, want_rotated=False,
     _buffer(scales, "scales", torch.uint8, R * C // 32, x.device)
     if rot is not None:
         _buffer(rot, "rotated", torch.float32, R * C, x.device)
+    st = _status_word(status, x.device)
     name = "mxfp4_rht_quantize_oas" if oas else "mxfp4_rht_quantize"
     _check(getattr(lib(), name)(_ptr(x), _dtype_code(x), R, C, sign_seed, rounding,
-                                sr_seed, _ptr(codes), _ptr(scales), _ptr(rot),
+                                sr_seed, _ptr(codes), _ptr(scales), _ptr(rot), st,
                                 _stream(x.device, stream)),
            name)
     return out
@@ -320,9 +336,10 @@ def scales_to_blocked(scales, out=None, stream=None):
     return out
 
 
-def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None):
+def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None, status=None):
     """mxfp4_gemm: C = A B^T in fp32 for MXFP4 operands given as K-major
-    codes [rows, k/2] and blocked scales (from scales_to_blocked)."""
+    codes [rows, k/2] and blocked scales (from scales_to_blocked). status:
+    optional int32 CUDA tensor of one element, the timeout status word."""
     for name, t in (("a_codes", a_codes), ("a_blocked", a_blocked),
                     ("b_codes", b_codes), ("b_blocked", b_blocked)):
         _cuda2d(t, name)
@@ -341,9 +358,48 @@ def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None):
     if out is None:
         out = torch.empty((m, n), dtype=torch.float32, device=a_codes.device)
     _buffer(out, "out", torch.float32, m * n, a_codes.device)
+    st = _status_word(status, a_codes.device)
     _check(lib().mxfp4_gemm(_ptr(a_codes), _ptr(a_blocked), _ptr(b_codes),
-                            _ptr(b_blocked), m, n, k, _ptr(out),
+                            _ptr(b_blocked), m, n, k, _ptr(out), st,
                             _stream(a_codes.device, stream)), "mxfp4_gemm")
+    return out
+
+
+def gemm_quantize_a(x, b_codes, b_blocked, out=None, want_a=False, stream=None,
+                    status=None):
+    """mxfp4_gemm_quantize_a: C = Q_D(x) B^T in fp32, x bf16 [m, k] (k a
+    multiple of 256) quantized 1x32 nearest-even inside the GEMM's load
+    stage, B given as K-major codes [n, k/2] and blocked scales. Returns C,
+    or (C, a_codes, a_scales) with want_a (Q_D(x) in the ROWS layout)."""
+    _cuda2d(x, "x")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    m, k = x.shape
+    for name, t in (("b_codes", b_codes), ("b_blocked", b_blocked)):
+        _cuda2d(t, name)
+        if t.dtype != torch.uint8:
+            raise TypeError("%s must be uint8" % name)
+        _on_device(t, name, x.device)
+    n = b_codes.shape[0]
+    if b_codes.shape[1] * 2 != k:
+        raise ValueError("b_codes must have k/2 bytes per row")
+    need = -(-n // 128) * 128 * (-(-k // 128) * 4)
+    if b_blocked.numel() != need:
+        raise ValueError("b_blocked must hold %d bytes" % need)
+    d = x.device
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.float32, device=d)
+        if want_a:
+            out = (out, _empty_u8((m, k // 2), d), _empty_u8((m, k // 32), d))
+    c, ac, as_ = (out if want_a else (out, None, None))
+    _buffer(c, "out", torch.float32, m * n, d)
+    if want_a:
+        _buffer(ac, "a_codes", torch.uint8, m * k // 2, d)
+        _buffer(as_, "a_scales", torch.uint8, m * k // 32, d)
+    st = _status_word(status, d)
+    _check(lib().mxfp4_gemm_quantize_a(_ptr(x), m, n, k, _ptr(b_codes), _ptr(b_blocked),
+                                       _ptr(c), _ptr(ac), _ptr(as_), st,
+                                       _stream(d, stream)), "mxfp4_gemm_quantize_a")
     return out
 
 
@@ -364,4 +420,5 @@ mxfp4_qramp_step = qramp_step
 mxfp4_qema_quantize = qema_quantize
 mxfp4_scales_to_blocked = scales_to_blocked
 mxfp4_gemm = gemm
+mxfp4_gemm_quantize_a = gemm_quantize_a
 mxfp4_status_string = status_string

@@ -6,7 +6,9 @@ explicit intrinsics).
 """
 import glob
 import os
+import shutil
 import subprocess
+import tempfile
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -31,17 +33,42 @@ def _stale():
     return any(os.path.getmtime(d) > t for d in deps)
 
 
+def _compile(out: str, defines=(), verbose: bool = False) -> None:
+    """Compile each .cu under csrc/ to an object in parallel, then link them
+    into the shared library `out` (written atomically)."""
+    nvcc = os.environ.get("NVCC", "nvcc")
+    flags = NVCC_FLAGS + ["-D" + d for d in defines] + (["-Xptxas", "-v"] if verbose else [])
+    tmpdir = tempfile.mkdtemp(prefix="mxfp4_build_")
+    try:
+        objs, procs = [], []
+        for src in sources():
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            objs.append(obj)
+            procs.append((src, subprocess.Popen([nvcc] + flags + ["-c", "-o", obj, src])))
+        failed = [src for src, pr in procs if pr.wait() != 0]
+        if failed:
+            raise RuntimeError("nvcc failed on " + ", ".join(failed))
+        tmp = out + ".tmp%d" % os.getpid()
+        subprocess.run([nvcc] + NVCC_FLAGS + ["-shared", "-o", tmp] + objs, check=True)
+        os.replace(tmp, out)
+    finally:
+        shutil.rmtree(tmpdir, ignore_errors=True)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every .cu under csrc/ into libmxfp4.so if it is out of date."""
     if not force and not _stale():
         return LIB
-    nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + [
-        "-shared", "-o", tmp] + sources()
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    _compile(LIB, verbose=verbose)
     return LIB
+
+
+def build_variant(out: str, defines) -> str:
+    """The same library built with extra preprocessor definitions (e.g.
+    MXFP4_ACC_WAIT_POLLS=0, the test build whose accumulator waits give up
+    at once) into `out`, outside the package."""
+    _compile(out, defines=defines)
+    return out
 
 
 if __name__ == "__main__":

@@ -14,6 +14,11 @@ bool aligned16(const void* p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// The optional status word (NULL passes).
+bool aligned4(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 3u) == 0;
+}
+
 // rows, cols > 0, each at most MXFP4_MAX_DIM, product below 2^46.
 bool dims_ok(int64_t rows, int64_t cols) {
   if (rows <= 0 || cols <= 0) return false;
@@ -126,33 +131,35 @@ static mxfp4_status rht_quantize_with_rule(const void* x, int dtype, int64_t row
                                            int64_t cols, uint64_t sign_seed,
                                            int rounding, uint64_t sr_seed,
                                            uint8_t* codes, uint8_t* scales,
-                                           float* rotated, void* stream, bool oas) {
+                                           float* rotated, int* status, void* stream,
+                                           bool oas) {
   if (!dtype_ok(dtype) || !rounding_ok(rounding)) return MXFP4_ERR_ENUM;
   if (!x || !codes || !scales) return MXFP4_ERR_NULL;
   if (!dims_ok(rows, cols) || cols % 32) return MXFP4_ERR_SHAPE;
-  if (!aligned16(x) || !aligned16(codes) || (rotated && !aligned16(rotated)))
+  if (!aligned16(x) || !aligned16(codes) || (rotated && !aligned16(rotated)) ||
+      !aligned4(status))
     return MXFP4_ERR_ALIGN;
   return from_cuda(mxfp4::launch_rht_quant(
       x, dtype == MXFP4_BF16, rows, cols, sign_seed, rounding == MXFP4_SR,
-      sr_seed, codes, scales, rotated, as_stream(stream), oas));
+      sr_seed, codes, scales, rotated, status, as_stream(stream), oas));
 }
 
 mxfp4_status mxfp4_rht_quantize(const void* x, int dtype, int64_t rows,
                                 int64_t cols, uint64_t sign_seed,
                                 int rounding, uint64_t sr_seed,
                                 uint8_t* codes, uint8_t* scales,
-                                float* rotated, void* stream) {
+                                float* rotated, int* status, void* stream) {
   return rht_quantize_with_rule(x, dtype, rows, cols, sign_seed, rounding, sr_seed, codes,
-                                scales, rotated, stream, false);
+                                scales, rotated, status, stream, false);
 }
 
 mxfp4_status mxfp4_rht_quantize_oas(const void* x, int dtype, int64_t rows,
                                     int64_t cols, uint64_t sign_seed,
                                     int rounding, uint64_t sr_seed,
                                     uint8_t* codes, uint8_t* scales,
-                                    float* rotated, void* stream) {
+                                    float* rotated, int* status, void* stream) {
   return rht_quantize_with_rule(x, dtype, rows, cols, sign_seed, rounding, sr_seed, codes,
-                                scales, rotated, stream, true);
+                                scales, rotated, status, stream, true);
 }
 
 mxfp4_status mxfp4_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
@@ -219,18 +226,33 @@ mxfp4_status mxfp4_scales_to_blocked(const uint8_t* scales, int64_t rows,
 mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                         const uint8_t* b_codes, const uint8_t* b_scales,
                         int64_t m, int64_t n, int64_t k, float* c,
-                        void* stream) {
+                        int* status, void* stream) {
   if (!a_codes || !a_scales || !b_codes || !b_scales || !c)
     return MXFP4_ERR_NULL;
   if (!dims_ok(m, k) || !dims_ok(n, k) || !dims_ok(m, n) || k % 32)
     return MXFP4_ERR_SHAPE;
   if ((m + 127) / 128 > 65535) return MXFP4_ERR_SHAPE;  // grid y
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) ||
-      !aligned16(b_scales) || !aligned16(c))
+      !aligned16(b_scales) || !aligned16(c) || !aligned4(status))
     return MXFP4_ERR_ALIGN;
   return from_cuda(mxfp4::launch_gemm_mxf4(a_codes, a_scales, b_codes,
-                                           b_scales, m, n, k, c,
+                                           b_scales, m, n, k, c, status,
                                            as_stream(stream)));
+}
+
+mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t k,
+                                   const uint8_t* b_codes, const uint8_t* b_scales,
+                                   float* c, uint8_t* a_codes, uint8_t* a_scales,
+                                   int* status, void* stream) {
+  if (!x || !b_codes || !b_scales || !c || (a_codes == nullptr) != (a_scales == nullptr))
+    return MXFP4_ERR_NULL;
+  if (!dims_ok(m, k) || !dims_ok(n, k) || !dims_ok(m, n) || k % 256)
+    return MXFP4_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(c) ||
+      !aligned16(a_codes) || !aligned4(status))
+    return MXFP4_ERR_ALIGN;
+  return from_cuda(mxfp4::launch_gemm_qa(x, m, n, k, b_codes, b_scales, c, a_codes,
+                                         a_scales, status, as_stream(stream)));
 }
 
 const char* mxfp4_status_string(int status) {
@@ -239,8 +261,9 @@ const char* mxfp4_status_string(int status) {
     case MXFP4_ERR_NULL: return "a required pointer is NULL";
     case MXFP4_ERR_SHAPE:
       return "bad shape: rows/cols must be positive, within the size limit, "
-             "and the group axis a multiple of 32";
-    case MXFP4_ERR_ALIGN: return "a tensor pointer is not 16-byte aligned";
+             "and the group axis a multiple of 32 (of 256 for the fused GEMM)";
+    case MXFP4_ERR_ALIGN:
+      return "a tensor pointer is not 16-byte aligned (a status word: 4-byte)";
     case MXFP4_ERR_ENUM: return "dtype, axis or rounding out of range";
     case MXFP4_ERR_CUDA: return "CUDA launch failed";
     default: return "unknown status";

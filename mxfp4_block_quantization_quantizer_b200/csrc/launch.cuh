@@ -36,11 +36,13 @@ cudaError_t launch_double_quant(const void* x, bool bf16, int64_t rows,
                                 uint8_t* col_codes, uint8_t* col_scales,
                                 cudaStream_t s, bool oas = false);
 
+// status: device word or nullptr; the tensor-core kernel ORs 1 into it when
+// one of its bounded waits ran out.
 cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
                              int64_t cols, uint64_t sign_seed, bool sr,
                              uint64_t sr_seed, uint8_t* codes,
-                             uint8_t* scales, float* rotated, cudaStream_t s,
-                             bool oas = false);
+                             uint8_t* scales, float* rotated, int* status,
+                             cudaStream_t s, bool oas = false);
 
 cudaError_t launch_osc_step(float* w, float* w_snap, float* d_w, float* d_q,
                             int64_t rows, int64_t cols, bool window_end,
@@ -66,10 +68,19 @@ cudaError_t launch_scales_blocked(const uint8_t* scales, int64_t rows,
                                   cudaStream_t s);
 
 // C[m][n] = sum_k A[m][k] B[n][k] on MXFP4 operands (K-major codes,
-// blocked scales), fp32 out, on the block-scaled tensor cores.
+// blocked scales), fp32 out, on the block-scaled tensor cores; status as for
+// launch_rht_quant.
 cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
                              const uint8_t* b, const uint8_t* b_scales,
                              int64_t m, int64_t n, int64_t k, float* c,
-                             cudaStream_t s);
+                             int* status, cudaStream_t s);
+
+// C = Q_D(X) B^T with X (bf16 [m][k], k a multiple of 256) quantized 1x32
+// nearest-even inside the GEMM's load stage; a_codes / a_scales (ROWS
+// layout) receive that quantization when not null.
+cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k,
+                           const uint8_t* b, const uint8_t* b_scales, float* c,
+                           uint8_t* a_codes, uint8_t* a_scales, int* status,
+                           cudaStream_t s);
 
 }  // namespace mxfp4

@@ -181,7 +181,7 @@ struct __align__(1024) RhtSmem {
   uint4 out_codes[2][4][32][kRtGroups];           // staged codes [tile parity][quarter][row]
   uint8_t out_scales[2][4][32][kRtGroups];
   unsigned long long full[kRtStages], empty[kRtStages], acc_full[kRtAccBufs],
-      acc_empty[kRtAccBufs];
+      acc_empty[kRtAccBufs], drain;
   uint32_t tmem_base;
   int failed;
 };
@@ -275,7 +275,8 @@ template <bool SR, bool ROT, bool STAGED, bool OAS>
 __global__ void __launch_bounds__(kRtThreads, 1)
     k_rht_tc(const __grid_constant__ CUtensorMap tm_x, int64_t rows, int64_t cols,
              uint32_t sign_key, RngKey key, uint8_t* __restrict__ codes,
-             uint8_t* __restrict__ scales, float* __restrict__ rotated) {
+             uint8_t* __restrict__ scales, float* __restrict__ rotated,
+             int* __restrict__ status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte swizzle wants 1024-byte aligned tiles (1 KB of slack)
   RhtSmem& sm = *reinterpret_cast<RhtSmem*>(
@@ -297,6 +298,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.acc_empty[b])),
                    "r"(kRtEpiWarps));
     }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.drain)));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     sm.failed = 0;
   }
@@ -319,10 +321,15 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 #pragma unroll
     for (int s = 0; s < kRtStages; ++s) slot_cb[s] = -1;
     uint32_t s = 0, ph = 0;
+    // stages with a load issued and the phase parity of each one's last
+    // load (the same in every lane): every load lands before the CTA ends
+    uint32_t issued = 0, last_ph = 0;
     int64_t cb = t_begin / n_rt, rt = t_begin % n_rt;
     for (int64_t t = t_begin; t < t_end; ++t, rt = rt + 1 == n_rt ? 0 : rt + 1,
                  cb += rt == 0 ? 1 : 0) {
-      if (!wait_parity_sleep(&sm.empty[s], ph ^ 1u)) {  // runs ahead of the epilogue
+      // runs ahead of the epilogue; the lanes agree on the outcome
+      if (!__all_sync(0xFFFFFFFFu,
+                      wait_parity_or_failed<true>(&sm.empty[s], ph ^ 1u, &sm.failed))) {
         atomicExch(&sm.failed, 1);
         break;
       }
@@ -358,6 +365,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       // the async proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
+      issued |= 1u << s;
+      last_ph = (last_ph & ~(1u << s)) | (ph << s);
       if (lane == 0) {
         expect_tx(&sm.full[s], (kRtGroups / 2) * 128 * 128);
 #pragma unroll
@@ -371,6 +380,11 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         ph ^= 1u;
       }
     }
+    // drain (immediate unless a wait ran out)
+    if (lane == 0)
+      for (uint32_t st = 0; st < kRtStages; ++st)
+        if ((issued >> st) & 1u) wait_parity(&sm.full[st], (last_ph >> st) & 1u);
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint64_t x_d0 = smem_desc_sw128(&sm.x[0][0][0][0]);
@@ -384,8 +398,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
                          kHk = (2 * 32 * 16) >> 4;
       uint32_t s = 0, ph = 0, b = 0, bph = 0;
       for (int64_t t = t_begin; t < t_end; ++t) {
-        if (!wait_parity_sleep(&sm.full[s], ph) ||
-            !wait_parity_sleep(&sm.acc_empty[b], bph ^ 1u)) {
+        if (!wait_parity_or_failed<true>(&sm.full[s], ph, &sm.failed) ||
+            !wait_parity_or_failed<true>(&sm.acc_empty[b], bph ^ 1u, &sm.failed)) {
           atomicExch(&sm.failed, 1);
           break;
         }
@@ -409,6 +423,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
           bph ^= 1u;
         }
       }
+      // drain: every MMA issued has completed before the stages or the
+      // tensor memory can go away
+      commit_to(&sm.drain);
+      if (!wait_parity(&sm.drain, 0)) atomicExch(&sm.failed, 1);
     }
     __syncwarp();
   } else {
@@ -420,18 +438,28 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     for (int64_t t = t_begin; t < t_end; ++t, rt = rt + 1 == n_rt ? 0 : rt + 1,
                  cb += rt == 0 ? 1 : 0) {
       const int64_t r = rt * 128 + 32 * q + lane;
-      // after a failure every warp still runs every tile (without waiting),
-      // so the quarter barriers of the staged stores stay matched
-      const bool ok = !failed_flag(&sm.failed) && wait_parity(&sm.acc_full[b], bph);
+      // after a failure every warp still runs every tile, without waiting
+      // and without touching tensor memory (NaN rotations, zero codes,
+      // scale 0xFF), so the quarter barriers of the staged stores stay
+      // matched
+      const bool ok = __all_sync(0xFFFFFFFFu, !failed_flag(&sm.failed) &&
+                                                  wait_parity(&sm.acc_full[b], bph,
+                                                              kAccWaitLimit));
       if (!ok) atomicExch(&sm.failed, 1);
-      asm volatile("tcgen05.fence::after_thread_sync;");
+      if (ok) asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll 1
       for (int gi = 0; gi < kPer; ++gi) {
         const int g = kPer * gs + gi;
         uint32_t zb[32];
-        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + 32u * kRtGroups * b + 32u * uint32_t(g), zb);
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (gi == kPer - 1) {  // the accumulator is read: release it
+        if (ok) {
+          tmem_ld32(tmem + (uint32_t(32 * q) << 16) + 32u * kRtGroups * b + 32u * uint32_t(g),
+                    zb);
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) zb[j] = kNaNf32;
+        }
+        if (ok && gi == kPer - 1) {  // the accumulator is read: release it
           asm volatile("tcgen05.fence::before_thread_sync;");
           __syncwarp();
           if (lane == 0)
@@ -490,6 +518,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
+  report_failure(status, &sm.failed);
   if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(32 * kRtGroups * kRtAccBufs));
@@ -498,7 +527,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
 template <bool SR, bool ROT, bool STAGED, bool OAS>
 cudaError_t rht_tc_impl(const CUtensorMap& mx, int64_t rows, int64_t cols,
                         uint32_t sign_key, RngKey key, uint8_t* codes, uint8_t* scales,
-                        float* rotated, cudaStream_t s) {
+                        float* rotated, int* status, cudaStream_t s) {
   auto kern = k_rht_tc<SR, ROT, STAGED, OAS>;
   constexpr size_t smem = sizeof(RhtSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
@@ -506,7 +535,8 @@ cudaError_t rht_tc_impl(const CUtensorMap& mx, int64_t rows, int64_t cols,
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((rows + 127) / 128) * ((cols + 32 * kRtGroups - 1) / (32 * kRtGroups));
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kRtThreads, smem, tiles);
-  kern<<<grid, kRtThreads, smem, s>>>(mx, rows, cols, sign_key, key, codes, scales, rotated);
+  kern<<<grid, kRtThreads, smem, s>>>(mx, rows, cols, sign_key, key, codes, scales, rotated,
+                                      status);
   return cudaGetLastError();
 }
 
@@ -535,7 +565,8 @@ cudaError_t rht_impl(const void* x, int64_t rows, int64_t cols,
 template <bool OAS>
 static cudaError_t rht_dispatch(const void* x, bool bf16, int64_t rows, int64_t cols,
                                 uint32_t sign_key, RngKey key, bool sr, uint8_t* codes,
-                                uint8_t* scales, float* rotated, cudaStream_t s) {
+                                uint8_t* scales, float* rotated, int* status,
+                                cudaStream_t s) {
   const bool rot = rotated != nullptr;
   if (bf16) {
     // X as a byte array [rows][2 cols] for the TMA: 128-byte boxes
@@ -543,13 +574,13 @@ static cudaError_t rht_dispatch(const void* x, bool bf16, int64_t rows, int64_t 
     if (!encode_rows_sw128(&mx, x, rows, 2 * cols, 128)) return cudaErrorInvalidValue;
     if (sr)
       return rot ? rht_tc_impl<true, true, false, OAS>(mx, rows, cols, sign_key, key, codes,
-                                                       scales, rotated, s)
+                                                       scales, rotated, status, s)
                  : rht_tc_impl<true, false, false, OAS>(mx, rows, cols, sign_key, key, codes,
-                                                        scales, rotated, s);
+                                                        scales, rotated, status, s);
     return rot ? rht_tc_impl<false, true, false, OAS>(mx, rows, cols, sign_key, key, codes,
-                                                      scales, rotated, s)
+                                                      scales, rotated, status, s)
                : rht_tc_impl<false, false, true, OAS>(mx, rows, cols, sign_key, key, codes,
-                                                      scales, rotated, s);
+                                                      scales, rotated, status, s);
   }
   if (sr)
     return rot ? rht_impl<true, true, OAS>(x, rows, cols, sign_key, key, codes,
@@ -565,14 +596,14 @@ static cudaError_t rht_dispatch(const void* x, bool bf16, int64_t rows, int64_t 
 cudaError_t launch_rht_quant(const void* x, bool bf16, int64_t rows,
                              int64_t cols, uint64_t sign_seed, bool sr,
                              uint64_t sr_seed, uint8_t* codes,
-                             uint8_t* scales, float* rotated,
+                             uint8_t* scales, float* rotated, int* status,
                              cudaStream_t s, bool oas) {
   const uint32_t sign_key = stream_key(sign_seed, 1);
   const RngKey key = make_key(sr_seed, 0);
   return oas ? rht_dispatch<true>(x, bf16, rows, cols, sign_key, key, sr, codes, scales,
-                                  rotated, s)
+                                  rotated, status, s)
              : rht_dispatch<false>(x, bf16, rows, cols, sign_key, key, sr, codes, scales,
-                                   rotated, s);
+                                   rotated, status, s);
 }
 
 }  // namespace mxfp4

@@ -16,6 +16,18 @@ namespace {
 // thread for a while): a wait that runs out reports failure instead of
 // spinning forever.
 constexpr long long kWaitLimit = 1ll << 22;
+// The waits of the threads that read the accumulator out of tensor memory
+// for its completion. A test build defines MXFP4_ACC_WAIT_POLLS to 0, so
+// that on a normal input those waits give up at once and the timeout path
+// (NaN or zero-scale tiles, the caller's status word, the drains) runs;
+// every other wait keeps kWaitLimit.
+#ifndef MXFP4_ACC_WAIT_POLLS
+#define MXFP4_ACC_WAIT_POLLS (1ll << 22)
+#endif
+constexpr long long kAccWaitLimit = MXFP4_ACC_WAIT_POLLS;
+// Bit the tensor-core kernels OR into the caller's status word when a wait
+// ran out (MXFP4_STATUS_WAIT_TIMEOUT of the public header).
+constexpr int kStatusWaitTimeout = 1;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,9 +58,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p) {
 }
 
 __device__ __forceinline__ bool wait_parity(unsigned long long* bar,
-                                            uint32_t parity) {
+                                            uint32_t parity,
+                                            long long limit = kWaitLimit) {
   const uint32_t a = smem_u32(bar);
-  for (long long i = 0; i < kWaitLimit; ++i) {
+  for (long long i = 0; i < limit; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -84,6 +97,30 @@ __device__ __forceinline__ bool wait_parity_sleep(unsigned long long* bar,
   return false;
 }
 
+// wait_parity for a barrier that another role of the CTA feeds: gives up
+// as soon as *failed is set (that role timed out and stopped), checking the
+// flag every 64 polls; with SLEEP the thread naps between polls as in
+// wait_parity_sleep.
+template <bool SLEEP>
+__device__ __forceinline__ bool wait_parity_or_failed(unsigned long long* bar,
+                                                      uint32_t parity, const int* failed) {
+  const uint32_t a = smem_u32(bar);
+  for (long long i = 0; i < kWaitLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 63) == 63 && *static_cast<const volatile int*>(failed) != 0) return false;
+    if (SLEEP) __nanosleep(kPollSleepNs);
+  }
+  return false;
+}
+
 __device__ __forceinline__ void expect_tx(unsigned long long* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -109,6 +146,13 @@ __device__ __forceinline__ void commit_to(unsigned long long* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_u32(bar)));
+}
+
+// Thread 0, after the kernel's last __syncthreads: OR the timeout bit into
+// the caller's status word if any wait of this CTA ran out.
+__device__ __forceinline__ void report_failure(int* status, const int* failed) {
+  if (threadIdx.x == 0 && status != nullptr && *static_cast<const volatile int*>(failed) != 0)
+    atomicOr(status, kStatusWaitTimeout);
 }
 
 // cuTensorMapEncodeTiled through the entry point the runtime hands out (no

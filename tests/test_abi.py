@@ -17,6 +17,7 @@ OK, NULL, SHAPE, ALIGN, ENUM, CUDA = range(6)
 P = ctypes.c_void_p(4096)       # a 16-byte aligned non-null pointer
 PODD = ctypes.c_void_p(4096 + 8)  # misaligned by 8 bytes
 NUL = ctypes.c_void_p(0)
+P2 = ctypes.c_void_p(4096 + 2)  # not even 4-byte aligned
 
 
 def declared_symbols():
@@ -83,10 +84,10 @@ def test_overflow_aware_double_and_rotation_reject_bad_arguments():
     assert L.mxfp4_double_quantize_oas(P, 1, 48, 64, 0, P, P, P, P, NUL) == SHAPE
     assert L.mxfp4_double_quantize_oas(P, 1, 64, 64, 0, P, NUL, P, P, NUL) == NULL
     assert L.mxfp4_double_quantize_oas(PODD, 1, 64, 64, 0, P, P, P, P, NUL) == ALIGN
-    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 40, 0, 0, 0, P, P, NUL, NUL) == SHAPE
-    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 3, 0, P, P, NUL, NUL) == ENUM
-    assert L.mxfp4_rht_quantize_oas(NUL, 1, 64, 64, 0, 0, 0, P, P, NUL, NUL) == NULL
-    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 0, 0, P, P, PODD, NUL) == ALIGN
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 40, 0, 0, 0, P, P, NUL, NUL, NUL) == SHAPE
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 3, 0, P, P, NUL, NUL, NUL) == ENUM
+    assert L.mxfp4_rht_quantize_oas(NUL, 1, 64, 64, 0, 0, 0, P, P, NUL, NUL, NUL) == NULL
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 0, 0, P, P, PODD, NUL, NUL) == ALIGN
 
 
 def test_other_entry_points_reject_bad_arguments():
@@ -99,9 +100,9 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_double_quantize(P, 1, 48, 64, 0, P, P, P, P, NUL) == SHAPE
     assert L.mxfp4_double_quantize(P, 1, 64, 64, 0, P, P, NUL, P, NUL) == NULL
     assert L.mxfp4_double_quantize(P, 1, 64, 64, 0, P, P, PODD, P, NUL) == ALIGN
-    assert L.mxfp4_rht_quantize(P, 1, 64, 40, 0, 0, 0, P, P, NUL, NUL) == SHAPE
-    assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 3, 0, P, P, NUL, NUL) == ENUM
-    assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 0, 0, P, P, PODD, NUL) == ALIGN
+    assert L.mxfp4_rht_quantize(P, 1, 64, 40, 0, 0, 0, P, P, NUL, NUL, NUL) == SHAPE
+    assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 3, 0, P, P, NUL, NUL, NUL) == ENUM
+    assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 0, 0, P, P, PODD, NUL, NUL) == ALIGN
     assert L.mxfp4_osc_step(P, P, NUL, P, 64, 64, 0, 4.0, NUL, NUL) == NULL
     assert L.mxfp4_osc_step(P, P, P, P, 64, 40, 0, 4.0, NUL, NUL) == SHAPE
     assert L.mxfp4_osc_step(P, PODD, P, P, 64, 64, 0, 4.0, NUL, NUL) == ALIGN
@@ -123,11 +124,23 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_scales_to_blocked(P, 128, -4, P, NUL) == SHAPE
     assert L.mxfp4_scales_to_blocked(P, 1 << 32, 4, P, NUL) == SHAPE
     assert L.mxfp4_scales_to_blocked(PODD, 128, 4, PODD, NUL) == ALIGN
-    assert L.mxfp4_gemm(P, P, P, NUL, 128, 128, 256, P, NUL) == NULL
-    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 48, P, NUL) == SHAPE
-    assert L.mxfp4_gemm(P, P, P, P, 0, 128, 256, P, NUL) == SHAPE
-    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, PODD, NUL) == ALIGN
-    assert L.mxfp4_gemm(P, PODD, P, P, 128, 128, 256, P, NUL) == ALIGN
+    assert L.mxfp4_gemm(P, P, P, NUL, 128, 128, 256, P, NUL, NUL) == NULL
+    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 48, P, NUL, NUL) == SHAPE
+    assert L.mxfp4_gemm(P, P, P, P, 0, 128, 256, P, NUL, NUL) == SHAPE
+    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, PODD, NUL, NUL) == ALIGN
+    assert L.mxfp4_gemm(P, PODD, P, P, 128, 128, 256, P, NUL, NUL) == ALIGN
+    g = L.mxfp4_gemm_quantize_a
+    assert g(NUL, 128, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == NULL
+    assert g(P, 128, 256, 256, P, P, P, P, NUL, NUL, NUL) == NULL   # codes without scales
+    assert g(P, 128, 256, 128, P, P, P, NUL, NUL, NUL, NUL) == SHAPE  # k % 256
+    assert g(P, 0, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == SHAPE
+    assert g(PODD, 128, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == ALIGN
+    assert g(P, 128, 256, 256, P, P, P, PODD, P, NUL, NUL) == ALIGN
+    assert g(P, 128, 256, 256, P, P, P, NUL, NUL, P2, NUL) == ALIGN
+    # the status word needs 4-byte alignment only
+    assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, P, P2, NUL) == ALIGN
+    assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 0, 0, P, P, NUL, P2, NUL) == ALIGN
+    assert L.mxfp4_rht_quantize_oas(P, 1, 64, 64, 0, 0, 0, P, P, NUL, P2, NUL) == ALIGN
 
 
 def test_binding_refuses_host_tensors():

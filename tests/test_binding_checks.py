@@ -135,3 +135,37 @@ def test_qema_blocked_gemm_and_tracker_reject_bad_buffers(fake):
     B.scales_to_blocked(u8(130, 5), out=u8(256, 8))
     B.gemm(a, ab, a, ab, 128, out=torch.zeros((128, 128)))
     assert fake.calls == ["mxfp4_scales_to_blocked", "mxfp4_gemm"]
+
+
+def test_status_word_must_be_one_int32(fake):
+    a, ab = u8(128, 64), u8(128, 4)
+    for bad in (torch.zeros(2, dtype=torch.int32), torch.zeros(1, dtype=torch.int64),
+                torch.zeros(1, dtype=torch.float32)):
+        with pytest.raises(ValueError):
+            B.gemm(a, ab, a, ab, 128, status=bad)
+        with pytest.raises(ValueError):
+            B.rht_quantize(X, status=bad)
+    assert fake.calls == []
+    B.gemm(a, ab, a, ab, 128, status=torch.zeros(1, dtype=torch.int32))
+    B.rht_quantize(X, status=torch.zeros(1, dtype=torch.int32))
+    assert fake.calls == ["mxfp4_gemm", "mxfp4_rht_quantize"]
+
+
+def test_gemm_quantize_a_checks_its_buffers(fake):
+    x = torch.zeros((128, 256), dtype=torch.bfloat16)
+    bc, bb = u8(256, 128), u8(256, 8)
+    with pytest.raises(TypeError):      # X must be bf16
+        B.gemm_quantize_a(x.float(), bc, bb)
+    with pytest.raises(ValueError):     # B codes of another k
+        B.gemm_quantize_a(x, u8(256, 64), bb)
+    with pytest.raises(ValueError):     # blocked scales short
+        B.gemm_quantize_a(x, bc, u8(256, 7))
+    with pytest.raises(ValueError):     # C short
+        B.gemm_quantize_a(x, bc, bb, out=torch.zeros((128, 255)))
+    with pytest.raises(ValueError):     # A codes short
+        B.gemm_quantize_a(x, bc, bb, want_a=True,
+                          out=(torch.zeros((128, 256)), u8(128, 127), u8(128, 8)))
+    assert fake.calls == []
+    c, ac, as_ = B.gemm_quantize_a(x, bc, bb, want_a=True)
+    assert c.shape == (128, 256) and ac.shape == (128, 128) and as_.shape == (128, 8)
+    assert fake.calls == ["mxfp4_gemm_quantize_a"]

@@ -1,0 +1,108 @@
+"""The forward GEMM with the activation quantized in its load stage
+(mxfp4_gemm_quantize_a, C = Q_D(X) B^T) against the two-step path it
+replaces and against the oracle.
+
+- Q_D(X) as the fused kernel writes it out equals mxfp4_quantize's ROWS RNE
+  codes and scales byte for byte, and the oracle's;
+- C equals mxfp4_gemm on those codes bit for bit (same tiles, same MMA
+  sequence) and lies within the fp32 accumulation bound of the oracle's
+  exact product: (k - 1) 2^-24 sum_j |a_j b_j|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_block_quantization_quantizer_b200 as m
+import oracle as O
+from mxfp4_block_quantization_quantizer_b200 import workloads as W
+from gpu_util import to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def weight(n, k, seed):
+    """A pre-quantized weight: ROWS RNE codes and scales of N(0,1) bf16."""
+    w = W.normal_bf16(n, k, seed)
+    wc, ws = m.quantize(to_dev(w), m.ROWS, m.RNE)
+    return wc, ws
+
+
+def check_against_oracle(c, xc, xs, wc, ws, k, rows=None):
+    """C (rows `rows` of it) within the accumulation bound of the oracle's
+    fp64 product of the dequantized operands."""
+    if rows is not None:
+        xc, xs, c = xc[rows], xs[rows], c[rows]
+    want = O.gemm(xc, xs, wc, ws, k)
+    da = np.abs(O.dequantize(xc, xs, xc.shape[0], k, O.ROWS, "f32").astype(np.float64))
+    db = np.abs(O.dequantize(wc, ws, wc.shape[0], k, O.ROWS, "f32").astype(np.float64))
+    bound = (k - 1) * 2.0 ** -24 * (da @ db.T)
+    err = np.abs(c.astype(np.float64) - want)
+    assert np.all(err <= bound), "max error / bound %g" % (err / np.maximum(bound, 1e-300)).max()
+
+
+@pytest.mark.parametrize("mnk", [(128, 256, 256),    # one tile, one stage
+                                 (200, 136, 512),    # ragged rows and columns
+                                 (384, 520, 768),    # 3 x 3 tiles, a 8-column edge tile
+                                 (1000, 64, 1024),   # narrow output, many row tiles
+                                 (256, 768, 2560)])  # 10 stages: the rings wrap
+def test_fused_equals_quantize_then_gemm(mnk):
+    mm, nn, k = mnk
+    x = W.normal_bf16(mm, k, 21, 0.005, 50.0)
+    x[0, :32] = 0          # an all-zero group
+    xd = to_dev(x)
+    wc, ws = weight(nn, k, 22)
+    wb = m.scales_to_blocked(ws)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, want_a=True, status=st)
+    assert int(st.item()) == 0
+    qc, qs = m.quantize(xd, m.ROWS, m.RNE)
+    assert torch.equal(ac, qc) and torch.equal(as_, qs)
+    oc, os_ = O.quantize(x, O.ROWS, O.RNE)
+    assert np.array_equal(to_np(ac), oc) and np.array_equal(to_np(as_), os_)
+    ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, k)
+    assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+    check_against_oracle(to_np(c), oc, os_, to_np(wc), to_np(ws), k)
+    # without the optional outputs: the same C
+    c2 = m.gemm_quantize_a(xd, wc, wb)
+    assert torch.equal(c2.view(torch.int32), c.view(torch.int32))
+
+
+def test_special_values_follow_the_quantizer():
+    """Groups whose maximum is inf or NaN get scale byte 0xFF (NaN) in the
+    quantizer; the fused GEMM quantizes them the same way."""
+    k = 256
+    x = W.normal_bf16(128, k, 23)
+    xi = x.view(np.uint16)
+    xi[3, 5] = 0x7F80      # +inf
+    xi[9, 40] = 0xFFC1     # NaN
+    xi[17, 100] = 0x0001   # subnormal in an otherwise normal group
+    xd = to_dev(x)
+    wc, ws = weight(256, k, 24)
+    c, ac, as_ = m.gemm_quantize_a(xd, wc, m.scales_to_blocked(ws), want_a=True)
+    qc, qs = m.quantize(xd, m.ROWS, m.RNE)
+    assert torch.equal(ac, qc) and torch.equal(as_, qs)
+    ref = m.gemm(qc, m.scales_to_blocked(qs), wc, m.scales_to_blocked(ws), k)
+    assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+    assert torch.isnan(c[3]).all() and torch.isnan(c[9]).all()
+
+
+@pytest.mark.parametrize("n", [256, 1024])
+def test_fused_on_the_sweep_activation(n):
+    """The benchmark's activation (8192 x 28672 bf16 with outliers) against
+    a weight of n rows: all of C and all of Q_D(X) against the two-step path
+    on the GPU, and sampled rows of C against the oracle."""
+    x = W.sweep(seed=5)
+    xd = to_dev(x)
+    K = x.shape[1]
+    wc, ws = weight(n, K, 6)
+    wb = m.scales_to_blocked(ws)
+    c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, want_a=True)
+    qc, qs = m.quantize(xd, m.ROWS, m.RNE)
+    assert torch.equal(ac, qc) and torch.equal(as_, qs)
+    ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, K)
+    assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+    rows = np.array([0, 1, 127, 128, 4095, 4096, 8190, 8191])
+    oc, os_ = O.quantize(x[rows], O.ROWS, O.RNE, row0=0)
+    # the oracle's row quantization of sampled rows is the GPU's
+    assert np.array_equal(to_np(ac)[rows], oc) and np.array_equal(to_np(as_)[rows], os_)
+    check_against_oracle(to_np(c)[rows], oc, os_, to_np(wc), to_np(ws), K)

@@ -313,6 +313,15 @@ def check_rht(x, sign_seed, rnd, sr_seed, codes, scales, rot, row0=0):
     tol = 1e-6 * np.maximum(np.abs(y_ref), rms)
     err = np.abs(rot.astype(np.float64) - y_ref)
     assert np.all(err <= tol), "rotation error %g > tol" % (err / np.maximum(tol, 1e-300)).max()
+    # the strict per-element relative error, where the group's signed sum
+    # does not cancel (condition number sum|x| / (sqrt(32) |y|) <= 2) and y
+    # is far from the subnormals: within 1e-6 of y itself
+    cond = np.repeat(np.abs(xg).sum(axis=1) / math.sqrt(32), 32).reshape(y_ref.shape)
+    ay = np.abs(y_ref)
+    sel = (ay >= 2.0 ** -102) & (cond <= 2.0 * ay)
+    if sel.any():
+        strict = (err[sel] / ay[sel]).max()
+        assert strict <= 1e-6, "strict relative rotation error %g" % strict
     qc, qs = O.quantize(rot, O.ROWS, rnd, sr_seed, row0)
     assert_bits_equal(codes, qc, "codes of the rotated values")
     assert_bits_equal(scales, qs, "scales of the rotated values")
