@@ -63,7 +63,7 @@ NEXT_OPS = {"qema_quant": (4 + 4 + 4 + 0.5 + 1 / 32, (4096, 14336)),
             "gemm_mxf4": (None, (8192, 8192, 28672)),
             # the same with X quantized in the GEMM's load stage, against
             # quantize + blocked scales + GEMM, for W's first N rows
-            "gemm_quant_a": (None, (256, 1024, 8192))}
+            "gemm_quant_a": (None, (256, 512, 1024, 8192))}
 
 
 def alg_bytes(op):

@@ -369,7 +369,9 @@ mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
  *   a_codes   device [m][k/2], 16-byte aligned, or NULL: receives the codes
  *             of Q_D(X) in the ROWS layout
  *   a_scales  device [m][k/32], or NULL; given exactly when a_codes is
- *   status    device int or NULL, as in mxfp4_gemm
+ *   status    device int or NULL, as in mxfp4_gemm; when it is set, the
+ *             tiles of C that were not completed hold NaN or were left
+ *             unwritten
  * k must be a multiple of 256; m, n > 0 within the size limit. X is read
  * and quantized once per 256 columns of C (tiles that run together share
  * it through L2), so the fusion pays where n is small; for large n the

@@ -258,12 +258,12 @@ constexpr uint32_t kPSfCol = 256;  // per stage: 8 SFA columns, then 16 SFB
 constexpr int64_t kGroupM = 16;
 __device__ __forceinline__ void tile_coords(int64_t tile, int64_t m_tiles,
                                             int64_t nt_n, int64_t& m0,
-                                            int64_t& n0) {
+                                            int64_t& n0, int64_t rows = kGM) {
   const int64_t per_group = kGroupM * nt_n;
   const int64_t g = tile / per_group, r = tile % per_group;
   const int64_t rest = m_tiles - g * kGroupM;
   const int64_t gm = rest < kGroupM ? rest : kGroupM;
-  m0 = (g * kGroupM + r % gm) * kGM;
+  m0 = (g * kGroupM + r % gm) * rows;
   n0 = (r / gm) * kPN;
 }
 
@@ -576,65 +576,88 @@ __global__ void __launch_bounds__(kPThreads, 1)
 // (source: "Oscillation-Reduced MXFP4 Training for Vision Transformers",
 // rebuttal Question 2: the forward GEMM on Q_D(X) and Q_D(W)). B is a
 // K-major MXFP4 operand as above (the pre-quantized weight). Same tiles
-// (128 x 256), tile order, MMA issue and epilogue as k_gemm_mxf4_pipe; A
-// never exists in global memory unless asked for:
-//   warp 0:   one thread issues the TMA loads of bf16 X in half-stages of
-//             128 K-elements (two 128-byte-swizzled boxes of 64 x 128) into
-//             a kQX-deep ring, and of B's codes and scales into the operand
-//             stage;
+// (128 x 256), tile order and MMA issue as k_gemm_mxf4_pipe; A never exists
+// in global memory unless asked for:
+//   warp 0:   one thread issues the TMA loads of bf16 X in slots of
+//             128-byte-swizzled boxes of 64 columns into a kQX-deep ring;
+//   warp 2:   one thread loads B's codes and scales into the operand stage
+//             (its own thread, so that X keeps streaming while B waits for
+//             a free stage);
 //   warp 1:   tensor memory; one thread waits for both halves of a stage
 //             (B landed, A quantized) and issues the MMAs as above;
-//   warps 2-9: epilogue, 64 columns per pass (the register budget of 576
-//             threads), the accumulator released after the second pass;
-//   warps 10-17: quantizers. Per half-stage a thread quantizes the two row
-//             groups of one 128-byte X row (row = thread % 128) with the
-//             rows quantizer's own steps (bf16 absmax, OCP scale byte,
-//             product with 2^-e, nearest-even E2M1: bit-identical codes),
-//             writes the 16-byte code chunk into the operand stage at its
-//             place in the 128-byte-swizzled K-major layout of the MMA and
-//             the scale byte into the blocked tile that tcgen05.cp copies
-//             to tensor memory; then fence.proxy.async makes the stage
-//             visible to the tensor cores. The CTAs of the first column
-//             tile can also write the codes and scales to global memory in
-//             the ROWS layout of mxfp4_quantize.
+//   warps 3-18 (workers): during a tile's main loop each thread quantizes
+//             one row group of every X half-stage (row = thread % 128) with
+//             the rows quantizer's arithmetic (bf16 absmax, OCP scale byte,
+//             the product with 2^-e formed as one exact mixed-precision
+//             multiply of the bf16 input, nearest-even E2M1: bit-identical
+//             codes), writes the 16-byte code chunk into the operand stage
+//             at its place in the 128-byte-swizzled K-major layout of the
+//             MMA and the scale byte into the blocked tile that tcgen05.cp
+//             copies to tensor memory, then releases the X slot; once the
+//             first stage of the next tile is quantized (the MMAs of the
+//             previous one have drained meanwhile) the workers read the
+//             previous tile's accumulator (warp w: lane quarter w % 4,
+//             64 columns) and store it. The CTAs of the first column tile
+//             can also write the codes and scales to global memory in the
+//             ROWS layout of mxfp4_quantize.
 // X is re-read (from L2 when neighbouring CTAs share it) and re-quantized
-// once per column tile, so the fusion pays where N is small.
+// once per column tile, so the fusion pays where N is small. RT is the
+// number of X rows a tile covers: 128, or 64 when 128-row tiles would leave
+// SMs idle (a small N); then the MMA still spans 128 rows, of which the last
+// 64 are left over in shared memory and never stored, and an X slot holds a
+// whole K = 256 stage of the 64 rows.
 // ---------------------------------------------------------------------------
 
-constexpr int kQS = 2;     // operand stages (K = 256 each)
-constexpr int kQX = 3;     // X half-stages (K = 128 each)
-constexpr int kQWarps = 8;
-constexpr int kQThreads = 32 * (2 + kPEpiWarps + kQWarps);
-constexpr int kQFirst = 32 * (2 + kPEpiWarps);  // first quantizer thread
+constexpr int kQWorkers = 16;
+constexpr int kQFirstWorker = 3;   // warps 0-2: X loads, MMA, B loads
+constexpr int kQThreads = 32 * (kQFirstWorker + kQWorkers);
 
-struct __align__(1024) QaSmem {
-  uint8_t a[kQS][kGM][128];       // 128 rows x 128 bytes, 128B-swizzled
-  uint8_t b[kQS][kPN][128];
-  uint8_t x[kQX][2][kGM][128];    // two boxes of 64 bf16 x 128 rows, swizzled
-  uint8_t epi[kPEpiWarps][32][64];
-  uint8_t sfa[kQS][2][512];
-  uint8_t sfb[kQS][2][2][512];
-  unsigned long long full_b[kQS], full_a[kQS], empty[kQS], x_full[kQX], x_empty[kQX];
-  unsigned long long acc_full, acc_empty, drain;
-  uint32_t tmem_base;
-  int failed;
+// Shared memory of k_gemm_qa<RT> (byte offsets from a 1024-aligned base):
+// the X ring (kQX slots of 32 KB), the A ring (kQA stages of RT rows x 128
+// code bytes), the B ring (kQB stages of 256 rows x 128 bytes), the blocked
+// scale tiles of A and B per stage, the mbarriers. With RT = 64 the MMA
+// still reads 128 rows of A: a stage's last 64 rows are the next 8 KB of
+// shared memory (the next A stage, or the first B stage), whose products
+// land in accumulator rows that are never stored; the 8 KB saved per stage
+// buy a third B stage.
+template <int RT>
+struct QaLayout {
+  static constexpr int kQX = 3, kQA = 2, kQB = RT == 64 ? 3 : 2;
+  static constexpr uint32_t kXSlot = 2 * kGM * 128;
+  static constexpr uint32_t kAStage = RT * 128;
+  static constexpr uint32_t kBStage = kPN * 128;
+  static constexpr uint32_t kX = 0;
+  static constexpr uint32_t kA = kX + kQX * kXSlot;
+  static constexpr uint32_t kB = kA + kQA * kAStage;
+  static constexpr uint32_t kSfa = kB + kQB * kBStage;
+  static constexpr uint32_t kSfb = kSfa + kQA * 1024;
+  static constexpr uint32_t kBar = kSfb + kQB * 2048;
+  // barriers: full_b, empty_b [kQB]; full_a, empty_a [kQA]; x_full, x_empty
+  // [kQX]; acc_full, acc_empty, drain; then tmem_base and the failure flag
+  static constexpr uint32_t kFullB = kBar, kEmptyB = kFullB + 8 * kQB;
+  static constexpr uint32_t kFullA = kEmptyB + 8 * kQB, kEmptyA = kFullA + 8 * kQA;
+  static constexpr uint32_t kXFull = kEmptyA + 8 * kQA, kXEmpty = kXFull + 8 * kQX;
+  static constexpr uint32_t kAccFull = kXEmpty + 8 * kQX, kAccEmpty = kAccFull + 8;
+  static constexpr uint32_t kDrain = kAccEmpty + 8, kTmemBase = kDrain + 8;
+  static constexpr uint32_t kFailed = kTmemBase + 4;
+  static constexpr uint32_t kBytes = kFailed + 4;
+  static_assert(kA % 1024 == 0 && kB % 1024 == 0 && kAStage % 1024 == 0, "swizzle atoms");
+  static_assert(kA + (kQA - 1) * kAStage + kGM * 128 <= kSfa, "A padding rows in bounds");
 };
 
 // One 32-element group of X from its four 16-byte chunks (bf16, in order),
 // quantized as the rows quantizer does with nearest-even rounding: the code
-// chunk (element j in nibble j % 8 of word j / 8) and the scale byte.
+// chunk (element j in nibble j % 8 of word j / 8) and the scale byte. The
+// scaled values v = x 2^-e come from one mixed-precision product of the bf16
+// input with 2^-e (a normal bf16 power of two for every byte the OCP rule
+// gives), rounded once: the fp32 product the rows quantizer forms after
+// widening.
 __device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t& sb) {
-  float v[32];
   uint32_t mx[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const uint4 q = w[k];
-    v[8 * k] = bf16_lo(q.x), v[8 * k + 1] = bf16_hi(q.x);
-    v[8 * k + 2] = bf16_lo(q.y), v[8 * k + 3] = bf16_hi(q.y);
-    v[8 * k + 4] = bf16_lo(q.z), v[8 * k + 5] = bf16_hi(q.z);
-    v[8 * k + 6] = bf16_lo(q.w), v[8 * k + 7] = bf16_hi(q.w);
-    mx[2 * k] = bf16x2_absmax_nan(q.x, q.y);
-    mx[2 * k + 1] = bf16x2_absmax_nan(q.z, q.w);
+    mx[2 * k] = bf16x2_absmax_nan(w[k].x, w[k].y);
+    mx[2 * k + 1] = bf16x2_absmax_nan(w[k].z, w[k].w);
   }
 #pragma unroll
   for (int n = 4; n >= 1; n /= 2)
@@ -642,155 +665,164 @@ __device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t
     for (int i = 0; i < n; ++i) mx[i] = bf16x2_absmax_nan(mx[i], mx[i + n]);
   const uint32_t mm = mx[0] & 0x7FFF7FFFu;
   sb = scale_byte(max(mm << 16, mm & 0xFFFF0000u));
-  const float mul = inv_scale(sb);
+  const unsigned short s16 = bf16_inv_scale(sb);
+  uint32_t out[4];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] *= mul;
-  uint4 out;
-  out.x = e2m1x8_rn(v);
-  out.y = e2m1x8_rn(v + 8);
-  out.z = e2m1x8_rn(v + 16);
-  out.w = e2m1x8_rn(v + 24);
-  if (sb == 0xFFu) out = make_uint4(0, 0, 0, 0);
-  return out;
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t* q = reinterpret_cast<const uint32_t*>(&w[k]);
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      v[2 * t] = bf16lo_mul(q[t], s16);
+      v[2 * t + 1] = bf16hi_mul(q[t], s16);
+    }
+    out[k] = e2m1x8_rn(v);
+  }
+  if (sb == 0xFFu) return make_uint4(0, 0, 0, 0);
+  return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+template <int RT>
 __global__ void __launch_bounds__(kQThreads, 1)
     k_gemm_qa(const __grid_constant__ CUtensorMap tm_x,
               const __grid_constant__ CUtensorMap tm_b,
-              const __grid_constant__ CUtensorMap tm_c, bool tma_store,
               const uint8_t* __restrict__ sfb, int64_t m, int64_t n, int64_t k,
               float* __restrict__ c, uint8_t* __restrict__ a_codes,
               uint8_t* __restrict__ a_scales, int* __restrict__ status) {
+  using L = QaLayout<RT>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  QaSmem& sm = *reinterpret_cast<QaSmem*>(
-      smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  uint8_t* const sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  auto bar = [&](uint32_t off, int i) {
+    return reinterpret_cast<unsigned long long*>(sm + off) + i;
+  };
+  int* const failed = reinterpret_cast<int*>(sm + L::kFailed);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t k_tiles = k / 128;
   const int64_t n_kb = k / 256;
   const int64_t n_row_tiles = (n + 127) / 128;
-  const int64_t m_tiles = (m + kGM - 1) / kGM;
+  const int64_t m_tiles = (m + RT - 1) / RT;
   const int64_t n_col_tiles = (n + kPN - 1) / kPN;
   const int64_t n_tiles = m_tiles * n_col_tiles;
+  // X slots per K = 256 stage, 64-column boxes per slot, K-elements per slot
+  constexpr int kSlots = RT == 128 ? 2 : 1;
+  constexpr int kBoxes = 4 / kSlots;
+  constexpr int kSlotK = 256 / kSlots;
+  static_assert(RT * 128 * kBoxes == L::kXSlot, "X slot size");
 
   if (tid == 0) {
-    for (int s = 0; s < kQS; ++s) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.full_b[s])));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.full_a[s])),
-                   "r"(kQWarps));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.empty[s])));
-    }
-    for (int h = 0; h < kQX; ++h) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.x_full[h])));
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.x_empty[h])),
-                   "r"(kQWarps));
-    }
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.acc_full)));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&sm.acc_empty)),
-                 "r"(kPEpiWarps));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&sm.drain)));
+    auto init = [&](uint32_t off, int i, uint32_t count) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar(off, i))),
+                   "r"(count));
+    };
+    for (int i = 0; i < L::kQB; ++i) init(L::kFullB, i, 1), init(L::kEmptyB, i, 1);
+    for (int i = 0; i < L::kQA; ++i) init(L::kFullA, i, kQWorkers), init(L::kEmptyA, i, 1);
+    for (int i = 0; i < L::kQX; ++i) init(L::kXFull, i, 1), init(L::kXEmpty, i, kQWorkers);
+    init(L::kAccFull, 0, 1);
+    init(L::kAccEmpty, 0, kQWorkers);
+    init(L::kDrain, 0, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    sm.failed = 0;
+    *failed = 0;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(&sm.tmem_base)), "r"(kPTmemCols));
+                 ::"r"(smem_u32(sm + L::kTmemBase)), "r"(kPTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;");
-  const uint32_t tmem = sm.tmem_base;
+  const uint32_t tmem = *reinterpret_cast<const uint32_t*>(sm + L::kTmemBase);
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 2) {
+    // warp 0: X into its ring; warp 2: B into its ring. Two threads, so
+    // that neither ring waits on the other's consumer.
     if (lane == 0) {
-      uint32_t s = 0, ph = 0, xs = 0, xph = 0;
-      // rings with a load issued, and the phase parity of each slot's last
+      const bool loads_x = warp == 0;
+      const int ring = loads_x ? L::kQX : L::kQB;
+      uint32_t s = 0, ph = 0;
+      // slots with a load issued, and the phase parity of each one's last
       // load: every load lands before the CTA ends
-      uint32_t issued_b = 0, last_b = 0, issued_x = 0, last_x = 0;
+      uint32_t issued = 0, last = 0;
       bool stop = false;
       for (int64_t tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
         int64_t m0, n0;
-        tile_coords(tile, m_tiles, n_col_tiles, m0, n0);
+        tile_coords(tile, m_tiles, n_col_tiles, m0, n0, RT);
         const int64_t rb = n0 / 128;
         const bool half1 = rb + 1 < n_row_tiles;
-        const uint32_t bbytes = kPN * 128 + (half1 ? 2048 : 1024);
+        const uint32_t bbytes = L::kBStage + (half1 ? 2048 : 1024);
         const uint8_t* pb0 = sfb + rb * k_tiles * 512;
         const uint8_t* pb1 = pb0 + k_tiles * 512;
         for (int64_t kb = 0; kb < n_kb && !stop; ++kb) {
-          for (int h = 0; h < 2; ++h) {
-            if (!wait_parity_or_failed<false>(&sm.x_empty[xs], xph ^ 1u, &sm.failed)) {
+          for (int h = 0; h < (loads_x ? kSlots : 1); ++h) {
+            if (!wait_parity_or_failed<false>(bar(loads_x ? L::kXEmpty : L::kEmptyB, s),
+                                              ph ^ 1u, failed)) {
               stop = true;
               break;
             }
-            issued_x |= 1u << xs;
-            last_x = (last_x & ~(1u << xs)) | (xph << xs);
-            expect_tx(&sm.x_full[xs], 2 * kGM * 128);
+            issued |= 1u << s;
+            last = (last & ~(1u << s)) | (ph << s);
+            if (loads_x) {
+              unsigned long long* full = bar(L::kXFull, s);
+              expect_tx(full, L::kXSlot);
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
-              tma_load_2d(&sm.x[xs][j][0][0], &tm_x, int((kb * 256 + 128 * h + 64 * j) * 2),
-                          int(m0), &sm.x_full[xs]);
-            if (++xs == kQX) {
-              xs = 0;
-              xph ^= 1u;
+              for (int j = 0; j < kBoxes; ++j)
+                tma_load_2d(sm + L::kX + s * L::kXSlot + j * RT * 128, &tm_x,
+                            int((kb * 256 + kSlotK * h + 64 * j) * 2), int(m0), full);
+            } else {
+              unsigned long long* full = bar(L::kFullB, s);
+              uint8_t* sfb_s = sm + L::kSfb + s * 2048;
+              expect_tx(full, bbytes);
+              tma_load_2d(sm + L::kB + s * L::kBStage, &tm_b, int(kb) * 128, int(n0), full);
+              bulk_load(sfb_s, pb0 + kb * 1024, 1024, full);
+              if (half1) bulk_load(sfb_s + 1024, pb1 + kb * 1024, 1024, full);
+            }
+            if (++s == uint32_t(ring)) {
+              s = 0;
+              ph ^= 1u;
             }
           }
-          if (stop) break;
-          if (!wait_parity_or_failed<false>(&sm.empty[s], ph ^ 1u, &sm.failed)) {
-            stop = true;
-            break;
-          }
-          issued_b |= 1u << s;
-          last_b = (last_b & ~(1u << s)) | (ph << s);
-          expect_tx(&sm.full_b[s], bbytes);
-          tma_load_2d(&sm.b[s][0][0], &tm_b, int(kb) * 128, int(n0), &sm.full_b[s]);
-          bulk_load(&sm.sfb[s][0][0][0], pb0 + kb * 1024, 1024, &sm.full_b[s]);
-          if (half1) bulk_load(&sm.sfb[s][1][0][0], pb1 + kb * 1024, 1024, &sm.full_b[s]);
-          if (++s == kQS) {
-            s = 0;
-            ph ^= 1u;
-          }
         }
-        if (failed_flag(&sm.failed)) stop = true;
+        if (failed_flag(failed)) stop = true;
       }
-      if (stop) atomicExch(&sm.failed, 1);
+      if (stop) atomicExch(failed, 1);
       // drain (immediate unless a wait ran out)
-      for (uint32_t st = 0; st < kQX; ++st)
-        if ((issued_x >> st) & 1u) wait_parity(&sm.x_full[st], (last_x >> st) & 1u);
-      for (uint32_t st = 0; st < kQS; ++st)
-        if ((issued_b >> st) & 1u) wait_parity(&sm.full_b[st], (last_b >> st) & 1u);
+      for (int st = 0; st < ring; ++st)
+        if ((issued >> st) & 1u)
+          wait_parity(bar(loads_x ? L::kXFull : L::kFullB, st), (last >> st) & 1u);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t sf = tmem + kPSfCol;
-      const uint64_t a_d0 = smem_desc_sw128(&sm.a[0][0][0]);
-      const uint64_t b_d0 = smem_desc_sw128(&sm.b[0][0][0]);
-      const uint64_t sfa_d0 = smem_desc(&sm.sfa[0][0][0], 16, 128);
-      const uint64_t sfb_d0 = smem_desc(&sm.sfb[0][0][0][0], 16, 128);
-      constexpr uint32_t kAStep = (kGM * 128) >> 4, kBStep = (kPN * 128) >> 4;
+      const uint64_t a_d0 = smem_desc_sw128(sm + L::kA);
+      const uint64_t b_d0 = smem_desc_sw128(sm + L::kB);
+      const uint64_t sfa_d0 = smem_desc(sm + L::kSfa, 16, 128);
+      const uint64_t sfb_d0 = smem_desc(sm + L::kSfb, 16, 128);
+      constexpr uint32_t kAStep = L::kAStage >> 4, kBStep = L::kBStage >> 4;
       constexpr uint32_t kSfaStep = 1024 >> 4, kSfbStep = 2048 >> 4, kSfTile = 512 >> 4;
-      uint32_t s = 0, ph = 0;
+      uint32_t sa = 0, pha = 0, sb = 0, phb = 0;
       int64_t ti = 0;
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
-        if (!wait_parity_or_failed<false>(&sm.acc_empty, uint32_t(ti & 1) ^ 1u, &sm.failed) ||
-            failed_flag(&sm.failed)) {
+        if (!wait_parity_or_failed<false>(bar(L::kAccEmpty, 0), uint32_t(ti & 1) ^ 1u,
+                                          failed) ||
+            failed_flag(failed)) {
           ok = false;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;");
         for (int64_t kb = 0; kb < n_kb; ++kb) {
-          if (!wait_parity_or_failed<false>(&sm.full_b[s], ph, &sm.failed) ||
-              !wait_parity_or_failed<false>(&sm.full_a[s], ph, &sm.failed)) {
+          if (!wait_parity_or_failed<false>(bar(L::kFullB, sb), phb, failed) ||
+              !wait_parity_or_failed<false>(bar(L::kFullA, sa), pha, failed)) {
             ok = false;
             break;
           }
           asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            copy_scales_desc(sf + 4 * j, sfa_d0 + (s * kSfaStep + j * kSfTile));
-            copy_scales_desc(sf + 8 + 8 * j, sfb_d0 + (s * kSfbStep + j * kSfTile));
-            copy_scales_desc(sf + 8 + 8 * j + 4, sfb_d0 + (s * kSfbStep + (2 + j) * kSfTile));
+            copy_scales_desc(sf + 4 * j, sfa_d0 + (sa * kSfaStep + j * kSfTile));
+            copy_scales_desc(sf + 8 + 8 * j, sfb_d0 + (sb * kSfbStep + j * kSfTile));
+            copy_scales_desc(sf + 8 + 8 * j + 4, sfb_d0 + (sb * kSfbStep + (2 + j) * kSfTile));
           }
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -798,160 +830,145 @@ __global__ void __launch_bounds__(kQThreads, 1)
             const uint32_t idesc = kIdescN256 | (sf_id << 29) | (sf_id << 4);
             const uint32_t tsfa = (sf + 4 * (t >> 1)) | (sf_id << 30);
             const uint32_t tsfb = (sf + 8 + 8 * (t >> 1)) | (sf_id << 30);
-            mma_mxf4(tmem, a_d0 + (s * kAStep + 2 * t), b_d0 + (s * kBStep + 2 * t), idesc,
+            mma_mxf4(tmem, a_d0 + (sa * kAStep + 2 * t), b_d0 + (sb * kBStep + 2 * t), idesc,
                      (kb == 0 && t == 0) ? 0u : 1u, tsfa, tsfb);
           }
-          commit_to(&sm.empty[s]);
-          if (++s == kQS) {
-            s = 0;
-            ph ^= 1u;
+          commit_to(bar(L::kEmptyA, sa));
+          commit_to(bar(L::kEmptyB, sb));
+          if (++sa == uint32_t(L::kQA)) {
+            sa = 0;
+            pha ^= 1u;
+          }
+          if (++sb == uint32_t(L::kQB)) {
+            sb = 0;
+            phb ^= 1u;
           }
         }
-        if (!ok) atomicExch(&sm.failed, 1);
-        commit_to(&sm.acc_full);
+        if (!ok) atomicExch(failed, 1);
+        commit_to(bar(L::kAccFull, 0));
       }
-      if (!ok) atomicExch(&sm.failed, 1);
+      if (!ok) atomicExch(failed, 1);
       // drain: every MMA and scale copy issued has completed
-      commit_to(&sm.drain);
-      if (!wait_parity(&sm.drain, 0)) atomicExch(&sm.failed, 1);
+      commit_to(bar(L::kDrain, 0));
+      if (!wait_parity(bar(L::kDrain, 0), 0)) atomicExch(failed, 1);
     }
     __syncwarp();
-  } else if (warp < 2 + kPEpiWarps) {
-    // epilogue: two warps per lane quarter, 128 columns each in two passes
+  } else {
+    // workers: thread qt quantizes row qt % RT, group qt / RT of every X
+    // slot; warp w stores lane quarter w % 4, columns 64 ((w - 3) / 4) of
+    // every accumulator
+    const int qt = tid - 32 * kQFirstWorker;
+    const int r = qt % RT;
+    const int g = qt / RT;             // group of the slot: box g / 2, group g % 2 of it
+    const uint32_t sw = uint32_t(r & 7);
+    const uint8_t* xrow = sm + L::kX + (g >> 1) * RT * 128 + r * 128;
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
-    int64_t ti = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++ti) {
-      int64_t m0, n0;
-      tile_coords(tile, m_tiles, n_col_tiles, m0, n0);
-      // after a failure the warp skips the tensor memory and the barriers
-      // and writes NaN over the rest of its tiles
-      const bool ok = __all_sync(0xFFFFFFFFu, !failed_flag(&sm.failed) &&
-                                                  wait_parity(&sm.acc_full, uint32_t(ti & 1),
-                                                              kAccWaitLimit));
-      if (!ok) atomicExch(&sm.failed, 1);
-      if (ok) asm volatile("tcgen05.fence::after_thread_sync;");
+    const int cblk = (warp - kQFirstWorker) >> 2;
+    uint32_t s = 0, ph = 0, xs = 0, xph = 0;
+    bool ok = true;
+    int64_t pend_ti = -1, pend_m0 = 0, pend_n0 = 0;
+
+    // the accumulator of tile ti (origin m0, n0) to C; after a failure,
+    // NaN without touching tensor memory or the barriers
+    auto drain_tile = [&](int64_t ti, int64_t m0, int64_t n0) {
+      const bool got = __all_sync(0xFFFFFFFFu, !failed_flag(failed) &&
+                                                   wait_parity(bar(L::kAccFull, 0),
+                                                               uint32_t(ti & 1),
+                                                               kAccWaitLimit));
+      if (!got) atomicExch(failed, 1);
+      uint32_t v[64];
+      if (got) {
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + 64u * uint32_t(cblk);
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+          uint32_t* d = v + 32 * cb;
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
+              "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
+              "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+              : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]),
+                "=r"(d[5]), "=r"(d[6]), "=r"(d[7]), "=r"(d[8]), "=r"(d[9]),
+                "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]),
+                "=r"(d[15]), "=r"(d[16]), "=r"(d[17]), "=r"(d[18]), "=r"(d[19]),
+                "=r"(d[20]), "=r"(d[21]), "=r"(d[22]), "=r"(d[23]), "=r"(d[24]),
+                "=r"(d[25]), "=r"(d[26]), "=r"(d[27]), "=r"(d[28]), "=r"(d[29]),
+                "=r"(d[30]), "=r"(d[31])
+              : "r"(tbase + 32u * uint32_t(cb)));
+        }
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;");
+        __syncwarp();
+        if (lane == 0)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
+                           smem_u32(bar(L::kAccEmpty, 0)))
+                       : "memory");
+      }
+      if (!got || failed_flag(failed)) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) v[j] = kNaNf32;
+      }
       const int64_t row = m0 + 32 * q + lane;
-#pragma unroll 1
-      for (int pass = 0; pass < 2; ++pass) {
-        const int64_t col0 = n0 + 128 * half + 64 * pass;
-        uint32_t v[64];
-        if (ok) {
-          const uint32_t tbase =
-              tmem + (uint32_t(32 * q) << 16) + 128u * uint32_t(half) + 64u * uint32_t(pass);
+      const int64_t col0 = n0 + 64 * cblk;
+      if (32 * q + lane < RT && row < m && col0 < n) {
+        float* out = c + row * n + col0;
+        if (col0 + 64 <= n && (n & 3) == 0) {
 #pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
-            uint32_t* d = v + 32 * cb;
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, "
-                "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
-                "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]),
-                  "=r"(d[5]), "=r"(d[6]), "=r"(d[7]), "=r"(d[8]), "=r"(d[9]),
-                  "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]),
-                  "=r"(d[15]), "=r"(d[16]), "=r"(d[17]), "=r"(d[18]), "=r"(d[19]),
-                  "=r"(d[20]), "=r"(d[21]), "=r"(d[22]), "=r"(d[23]), "=r"(d[24]),
-                  "=r"(d[25]), "=r"(d[26]), "=r"(d[27]), "=r"(d[28]), "=r"(d[29]),
-                  "=r"(d[30]), "=r"(d[31])
-                : "r"(tbase + 32u * uint32_t(cb)));
-          }
-          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-          if (pass == 1) {  // the accumulator is read: release it
-            asm volatile("tcgen05.fence::before_thread_sync;");
-            __syncwarp();
-            if (lane == 0)
-              asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                               smem_u32(&sm.acc_empty))
-                           : "memory");
-          }
-        }
-        if (!ok || failed_flag(&sm.failed)) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = kNaNf32;
-        }
-        if (tma_store) {
-          // 4 boxes of 32 rows x 16 fp32 through this warp's staging tile
-          // (64-byte swizzle, as in k_gemm_mxf4_pipe)
-          uint8_t* st = &sm.epi[warp - 2][0][0];
-#pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            if (lane == 0) bulk_wait_read();
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<uint4*>(st + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                  make_uint4(v[16 * cb + 4 * j], v[16 * cb + 4 * j + 1],
-                             v[16 * cb + 4 * j + 2], v[16 * cb + 4 * j + 3]);
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0 && col0 + 16 * cb < n && m0 + 32 * q < m)
-              tma_store_2d(&tm_c, int(col0 + 16 * cb), int(m0 + 32 * q), st);
-          }
-        } else if (row < m && col0 < n) {
-          float* out = c + row * n + col0;
+          for (int j = 0; j < 64; j += 4)
+            *reinterpret_cast<uint4*>(out + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        } else {
 #pragma unroll
           for (int j = 0; j < 64; ++j)
             if (col0 + j < n) out[j] = __uint_as_float(v[j]);
         }
       }
-    }
-  } else {
-    // quantizers: thread qt takes row qt % 128 and box qt / 128 (two groups)
-    // of every X half-stage
-    const int qt = tid - kQFirst;
-    const int r = qt & (kGM - 1);
-    const int box = qt >> 7;
-    const uint32_t sw = uint32_t(r & 7);
-    uint32_t s = 0, ph = 0, xs = 0, xph = 0;
-    bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+    };
+
+    int64_t ti = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
       int64_t m0, n0;
-      tile_coords(tile, m_tiles, n_col_tiles, m0, n0);
+      tile_coords(tile, m_tiles, n_col_tiles, m0, n0, RT);
       const int64_t row = m0 + r;
       const bool to_global = n0 == 0 && a_codes != nullptr && row < m;
       for (int64_t kb = 0; kb < n_kb; ++kb) {
-        // the operand stage is free once the MMAs of its last use completed
+        // the A stage is free once the MMAs of its last use completed
         if (!__all_sync(0xFFFFFFFFu,
-                        wait_parity_or_failed<false>(&sm.empty[s], ph ^ 1u, &sm.failed))) {
+                        wait_parity_or_failed<false>(bar(L::kEmptyA, s), ph ^ 1u, failed))) {
           ok = false;
           break;
         }
-        for (int h = 0; h < 2; ++h) {
+        uint8_t* const a_s = sm + L::kA + s * L::kAStage;
+        uint8_t* const sfa_s = sm + L::kSfa + s * 1024;
+        for (int h = 0; h < kSlots; ++h) {
           if (!__all_sync(0xFFFFFFFFu,
-                          wait_parity_or_failed<false>(&sm.x_full[xs], xph, &sm.failed))) {
+                          wait_parity_or_failed<false>(bar(L::kXFull, xs), xph, failed))) {
             ok = false;
             break;
           }
-          const uint8_t* xr = &sm.x[xs][box][r][0];
-          uint4 w[2][4];
+          const uint8_t* xr = xrow + xs * L::kXSlot;
+          uint4 w[4];
 #pragma unroll
-          for (int i = 0; i < 2; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              w[i][j] = *reinterpret_cast<const uint4*>(xr + (((4 * i + j) ^ sw) << 4));
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            uint32_t sb;
-            const uint4 code = qa_quantize_group(w[i], sb);
-            const int G = 4 * h + 2 * box + i;  // group within the stage's 256
-            *reinterpret_cast<uint4*>(&sm.a[s][r][(uint32_t(G) ^ sw) << 4]) = code;
-            sm.sfa[s][G >> 2][16 * (r & 31) + 4 * (r >> 5) + (G & 3)] = uint8_t(sb);
-            if (to_global) {
-              *reinterpret_cast<uint4*>(a_codes + row * (k / 2) + kb * 128 + 16 * G) = code;
-              a_scales[row * (k / 32) + kb * 8 + G] = uint8_t(sb);
-            }
+          for (int j = 0; j < 4; ++j)
+            w[j] = *reinterpret_cast<const uint4*>(xr + (((4 * (g & 1) + j) ^ sw) << 4));
+          uint32_t scb;
+          const uint4 code = qa_quantize_group(w, scb);
+          const int G = (8 / kSlots) * h + g;  // group within the stage's 256
+          *reinterpret_cast<uint4*>(a_s + r * 128 + ((uint32_t(G) ^ sw) << 4)) = code;
+          sfa_s[512 * (G >> 2) + 16 * (r & 31) + 4 * (r >> 5) + (G & 3)] = uint8_t(scb);
+          if (to_global) {
+            *reinterpret_cast<uint4*>(a_codes + row * (k / 2) + kb * 128 + 16 * G) = code;
+            a_scales[row * (k / 32) + kb * 8 + G] = uint8_t(scb);
           }
           // release the X slot after the stores that depend on every value
-          // loaded from it: the stores cannot issue before the loads have
-          // returned, and the arrival (a release) is ordered after the
-          // stores, so the next TMA load into the slot cannot overwrite data
-          // still being read
+          // loaded from it: a thread's arrival does not wait for its shared
+          // loads to return, so releasing right after issuing them let the
+          // next TMA load into the slot overwrite data still being read
           __syncwarp();
           if (lane == 0)
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                             smem_u32(&sm.x_empty[xs]))
+                             smem_u32(bar(L::kXEmpty, xs)))
                          : "memory");
-          if (++xs == kQX) {
+          if (++xs == uint32_t(L::kQX)) {
             xs = 0;
             xph ^= 1u;
           }
@@ -962,20 +979,29 @@ __global__ void __launch_bounds__(kQThreads, 1)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0)
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sm.full_a[s]))
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
+                           smem_u32(bar(L::kFullA, s)))
                        : "memory");
-        if (++s == kQS) {
+        if (++s == uint32_t(L::kQA)) {
           s = 0;
           ph ^= 1u;
         }
+        // the previous tile's accumulator, once this tile's first stage is
+        // on its way: its MMAs have drained meanwhile
+        if (kb == 0 && pend_ti >= 0) {
+          drain_tile(pend_ti, pend_m0, pend_n0);
+          pend_ti = -1;
+        }
       }
+      if (!ok) break;
+      pend_ti = ti, pend_m0 = m0, pend_n0 = n0;
     }
-    if (!ok) atomicExch(&sm.failed, 1);
+    if (!ok) atomicExch(failed, 1);
+    if (pend_ti >= 0) drain_tile(pend_ti, pend_m0, pend_n0);
   }
-  if (warp >= 2 && warp < 2 + kPEpiWarps && lane == 0) bulk_wait_all();  // C stores complete
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
-  report_failure(status, &sm.failed);
+  report_failure(status, failed);
   if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
                  ::"r"(tmem), "r"(kPTmemCols));
@@ -1045,28 +1071,43 @@ cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
   return cudaGetLastError();
 }
 
+namespace {
+
+template <int RT>
+cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, const uint8_t* b,
+                         const uint8_t* b_scales, float* c, uint8_t* a_codes,
+                         uint8_t* a_scales, int* status, cudaStream_t s) {
+  // X as a byte array [m][2k] for the TMA: 128-byte boxes of 64 bf16
+  CUtensorMap mx, mb;
+  if (!encode_rows_sw128(&mx, x, m, 2 * k, RT) || !encode_codes_map(&mb, b, n, k, kPN))
+    return cudaErrorInvalidValue;
+  constexpr size_t smem = QaLayout<RT>::kBytes + 1024;
+  static_assert(smem <= 227 * 1024, "fused GEMM shared memory");
+  auto kern = k_gemm_qa<RT>;
+  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((m + RT - 1) / RT) * ((n + kPN - 1) / kPN);
+  const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kQThreads, smem, tiles);
+  kern<<<grid, kQThreads, smem, s>>>(mx, mb, b_scales, m, n, k, c, a_codes, a_scales, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k,
                            const uint8_t* b, const uint8_t* b_scales, float* c,
                            uint8_t* a_codes, uint8_t* a_scales, int* status,
                            cudaStream_t s) {
   if (k % 256) return cudaErrorInvalidValue;
-  // X as a byte array [m][2k] for the TMA: 128-byte boxes of 64 bf16
-  CUtensorMap mx, mb, mc;
-  if (!encode_rows_sw128(&mx, x, m, 2 * k, kGM) || !encode_codes_map(&mb, b, n, k, kPN))
-    return cudaErrorInvalidValue;
-  const bool tma_store = encode_c_map(&mc, c, m, n);
-  if (!tma_store) mc = mb;  // unused
-  constexpr size_t smem = sizeof(QaSmem) + 1024;
-  static_assert(smem <= 227 * 1024, "fused GEMM shared memory");
-  cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(k_gemm_qa),
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  const int64_t tiles = ((m + kGM - 1) / kGM) * ((n + kPN - 1) / kPN);
-  const int grid =
-      persistent_grid(reinterpret_cast<const void*>(k_gemm_qa), kQThreads, smem, tiles);
-  k_gemm_qa<<<grid, kQThreads, smem, s>>>(mx, mb, mc, tma_store, b_scales, m, n, k, c,
-                                          a_codes, a_scales, status);
-  return cudaGetLastError();
+  // 64-row tiles where 128-row ones would not give every SM a tile
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles128 = ((m + 127) / 128) * ((n + kPN - 1) / kPN);
+  return tiles128 < sms
+             ? gemm_qa_impl<64>(x, m, n, k, b, b_scales, c, a_codes, a_scales, status, s)
+             : gemm_qa_impl<128>(x, m, n, k, b, b_scales, c, a_codes, a_scales, status, s);
 }
 
 }  // namespace mxfp4
