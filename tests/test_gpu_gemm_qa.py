@@ -44,7 +44,11 @@ def check_against_oracle(c, xc, xs, wc, ws, k, rows=None):
                                  (200, 136, 512),    # ragged rows and columns
                                  (384, 520, 768),    # 3 x 3 tiles, a 8-column edge tile
                                  (1000, 64, 1024),   # narrow output, many row tiles
-                                 (256, 768, 2560)])  # 10 stages: the rings wrap
+                                 (256, 768, 2560),   # 10 stages: the rings wrap
+                                 # several tiles per CTA with one stage each (the
+                                 # accumulator drained after the next tile's only
+                                 # stage): 64-row tiles, then 128-row tiles
+                                 (9000, 512, 256), (20000, 520, 256)])
 def test_fused_equals_quantize_then_gemm(mnk):
     mm, nn, k = mnk
     x = W.normal_bf16(mm, k, 21, 0.005, 50.0)
@@ -86,7 +90,7 @@ def test_special_values_follow_the_quantizer():
     assert torch.isnan(c[3]).all() and torch.isnan(c[9]).all()
 
 
-@pytest.mark.parametrize("n", [256, 1024])
+@pytest.mark.parametrize("n", [256, 512, 1024])
 def test_fused_on_the_sweep_activation(n):
     """The benchmark's activation (8192 x 28672 bf16 with outliers) against
     a weight of n rows: all of C and all of Q_D(X) against the two-step path
