@@ -678,6 +678,20 @@ def run_ours(args):
                     "TFLOP_s": flops / d_fused / 1e12, "shape": [gM, nn, gK],
                     "launches": args.steps,
                     "x_read_GB_s": 2.0 * gM * gK / d_fused / 1e9}
+                if nn == NEXT_OPS["gemm_quant_a"][1][0]:
+                    # the same with stochastic rounding (a gradient operand)
+                    d_fs = timed_alone(lambda: m.gemm_quantize_a(buf0["x"], bcn, bbn, m.SR,
+                                                                 SEED, out=outn))
+
+                    def two_step_sr():
+                        m.quantize(buf0["x"], m.ROWS, m.SR, SEED, out=qout)
+                        m.scales_to_blocked(qout[1], out=qblk)
+                        m.gemm(qout[0], qblk, bcn, bbn, gK, out=outn)
+                    d_ts = timed_alone(two_step_sr)
+                    next_ops["gemm_quant_a_sr_n%d" % nn] = {
+                        "us": d_fs * 1e6, "two_step_us": d_ts * 1e6,
+                        "speedup_vs_two_step": d_ts / d_fs, "shape": [gM, nn, gK],
+                        "launches": args.steps}
                 del bcn, bbn, outn
             del qout, qblk
             del ac, as_, bc, bs, ab, bb, gout

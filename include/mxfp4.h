@@ -353,21 +353,25 @@ mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                         int* status, void* stream);
 
 /*
- * Forward GEMM with the activation quantized in the GEMM's load stage:
- *   C[m][n] = sum_k Q_D(X)[m][k] * B[n][k]      (fp32 accumulate, fp32 out)
- * Q_D(X) is the 1x32 nearest-even quantization of X along k (ROWS), the
- * one mxfp4_quantize(x, MXFP4_BF16, m, k, MXFP4_ROWS, MXFP4_RNE, ...)
- * computes; B is given as in mxfp4_gemm (the pre-quantized weight). The
+ * GEMM with the activation quantized in the GEMM's load stage:
+ *   C[m][n] = sum_k Q(X)[m][k] * B[n][k]        (fp32 accumulate, fp32 out)
+ * Q(X) is the 1x32 quantization of X along k (ROWS) with `rounding`: RNE
+ * (Q_D, the forward GEMM Q_D(X) Q_D(W)^T) or SR (Q_S keyed by `seed`, e.g.
+ * a gradient quantized for a backward GEMM), exactly as mxfp4_quantize(x,
+ * MXFP4_BF16, m, k, MXFP4_ROWS, rounding, seed, ...) computes it; B is given
+ * as in mxfp4_gemm (for the forward GEMM the pre-quantized weight). The
  * result equals that quantization followed by mxfp4_scales_to_blocked and
- * mxfp4_gemm, bit for bit, but Q_D(X) never passes through global memory:
+ * mxfp4_gemm, bit for bit, but Q(X) never passes through global memory:
  * bf16 X tiles are quantized in shared memory into the tensor cores'
  * operand layout. Source: "Oscillation-Reduced MXFP4 Training for Vision
- * Transformers", rebuttal Question 2 (the forward GEMM Q_D(X) Q_D(W)^T).
+ * Transformers", rebuttal Question 2 (Q_D(X) Q_D(W)^T in the forward pass,
+ * Q_S in the backward pass).
  *   x         device bf16 [m][k], 16-byte aligned, read only
+ *   rounding  MXFP4_RNE or MXFP4_SR; seed keys SR (ignored for RNE)
  *   b_codes, b_scales  as in mxfp4_gemm, n rows
  *   c         device fp32 [m][n], written (every element)
  *   a_codes   device [m][k/2], 16-byte aligned, or NULL: receives the codes
- *             of Q_D(X) in the ROWS layout
+ *             of Q(X) in the ROWS layout
  *   a_scales  device [m][k/32], or NULL; given exactly when a_codes is
  *   status    device int or NULL, as in mxfp4_gemm; when it is set, the
  *             tiles of C that were not completed hold NaN or were left
@@ -378,9 +382,9 @@ mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
  * separate quantize + mxfp4_gemm is faster.
  */
 mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t k,
-                                   const uint8_t* b_codes, const uint8_t* b_scales,
-                                   float* c, uint8_t* a_codes, uint8_t* a_scales,
-                                   int* status, void* stream);
+                                   int rounding, uint64_t seed, const uint8_t* b_codes,
+                                   const uint8_t* b_scales, float* c, uint8_t* a_codes,
+                                   uint8_t* a_scales, int* status, void* stream);
 
 /* Static text for a status code; never NULL. */
 const char* mxfp4_status_string(int status);

@@ -73,8 +73,8 @@ def lib():
                                  ctypes.c_float, i64, vp, vp],
             "mxfp4_scales_to_blocked": [vp, i64, i64, vp, vp],
             "mxfp4_gemm": [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp],
-            "mxfp4_gemm_quantize_a": [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp,
-                                      vp],
+            "mxfp4_gemm_quantize_a": [vp, i64, i64, i64, i32, u64, vp, vp, vp, vp,
+                                      vp, vp, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -365,12 +365,13 @@ def gemm(a_codes, a_blocked, b_codes, b_blocked, k, out=None, stream=None, statu
     return out
 
 
-def gemm_quantize_a(x, b_codes, b_blocked, out=None, want_a=False, stream=None,
-                    status=None):
-    """mxfp4_gemm_quantize_a: C = Q_D(x) B^T in fp32, x bf16 [m, k] (k a
-    multiple of 256) quantized 1x32 nearest-even inside the GEMM's load
-    stage, B given as K-major codes [n, k/2] and blocked scales. Returns C,
-    or (C, a_codes, a_scales) with want_a (Q_D(x) in the ROWS layout)."""
+def gemm_quantize_a(x, b_codes, b_blocked, rounding=RNE, seed=0, out=None, want_a=False,
+                    stream=None, status=None):
+    """mxfp4_gemm_quantize_a: C = Q(x) B^T in fp32, x bf16 [m, k] (k a
+    multiple of 256) quantized 1x32 (rounding RNE, or SR keyed by seed)
+    inside the GEMM's load stage, B given as K-major codes [n, k/2] and
+    blocked scales. Returns C, or (C, a_codes, a_scales) with want_a (Q(x)
+    in the ROWS layout)."""
     _cuda2d(x, "x")
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bfloat16")
@@ -397,8 +398,8 @@ def gemm_quantize_a(x, b_codes, b_blocked, out=None, want_a=False, stream=None,
         _buffer(ac, "a_codes", torch.uint8, m * k // 2, d)
         _buffer(as_, "a_scales", torch.uint8, m * k // 32, d)
     st = _status_word(status, d)
-    _check(lib().mxfp4_gemm_quantize_a(_ptr(x), m, n, k, _ptr(b_codes), _ptr(b_blocked),
-                                       _ptr(c), _ptr(ac), _ptr(as_), st,
+    _check(lib().mxfp4_gemm_quantize_a(_ptr(x), m, n, k, rounding, seed, _ptr(b_codes),
+                                       _ptr(b_blocked), _ptr(c), _ptr(ac), _ptr(as_), st,
                                        _stream(d, stream)), "mxfp4_gemm_quantize_a")
     return out
 

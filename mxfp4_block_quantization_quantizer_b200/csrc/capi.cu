@@ -241,9 +241,10 @@ mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
 }
 
 mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t k,
-                                   const uint8_t* b_codes, const uint8_t* b_scales,
-                                   float* c, uint8_t* a_codes, uint8_t* a_scales,
-                                   int* status, void* stream) {
+                                   int rounding, uint64_t seed, const uint8_t* b_codes,
+                                   const uint8_t* b_scales, float* c, uint8_t* a_codes,
+                                   uint8_t* a_scales, int* status, void* stream) {
+  if (!rounding_ok(rounding)) return MXFP4_ERR_ENUM;
   if (!x || !b_codes || !b_scales || !c || (a_codes == nullptr) != (a_scales == nullptr))
     return MXFP4_ERR_NULL;
   if (!dims_ok(m, k) || !dims_ok(n, k) || !dims_ok(m, n) || k % 256)
@@ -251,8 +252,9 @@ mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t 
   if (!aligned16(x) || !aligned16(b_codes) || !aligned16(b_scales) || !aligned16(c) ||
       !aligned16(a_codes) || !aligned4(status))
     return MXFP4_ERR_ALIGN;
-  return from_cuda(mxfp4::launch_gemm_qa(x, m, n, k, b_codes, b_scales, c, a_codes,
-                                         a_scales, status, as_stream(stream)));
+  return from_cuda(mxfp4::launch_gemm_qa(x, m, n, k, rounding == MXFP4_SR, seed, b_codes,
+                                         b_scales, c, a_codes, a_scales, status,
+                                         as_stream(stream)));
 }
 
 const char* mxfp4_status_string(int status) {

@@ -646,13 +646,16 @@ struct QaLayout {
 };
 
 // One 32-element group of X from its four 16-byte chunks (bf16, in order),
-// quantized as the rows quantizer does with nearest-even rounding: the code
-// chunk (element j in nibble j % 8 of word j / 8) and the scale byte. The
-// scaled values v = x 2^-e come from one mixed-precision product of the bf16
-// input with 2^-e (a normal bf16 power of two for every byte the OCP rule
-// gives), rounded once: the fp32 product the rows quantizer forms after
-// widening.
-__device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t& sb) {
+// quantized as the rows quantizer does: the code chunk (element j in nibble
+// j % 8 of word j / 8) and the scale byte. Nearest rounding: the scaled
+// values v = x 2^-e come from one mixed-precision product of the bf16 input
+// with 2^-e (a normal bf16 power of two for every byte the OCP rule gives),
+// rounded once, the fp32 product the rows quantizer forms after widening.
+// Stochastic rounding (SR): bf16x8_sr_word, the rows quantizer's pair form,
+// with the group's counter base kh (its first pair index, keyed).
+template <bool SR>
+__device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t& sb,
+                                                   uint32_t kh) {
   uint32_t mx[8];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -667,26 +670,34 @@ __device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t
   sb = scale_byte(max(mm << 16, mm & 0xFFFF0000u));
   const unsigned short s16 = bf16_inv_scale(sb);
   uint32_t out[4];
+  if (SR) {
+    const uint32_t sat2 = bf16x2_six_scale(sb);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t* q = reinterpret_cast<const uint32_t*>(&w[k]);
-    float v[8];
+    for (int k = 0; k < 4; ++k)
+      out[k] = bf16x8_sr_word<false>(reinterpret_cast<const uint32_t*>(&w[k]), s16, sat2, kh,
+                                     uint32_t(k));
+  } else {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      v[2 * t] = bf16lo_mul(q[t], s16);
-      v[2 * t + 1] = bf16hi_mul(q[t], s16);
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t* q = reinterpret_cast<const uint32_t*>(&w[k]);
+      float v[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        v[2 * t] = bf16lo_mul(q[t], s16);
+        v[2 * t + 1] = bf16hi_mul(q[t], s16);
+      }
+      out[k] = e2m1x8_rn(v);
     }
-    out[k] = e2m1x8_rn(v);
   }
   if (sb == 0xFFu) return make_uint4(0, 0, 0, 0);
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-template <int RT>
+template <int RT, bool SR>
 __global__ void __launch_bounds__(kQThreads, 1)
     k_gemm_qa(const __grid_constant__ CUtensorMap tm_x,
               const __grid_constant__ CUtensorMap tm_b,
-              const uint8_t* __restrict__ sfb, int64_t m, int64_t n, int64_t k,
+              const uint8_t* __restrict__ sfb, int64_t m, int64_t n, int64_t k, RngKey key,
               float* __restrict__ c, uint8_t* __restrict__ a_codes,
               uint8_t* __restrict__ a_scales, int* __restrict__ status) {
   using L = QaLayout<RT>;
@@ -950,9 +961,14 @@ __global__ void __launch_bounds__(kQThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             w[j] = *reinterpret_cast<const uint4*>(xr + (((4 * (g & 1) + j) ^ sw) << 4));
-          uint32_t scb;
-          const uint4 code = qa_quantize_group(w, scb);
           const int G = (8 / kSlots) * h + g;  // group within the stage's 256
+          uint32_t kh = 0;
+          if (SR) {  // the group's first pair index, row-major over X
+            const uint64_t p0 = uint64_t(row * (k / 32) + kb * 8 + G) * 16u;
+            kh = inner_key(key, uint32_t(p0 >> 32)) + uint32_t(p0);
+          }
+          uint32_t scb;
+          const uint4 code = qa_quantize_group<SR>(w, scb, kh);
           *reinterpret_cast<uint4*>(a_s + r * 128 + ((uint32_t(G) ^ sw) << 4)) = code;
           sfa_s[512 * (G >> 2) + 16 * (r & 31) + 4 * (r >> 5) + (G & 3)] = uint8_t(scb);
           if (to_global) {
@@ -1073,9 +1089,9 @@ cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
 
 namespace {
 
-template <int RT>
-cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, const uint8_t* b,
-                         const uint8_t* b_scales, float* c, uint8_t* a_codes,
+template <int RT, bool SR>
+cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, RngKey key,
+                         const uint8_t* b, const uint8_t* b_scales, float* c, uint8_t* a_codes,
                          uint8_t* a_scales, int* status, cudaStream_t s) {
   // X as a byte array [m][2k] for the TMA: 128-byte boxes of 64 bf16
   CUtensorMap mx, mb;
@@ -1083,31 +1099,39 @@ cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, const u
     return cudaErrorInvalidValue;
   constexpr size_t smem = QaLayout<RT>::kBytes + 1024;
   static_assert(smem <= 227 * 1024, "fused GEMM shared memory");
-  auto kern = k_gemm_qa<RT>;
+  auto kern = k_gemm_qa<RT, SR>;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((m + RT - 1) / RT) * ((n + kPN - 1) / kPN);
   const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kQThreads, smem, tiles);
-  kern<<<grid, kQThreads, smem, s>>>(mx, mb, b_scales, m, n, k, c, a_codes, a_scales, status);
+  kern<<<grid, kQThreads, smem, s>>>(mx, mb, b_scales, m, n, k, key, c, a_codes, a_scales,
+                                     status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k,
-                           const uint8_t* b, const uint8_t* b_scales, float* c,
+cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k, bool sr,
+                           uint64_t seed, const uint8_t* b, const uint8_t* b_scales, float* c,
                            uint8_t* a_codes, uint8_t* a_scales, int* status,
                            cudaStream_t s) {
   if (k % 256) return cudaErrorInvalidValue;
+  const RngKey key = make_key(seed, 0);
   // 64-row tiles where 128-row ones would not give every SM a tile
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles128 = ((m + 127) / 128) * ((n + kPN - 1) / kPN);
-  return tiles128 < sms
-             ? gemm_qa_impl<64>(x, m, n, k, b, b_scales, c, a_codes, a_scales, status, s)
-             : gemm_qa_impl<128>(x, m, n, k, b, b_scales, c, a_codes, a_scales, status, s);
+  if (tiles128 < sms)
+    return sr ? gemm_qa_impl<64, true>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
+                                       status, s)
+              : gemm_qa_impl<64, false>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
+                                        status, s);
+  return sr ? gemm_qa_impl<128, true>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
+                                      status, s)
+            : gemm_qa_impl<128, false>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
+                                       status, s);
 }
 
 }  // namespace mxfp4

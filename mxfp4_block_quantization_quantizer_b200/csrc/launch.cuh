@@ -75,11 +75,11 @@ cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
                              int64_t m, int64_t n, int64_t k, float* c,
                              int* status, cudaStream_t s);
 
-// C = Q_D(X) B^T with X (bf16 [m][k], k a multiple of 256) quantized 1x32
-// nearest-even inside the GEMM's load stage; a_codes / a_scales (ROWS
-// layout) receive that quantization when not null.
-cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k,
-                           const uint8_t* b, const uint8_t* b_scales, float* c,
+// C = Q(X) B^T with X (bf16 [m][k], k a multiple of 256) quantized 1x32
+// (nearest-even, or stochastic keyed by seed) inside the GEMM's load stage;
+// a_codes / a_scales (ROWS layout) receive that quantization when not null.
+cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k, bool sr,
+                           uint64_t seed, const uint8_t* b, const uint8_t* b_scales, float* c,
                            uint8_t* a_codes, uint8_t* a_scales, int* status,
                            cudaStream_t s);
 

@@ -587,6 +587,33 @@ __device__ __forceinline__ void pair_randoms(uint32_t g, uint32_t& r_even, uint3
   r_even = (g ^ r_odd) & 0xFFFFu;
 }
 
+// Stochastic codes of 8 bf16 values of a 1x32 group (four packed words wq,
+// element 2k in the low half of wq[k]) whose scale byte sb is not 0xFF, as
+// the row quantizer forms them: each value is widened and scaled by 2^-e in
+// one exact mixed-precision product (s16 = bf16_inv_scale(sb)), after the
+// packed pairs are saturated at 6 2^e (sat2 = bf16x2_six_scale(sb); the
+// overflow-aware rule never exceeds 6); pair k of the 8 takes its random
+// numbers from the hash of counter kh + 4 q + k; the codes of a pair share
+// one byte merge and the signs come from the input words.
+template <bool OAS>
+__device__ __forceinline__ uint32_t bf16x8_sr_word(const uint32_t* wq, unsigned short s16,
+                                                   uint32_t sat2, uint32_t kh, uint32_t q) {
+  uint32_t pb[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t ws = OAS ? wq[k] : bf16x2_clamp_abs(wq[k], sat2);
+    uint32_t re, ro;
+    pair_randoms(mix32_pre(mad_u32(4u * q + uint32_t(k), 1u, kh)), re, ro);
+    const uint32_t te = mad_u32(sr_operand(bf16lo_mul(ws, s16)), 4u,
+                                mad_u32(re, 0xFFFFFF00u, kSrBase4));
+    const uint32_t to = mad_u32(sr_operand(bf16hi_mul(ws, s16)), 64u,
+                                mad_u32(ro, 0xFFFFF000u, kSrBase64));
+    pb[k] = pair_byte(to, te);
+  }
+  return pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) |
+         sign_nibbles_rows(wq[0], wq[1], wq[2], wq[3]);
+}
+
 // f16 halves as fp32 by an exact mixed-precision product with one (f16 1.0)
 // on the FMA pipe.
 __device__ __forceinline__ float f16lo_f32(uint32_t h, unsigned short one) {

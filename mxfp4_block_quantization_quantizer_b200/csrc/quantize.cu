@@ -106,30 +106,13 @@ __global__ void __launch_bounds__(kRowThreads)
 #pragma unroll
         for (int q = 0; q < 4; ++q) word[q] = sb == 0xFFu ? 0u : e2m1x8_rn(v + 8 * q);
       } else if (BF16 && sb != 0xFFu) {
-        // bf16: each value is widened and scaled by 2^-e in one exact
-        // mixed-precision product, after the packed pairs are saturated at
-        // 6 2^e (the overflow-aware rule never exceeds 6); the codes of a
-        // pair share one byte merge, the signs come from the input words
+        // bf16: the pair form on the packed input words (bf16x8_sr_word)
         const unsigned short s16 = bf16_inv_scale(sb);
         const uint32_t sat2 = bf16x2_six_scale(sb);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t* wq = reinterpret_cast<const uint32_t*>(&w[u][q]);
-          uint32_t pb[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t ws = OAS ? wq[k] : bf16x2_clamp_abs(wq[k], sat2);
-            uint32_t re, ro;
-            pair_randoms(mix32_pre(mad_u32(uint32_t(4 * q + k), 1u, kh)), re, ro);
-            const uint32_t te = mad_u32(sr_operand(bf16lo_mul(ws, s16)), 4u,
-                                        mad_u32(re, 0xFFFFFF00u, kSrBase4));
-            const uint32_t to = mad_u32(sr_operand(bf16hi_mul(ws, s16)), 64u,
-                                        mad_u32(ro, 0xFFFFF000u, kSrBase64));
-            pb[k] = pair_byte(to, te);
-          }
-          word[q] = pack_pair_bytes(pb[0], pb[1], pb[2], pb[3]) |
-                    sign_nibbles_rows(wq[0], wq[1], wq[2], wq[3]);
-        }
+        for (int q = 0; q < 4; ++q)
+          word[q] = bf16x8_sr_word<OAS>(reinterpret_cast<const uint32_t*>(&w[u][q]), s16, sat2,
+                                        kh, uint32_t(q));
       } else if (sb >= 2u && sb != 0xFFu) {
         // the power of two rides on the rounding (e2m1_sr_top_scaled)
         const float half = scale_half(sb), sat = OAS ? 0.0f : scale_six(sb);

@@ -130,13 +130,14 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, PODD, NUL, NUL) == ALIGN
     assert L.mxfp4_gemm(P, PODD, P, P, 128, 128, 256, P, NUL, NUL) == ALIGN
     g = L.mxfp4_gemm_quantize_a
-    assert g(NUL, 128, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == NULL
-    assert g(P, 128, 256, 256, P, P, P, P, NUL, NUL, NUL) == NULL   # codes without scales
-    assert g(P, 128, 256, 128, P, P, P, NUL, NUL, NUL, NUL) == SHAPE  # k % 256
-    assert g(P, 0, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == SHAPE
-    assert g(PODD, 128, 256, 256, P, P, P, NUL, NUL, NUL, NUL) == ALIGN
-    assert g(P, 128, 256, 256, P, P, P, PODD, P, NUL, NUL) == ALIGN
-    assert g(P, 128, 256, 256, P, P, P, NUL, NUL, P2, NUL) == ALIGN
+    assert g(P, 128, 256, 256, 2, 0, P, P, P, NUL, NUL, NUL, NUL) == ENUM
+    assert g(NUL, 128, 256, 256, 0, 0, P, P, P, NUL, NUL, NUL, NUL) == NULL
+    assert g(P, 128, 256, 256, 1, 0, P, P, P, P, NUL, NUL, NUL) == NULL  # codes, no scales
+    assert g(P, 128, 256, 128, 0, 0, P, P, P, NUL, NUL, NUL, NUL) == SHAPE  # k % 256
+    assert g(P, 0, 256, 256, 0, 0, P, P, P, NUL, NUL, NUL, NUL) == SHAPE
+    assert g(PODD, 128, 256, 256, 0, 0, P, P, P, NUL, NUL, NUL, NUL) == ALIGN
+    assert g(P, 128, 256, 256, 0, 0, P, P, P, PODD, P, NUL, NUL) == ALIGN
+    assert g(P, 128, 256, 256, 0, 0, P, P, P, NUL, NUL, P2, NUL) == ALIGN
     # the status word needs 4-byte alignment only
     assert L.mxfp4_gemm(P, P, P, P, 128, 128, 256, P, P2, NUL) == ALIGN
     assert L.mxfp4_rht_quantize(P, 1, 64, 64, 0, 0, 0, P, P, NUL, P2, NUL) == ALIGN

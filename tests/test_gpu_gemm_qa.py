@@ -1,9 +1,9 @@
-"""The forward GEMM with the activation quantized in its load stage
-(mxfp4_gemm_quantize_a, C = Q_D(X) B^T) against the two-step path it
-replaces and against the oracle.
+"""The GEMM with the activation quantized in its load stage
+(mxfp4_gemm_quantize_a, C = Q(X) B^T, Q nearest-even or stochastic) against
+the two-step path it replaces and against the oracle.
 
-- Q_D(X) as the fused kernel writes it out equals mxfp4_quantize's ROWS RNE
-  codes and scales byte for byte, and the oracle's;
+- Q(X) as the fused kernel writes it out equals mxfp4_quantize's ROWS codes
+  and scales (same rounding and seed) byte for byte, and the oracle's;
 - C equals mxfp4_gemm on those codes bit for bit (same tiles, same MMA
   sequence) and lies within the fp32 accumulation bound of the oracle's
   exact product: (k - 1) 2^-24 sum_j |a_j b_j|.
@@ -110,3 +110,45 @@ def test_fused_on_the_sweep_activation(n):
     # the oracle's row quantization of sampled rows is the GPU's
     assert np.array_equal(to_np(ac)[rows], oc) and np.array_equal(to_np(as_)[rows], os_)
     check_against_oracle(to_np(c)[rows], oc, os_, to_np(wc), to_np(ws), K)
+
+
+@pytest.mark.parametrize("mnk", [(200, 136, 512), (9000, 512, 256), (20000, 520, 256),
+                                 (384, 1024, 2560)])
+def test_fused_stochastic_rounding(mnk):
+    """Q_S(X) in the load stage (a gradient for a backward GEMM): the codes of
+    mxfp4_quantize with the same seed, and the two-step C."""
+    mm, nn, k = mnk
+    x = W.normal_bf16(mm, k, 25, 0.005, 50.0)
+    xd = to_dev(x)
+    wc, ws = weight(nn, k, 26)
+    wb = m.scales_to_blocked(ws)
+    c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, rounding=m.SR, seed=17, want_a=True)
+    qc, qs = m.quantize(xd, m.ROWS, m.SR, 17)
+    assert torch.equal(ac, qc) and torch.equal(as_, qs)
+    oc, os_ = O.quantize(x, O.ROWS, O.SR, 17)
+    assert np.array_equal(to_np(ac), oc) and np.array_equal(to_np(as_), os_)
+    ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, k)
+    assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+    check_against_oracle(to_np(c), oc, os_, to_np(wc), to_np(ws), k)
+    # another seed gives other codes
+    c2, ac2, _ = m.gemm_quantize_a(xd, wc, wb, rounding=m.SR, seed=18, want_a=True)
+    assert not torch.equal(ac2, ac)
+
+
+def test_fused_stochastic_rounding_on_the_sweep():
+    x = W.sweep(seed=5)
+    xd = to_dev(x)
+    K = x.shape[1]
+    wc, ws = weight(256, K, 6)
+    wb = m.scales_to_blocked(ws)
+    c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, rounding=m.SR, seed=5, want_a=True)
+    qc, qs = m.quantize(xd, m.ROWS, m.SR, 5)
+    assert torch.equal(ac, qc) and torch.equal(as_, qs)
+    ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, K)
+    assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+    # sampled rows against the oracle (its counters start at row0)
+    acn, asn, cn = to_np(ac), to_np(as_), to_np(c)
+    for r in (0, 4097, 8191):
+        oc, os_ = O.quantize(x[r:r + 1], O.ROWS, O.SR, 5, row0=r)
+        assert np.array_equal(acn[r:r + 1], oc) and np.array_equal(asn[r:r + 1], os_)
+        check_against_oracle(cn[r:r + 1], oc, os_, to_np(wc), to_np(ws), K)

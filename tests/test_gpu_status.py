@@ -46,7 +46,8 @@ def short_wait_lib(tmp_path_factory):
     vp, i32, i64, u64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint64
     L.mxfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
     L.mxfp4_rht_quantize.argtypes = [vp, i32, i64, i64, u64, i32, u64, vp, vp, vp, vp, vp]
-    L.mxfp4_gemm_quantize_a.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp]
+    L.mxfp4_gemm_quantize_a.argtypes = [vp, i64, i64, i64, i32, u64, vp, vp, vp, vp, vp, vp,
+                                        vp]
     for f in (L.mxfp4_gemm, L.mxfp4_rht_quantize, L.mxfp4_gemm_quantize_a):
         f.restype = i32
     return L
@@ -140,8 +141,8 @@ def test_fused_gemm_timeout_sets_status_and_poisons_tiles(short_wait_lib):
     wb = m.scales_to_blocked(ws)
     c = torch.zeros((384, 520), dtype=torch.float32, device="cuda")
     st = zero_status()
-    rc = short_wait_lib.mxfp4_gemm_quantize_a(ptr(xd), 384, 520, 768, ptr(wc), ptr(wb),
-                                              ptr(c), None, None, ptr(st), stream())
+    rc = short_wait_lib.mxfp4_gemm_quantize_a(ptr(xd), 384, 520, 768, m.RNE, 0, ptr(wc),
+                                              ptr(wb), ptr(c), None, None, ptr(st), stream())
     assert rc == 0
     torch.cuda.synchronize()
     assert int(st.item()) == m.STATUS_WAIT_TIMEOUT
