@@ -48,7 +48,10 @@ def check_against_oracle(c, xc, xs, wc, ws, k, rows=None):
                                  # several tiles per CTA with one stage each (the
                                  # accumulator drained after the next tile's only
                                  # stage): 64-row tiles, then 128-row tiles
-                                 (9000, 512, 256), (20000, 520, 256)])
+                                 (9000, 512, 256), (20000, 520, 256),
+                                 # one row; two weight rows; n not a multiple of 4
+                                 # (scalar stores of C)
+                                 (1, 256, 256), (65, 2, 512), (100, 130, 256)])
 def test_fused_equals_quantize_then_gemm(mnk):
     mm, nn, k = mnk
     x = W.normal_bf16(mm, k, 21, 0.005, 50.0)
