@@ -1,0 +1,111 @@
+"""Seeded random sweep over shapes, dtypes, value distributions, seeds and
+scale rules: every quantizer entry point against the oracle, bit for bit
+(the rotation through its own rule), and the fused GEMM against the
+two-step path. Each case is small enough for the oracle; together they
+cover many ragged tile positions, grid sizes and special values that the
+hand-picked cases do not.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_block_quantization_quantizer_b200 as m
+import oracle as O
+from gpu_util import BF16, assert_bits_equal, to_dev, to_np
+from test_gpu_parity import check_rht
+
+pytestmark = pytest.mark.gpu
+
+N_CASES = 64
+
+
+def random_tensor(g, rows, cols, dtype):
+    """A mix the kernels must handle alike: a random log-uniform spread of
+    magnitudes, exact zeros, signed zeros, subnormals, huge values, and now
+    and then an inf or NaN group."""
+    x = g.standard_normal((rows, cols)) * np.exp2(g.integers(-20, 20, size=(rows, cols)))
+    kind = g.integers(0, 6)
+    if kind == 1:
+        x[g.random((rows, cols)) < 0.2] = 0.0
+        x[g.random((rows, cols)) < 0.05] = -0.0
+    elif kind == 2:
+        x *= 2.0 ** -130                      # subnormal territory
+    elif kind == 3:
+        x *= 2.0 ** 100                       # near the top of the range
+    elif kind == 4:
+        r, c = g.integers(0, rows), g.integers(0, cols)
+        x[r, c] = [np.inf, -np.inf, np.nan][g.integers(0, 3)]
+    x = x.astype(np.float32)
+    return x.astype(BF16) if dtype == "bf16" else x
+
+
+def cases(seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for i in range(N_CASES):
+        rows = int(32 * g.integers(1, 20))
+        cols = int(32 * g.integers(1, 40))
+        out.append((i, rows, cols, ["bf16", "f32"][g.integers(0, 2)],
+                    int(g.integers(0, 2**32)), bool(g.integers(0, 2))))
+    return out
+
+
+@pytest.mark.parametrize("case", cases(101), ids=lambda c: "case%d" % c[0])
+def test_fuzz_quantize_and_dequantize(case):
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(1000 + i))
+    x = random_tensor(g, rows, cols, dtype)
+    xd = to_dev(x)
+    for axis in (m.ROWS, m.COLS):
+        for rnd in (m.RNE, m.SR):
+            c, s = m.quantize(xd, axis, rnd, seed, oas=oas)
+            oc, os_ = O.quantize(x, axis, rnd, seed, oas=oas)
+            assert_bits_equal(to_np(c), oc, "codes axis %d rnd %d" % (axis, rnd))
+            assert_bits_equal(to_np(s), os_, "scales axis %d rnd %d" % (axis, rnd))
+            for od, oname in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+                y = m.dequantize(c, s, rows, cols, axis, out_dtype=od)
+                want = O.dequantize(oc, os_, rows, cols, axis, oname)
+                assert_bits_equal(to_np(y), want, "dequantized axis %d" % axis)
+
+
+@pytest.mark.parametrize("case", cases(202), ids=lambda c: "case%d" % c[0])
+def test_fuzz_double_quantize(case):
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(2000 + i))
+    x = random_tensor(g, rows, cols, dtype)
+    got = m.double_quantize(to_dev(x), seed=seed, oas=oas)
+    for gt, w, name in zip(got, O.double_quantize(x, seed, oas=oas),
+                           ("row codes", "row scales", "col codes", "col scales")):
+        assert_bits_equal(to_np(gt), w, "double quantization " + name)
+
+
+@pytest.mark.parametrize("case", cases(303)[:24], ids=lambda c: "case%d" % c[0])
+def test_fuzz_rotation(case):
+    """Finite inputs of moderate range (the rotation's parity claim)."""
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(3000 + i))
+    x = (g.standard_normal((rows, cols)) * np.exp2(g.integers(-6, 6, size=(rows, cols))))
+    x = x.astype(np.float32)
+    x = x.astype(BF16) if dtype == "bf16" else x
+    for rnd in (m.RNE, m.SR):
+        codes, scales, rot = m.rht_quantize(to_dev(x), seed % 97, rnd, seed, want_rotated=True)
+        check_rht(x, seed % 97, rnd, seed, to_np(codes), to_np(scales), to_np(rot))
+
+
+@pytest.mark.parametrize("case", cases(404)[:24], ids=lambda c: "case%d" % c[0])
+def test_fuzz_fused_gemm(case):
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(4000 + i))
+    k = 256 * int(g.integers(1, 5))
+    n = int(g.integers(1, 600))
+    x = (g.standard_normal((rows, k)) * np.exp2(g.integers(-8, 8, size=(rows, k))))
+    xd = to_dev(x.astype(np.float32).astype(BF16))
+    w = to_dev(g.standard_normal((n, k)).astype(np.float32).astype(BF16))
+    wc, ws = m.quantize(w, m.ROWS, m.RNE)
+    wb = m.scales_to_blocked(ws)
+    for rnd in (m.RNE, m.SR):
+        c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, rounding=rnd, seed=seed, want_a=True)
+        qc, qs = m.quantize(xd, m.ROWS, rnd, seed)
+        assert torch.equal(ac, qc) and torch.equal(as_, qs)
+        ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, k)
+        assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
