@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kOscThreads)
         dq[j] = __fadd_rn(dq[j], fabsf(__fsub_rn(qw[j], qs[j])));
         if (WEND) {
           fl[j] = dq[j] > __fmul_rn(k1, dw[j]) ? 1 : 0;
-          count += fl[j];
+          count += ok ? fl[j] : 0u;  // threads past the last group redo group 0
           dw[j] = dq[j] = 0.0f;
         }
       }

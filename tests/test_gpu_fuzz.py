@@ -1,7 +1,8 @@
 """Seeded random sweep over shapes, dtypes, value distributions, seeds and
 scale rules: every quantizer entry point against the oracle, bit for bit
 (the rotation through its own rule), and the fused GEMM against the
-two-step path. Each case is small enough for the oracle; together they
+two-step path; the tracker, Q-Ramping and Q-EMA state bit for bit. Each
+case is small enough for the oracle; together they
 cover many ragged tile positions, grid sizes and special values that the
 hand-picked cases do not.
 """
@@ -11,7 +12,7 @@ import torch
 
 import mxfp4_block_quantization_quantizer_b200 as m
 import oracle as O
-from gpu_util import BF16, assert_bits_equal, to_dev, to_np
+from gpu_util import BF16, assert_bits_equal, assert_f32_equal_or_both_nan, to_dev, to_np
 from test_gpu_parity import check_rht
 
 pytestmark = pytest.mark.gpu
@@ -109,3 +110,77 @@ def test_fuzz_fused_gemm(case):
         assert torch.equal(ac, qc) and torch.equal(as_, qs)
         ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, k)
         assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+
+
+def tracker_weights(g, rows, cols):
+    """fp32 weights with one group maximum per group (a fixed scale) and many
+    values near a rounding edge, like the tracker workload."""
+    w = (g.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    w = np.clip(w, -2.0 ** -4, 2.0 ** -4)
+    w.reshape(-1, 32)[:, 0] = np.float32(2.0 ** -4 * 1.5)
+    edges = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]) * 2.0 ** -6
+    pick = g.random((rows, cols)) < 0.3
+    near = g.choice(edges, size=(rows, cols)) * (1 + g.uniform(-1e-3, 1e-3, (rows, cols)))
+    w[pick] = (near * np.sign(g.standard_normal((rows, cols))))[pick].astype(np.float32)
+    w.reshape(-1, 32)[:, 0] = np.float32(2.0 ** -4 * 1.5)
+    return w
+
+
+@pytest.mark.parametrize("case", cases(505)[:16], ids=lambda c: "case%d" % c[0])
+def test_fuzz_tracker_and_qramp(case):
+    """The tracker over a random window with a random threshold, and
+    Q-Ramping with random window, k1 and k2 over two epochs: every state
+    array and flag count bit for bit after every iteration."""
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(5000 + i))
+    w0 = tracker_weights(g, min(rows, 128), cols)
+    # the tracker
+    steps = int(g.integers(1, 30))
+    threshold = float(g.choice([0.5, 2.0, 4.0, 16.0]))
+    w, ws = to_dev(w0.copy()), to_dev(w0.copy())
+    dw, dq = torch.zeros_like(w), torch.zeros_like(w)
+    nflag = torch.zeros(1, dtype=torch.int64, device="cuda")
+    ow, ows, odw, odq = w0.copy(), w0.copy(), np.zeros_like(w0), np.zeros_like(w0)
+    flagged = 0
+    for t in range(steps):
+        end = t == steps - 1 or g.random() < 0.1
+        m.osc_synthetic_update(w, seed, t)
+        m.osc_step(w, ws, dw, dq, window_end=end, threshold=threshold, n_flagged=nflag)
+        O.osc_synthetic_update(ow, seed, t)
+        flagged += O.osc_step(ow, ows, odw, odq, window_end=end, threshold=threshold)
+    for gt, wv, name in zip((w, ws, dw, dq), (ow, ows, odw, odq), ("w", "w_snap", "d_w", "d_q")):
+        assert_bits_equal(to_np(gt), wv, "tracker " + name)
+    assert int(nflag.item()) == flagged
+    # Q-Ramping
+    track, k2, k1 = int(g.integers(0, 8)), int(g.integers(1, 7)), float(g.choice([2.0, 16.0]))
+    epoch = int(g.integers(1, 12))
+    z = np.zeros_like(w0)
+    ref = [w0.copy(), z.copy(), z.copy(), z.copy(), z.copy(), np.zeros(w0.shape, np.uint8)]
+    dev = [to_dev(a.copy()) for a in ref]
+    nflag.zero_()
+    total = 0
+    mag = (np.float32(1e-4) * np.abs(w0)).astype(np.float32)
+    for t in range(2 * epoch):
+        d = (np.where(g.random(w0.shape) < 0.5, -1.0, 1.0) * mag).astype(np.float32)
+        it = t % epoch
+        m.qramp_step(dev[0], to_dev(d), *dev[1:], it, track_iters=track, k1=k1, k2=k2,
+                     n_flagged=nflag)
+        total += O.qramp_step(ref[0], d, *ref[1:], it, track_iters=track, k1=k1, k2=k2)
+        for gt, r, name in zip(dev, ref, ("w", "w_snap", "d_w", "d_q", "acc", "flag")):
+            assert_bits_equal(to_np(gt), r, "qramp %s at %d" % (name, t))
+    assert int(nflag.item()) == total
+
+
+@pytest.mark.parametrize("case", cases(606)[:16], ids=lambda c: "case%d" % c[0])
+def test_fuzz_qema(case):
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(6000 + i))
+    w_np = random_tensor(g, rows, cols, "f32")
+    e_np = random_tensor(g, rows, cols, "f32")
+    beta = float(g.choice([0.0, 0.5, 0.9, 0.998, 1.0]))
+    e = to_dev(e_np)
+    c, s = m.qema_quantize(to_dev(w_np), e, beta)
+    oc, os_ = O.qema_quantize(w_np, e_np, beta)
+    assert_f32_equal_or_both_nan(to_np(e), e_np, "ema")   # NaN payloads may differ
+    assert_bits_equal(to_np(c), oc, "codes")
+    assert_bits_equal(to_np(s), os_, "scales")

@@ -505,6 +505,28 @@ def test_qramp_epochs(track, k2):
         assert total > 0
 
 
+def test_qramp_flag_count_with_a_ragged_last_block():
+    """96 groups (not a multiple of a block's 64): the threads past the last
+    group must not add to the flag count (they recompute group 0's flags
+    without storing them). Group 0 oscillates, so it has flags to count."""
+    w_np = W.osc_w(seed=6, rows=32, cols=96)
+    deltas = qramp_deltas(w_np, 4, 12)
+    for d in deltas:
+        d[0, :32] = np.where(np.arange(32) % 2 == 0, 1.0, -1.0) * np.float32(4e-3)
+    z = np.zeros_like(w_np)
+    ref = [w_np.copy(), z.copy(), z.copy(), z.copy(), z.copy(), np.zeros(w_np.shape, np.uint8)]
+    dev = [to_dev(a.copy()) for a in ref]
+    nflag = torch.zeros(1, dtype=torch.int64, device="cuda")
+    total = 0
+    for it, d in enumerate(deltas):
+        m.qramp_step(dev[0], to_dev(d), *dev[1:], it, track_iters=4, k1=0.5, k2=2,
+                     n_flagged=nflag)
+        total += O.qramp_step(ref[0], d, *ref[1:], it, track_iters=4, k1=0.5, k2=2)
+    assert_bits_equal(to_np(dev[5]), ref[5], "flags")
+    assert ref[5][0, :32].any()
+    assert int(nflag.item()) == total == int(ref[5].sum())
+
+
 def test_osc_update_alone_and_ragged_length():
     g = np.random.Generator(np.random.PCG64(2))
     w_np = g.normal(0, 0.02, size=(7, 13)).astype(np.float32)  # 91 elements
