@@ -184,3 +184,25 @@ def test_fuzz_qema(case):
     assert_f32_equal_or_both_nan(to_np(e), e_np, "ema")   # NaN payloads may differ
     assert_bits_equal(to_np(c), oc, "codes")
     assert_bits_equal(to_np(s), os_, "scales")
+
+
+@pytest.mark.parametrize("case", cases(707)[:24], ids=lambda c: "case%d" % c[0])
+def test_fuzz_blocked_scales_and_gemm(case):
+    """Random m, n and k (a multiple of 32: both GEMM kernels): the blocked
+    scale order byte for byte, and C within the fp32 accumulation bound of
+    the oracle's product."""
+    i, rows, cols, dtype, seed, oas = case
+    g = np.random.Generator(np.random.PCG64(7000 + i))
+    mm, nn, k = int(g.integers(1, 300)), int(g.integers(1, 300)), int(32 * g.integers(1, 24))
+    ca = g.integers(0, 256, size=(mm, k // 2), dtype=np.uint8)
+    cb = g.integers(0, 256, size=(nn, k // 2), dtype=np.uint8)
+    sa = g.integers(110, 145, size=(mm, k // 32), dtype=np.uint8)
+    sb = g.integers(110, 145, size=(nn, k // 32), dtype=np.uint8)
+    ba, bb = m.scales_to_blocked(to_dev(sa)), m.scales_to_blocked(to_dev(sb))
+    assert_bits_equal(to_np(ba), O.scales_to_blocked(sa), "blocked A scales")
+    assert_bits_equal(to_np(bb), O.scales_to_blocked(sb), "blocked B scales")
+    got = to_np(m.gemm(to_dev(ca), ba, to_dev(cb), bb, k)).astype(np.float64)
+    want = O.gemm(ca, sa, cb, sb, k)
+    da = np.abs(O.dequantize(ca, sa, mm, k, O.ROWS, "f32").astype(np.float64))
+    db = np.abs(O.dequantize(cb, sb, nn, k, O.ROWS, "f32").astype(np.float64))
+    assert np.all(np.abs(got - want) <= (k - 1) * 2.0 ** -24 * (da @ db.T))
