@@ -33,6 +33,31 @@ constexpr int kRhtRowsY = 32;   // rows per CTA step
 // fp32 nearest to 1/sqrt(32).
 constexpr float kInvSqrt32 = 0.17677669529663687f;
 
+// Stochastic codes of the 8 values y[j] mul (mul > 0), pair k taking its
+// random numbers from the hash of counter c0 + k, as e2m1x8_sr: the
+// magnitude is formed as |y[j]| mul, the same product as |y[j] mul|
+// (nearest rounding is symmetric), so the absolute value rides on the
+// multiply, and the sign comes from y[j]; each pair's hash is formed where
+// it is used.
+__device__ __forceinline__ uint32_t e2m1x8_sr_mul(const float* y, float mul, uint32_t c0) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 3; k >= 0; --k) {
+    uint32_t ne, no;
+    sr_noise64_pair(mix32_pre(mad_u32(uint32_t(k), 1u, c0)), ne, no);
+#pragma unroll
+    for (int par = 1; par >= 0; --par) {
+      const float yv = y[2 * k + par];
+      const float a = fabsf(yv) * mul;
+      float ry = fmaxf(a, __fmaf_ru(a, 0.5f, 0.5f));
+      ry = fminf(ry, 6.0f);  // |v| >= 6 saturates to 6
+      out = push_code(out, (__float_as_uint(ry) * 64u + (par ? no : ne)) |
+                               (__float_as_uint(yv) & 0x80000000u));
+    }
+  }
+  return out;
+}
+
 // fp32 inputs (bf16 inputs take the tensor-core kernel below).
 template <bool SR, bool ROT, bool OAS>
 __global__ void __launch_bounds__(kRhtThreads, 2)
@@ -120,16 +145,12 @@ __global__ void __launch_bounds__(kRhtThreads, 2)
     uint32_t wq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
       if (SR) {
-        const uint32_t p0 = uint32_t(pg) + 4 * q;
-        uint32_t h[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) h[t] = mix32_pre(mad_u32(uint32_t(t), 1u, kh + p0));
-        wq[q] = e2m1x8_sr(v, h);
+        wq[q] = e2m1x8_sr_mul(y + 8 * q, mul, kh + uint32_t(pg) + 4 * q);
       } else {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
         wq[q] = e2m1x8_rn(v);
       }
     }
@@ -248,16 +269,12 @@ __device__ __forceinline__ void rht_tc_quantize_group(float* y, int64_t r, int64
   uint32_t wq[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
     if (SR) {
-      const uint32_t p0 = uint32_t(pg) + 4 * q;
-      uint32_t h[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) h[t] = mix32_pre(mad_u32(uint32_t(t), 1u, kh + p0));
-      wq[q] = e2m1x8_sr(v, h);
+      wq[q] = e2m1x8_sr_mul(y + 8 * q, mul, kh + uint32_t(pg) + 4 * q);
     } else {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = y[8 * q + j] * mul;
       wq[q] = e2m1x8_rn(v);
     }
   }
