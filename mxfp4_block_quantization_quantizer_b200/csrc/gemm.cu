@@ -571,6 +571,112 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
 
 // ---------------------------------------------------------------------------
+// Thread-block clusters (the fused GEMM's shared quantization)
+// ---------------------------------------------------------------------------
+
+// This CTA's rank in its cluster, the cluster's index and the number of
+// clusters of a one-dimensional grid.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+  uint32_t r;
+  asm("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// The address in the cluster's shared window of the byte at shared address
+// a of the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t a, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(rank));
+  return d;
+}
+// Every thread of every CTA of the cluster (release, then acquire).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// wait_parity_or_failed for a barrier that other CTAs of the cluster also
+// complete (acquire at cluster scope).
+__device__ __forceinline__ bool wait_cluster_or_failed(unsigned long long* bar,
+                                                       uint32_t parity, const int* failed) {
+  const uint32_t a = smem_u32(bar);
+  for (long long i = 0; i < kWaitLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 63) == 63 && failed_flag(failed)) return false;
+  }
+  return false;
+}
+// Stores to this CTA's shared memory (a shared::cta address).
+__device__ __forceinline__ void st_smem_u8(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "h"(static_cast<unsigned short>(v))
+               : "memory");
+}
+__device__ __forceinline__ void st_smem(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[1]) { st_smem(a, v[0]); }
+__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[2]) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v[0]), "r"(v[1]) : "memory");
+}
+__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+// A plain store to another CTA's shared memory (a from cluster_addr).
+__device__ __forceinline__ void st_cluster(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+// Asynchronous stores into the shared memory of another CTA of the cluster
+// (a and the mbarrier bar both from cluster_addr, bar in the same CTA as
+// a): the bytes count towards bar's transaction count when they land, and
+// nothing waits for them here.
+__device__ __forceinline__ void st_async(uint32_t a, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.weak.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               ::"r"(a), "r"(v), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async(uint32_t a, const uint32_t (&v)[1], uint32_t bar) {
+  st_async(a, v[0], bar);
+}
+__device__ __forceinline__ void st_async(uint32_t a, const uint32_t (&v)[2], uint32_t bar) {
+  asm volatile(
+      "st.async.weak.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];"
+      ::"r"(a), "r"(v[0]), "r"(v[1]), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void st_async(uint32_t a, const uint32_t (&v)[4], uint32_t bar) {
+  asm volatile(
+      "st.async.weak.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, "
+      "%4}, [%5];" ::"r"(a),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(bar)
+      : "memory");
+}
+// commit_to on the mbarrier at the same offset in every CTA of cta_mask.
+__device__ __forceinline__ void commit_to_cluster(unsigned long long* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(cta_mask));
+}
+
+// ---------------------------------------------------------------------------
 // Forward GEMM with the activation quantized in the load stage:
 //   C = Q_D(X) B^T,  X bf16 [M][K] in 1x32 groups along K, nearest-even
 // (source: "Oscillation-Reduced MXFP4 Training for Vision Transformers",
@@ -585,46 +691,83 @@ __global__ void __launch_bounds__(kPThreads, 1)
 //             a free stage);
 //   warp 1:   tensor memory; one thread waits for both halves of a stage
 //             (B landed, A quantized) and issues the MMAs as above;
-//   warps 3-18 (workers): during a tile's main loop each thread quantizes
-//             one row group of every X half-stage (row = thread % 128) with
-//             the rows quantizer's arithmetic (bf16 absmax, OCP scale byte,
-//             the product with 2^-e formed as one exact mixed-precision
-//             multiply of the bf16 input, nearest-even E2M1: bit-identical
-//             codes), writes the 16-byte code chunk into the operand stage
-//             at its place in the 128-byte-swizzled K-major layout of the
-//             MMA and the scale byte into the blocked tile that tcgen05.cp
-//             copies to tensor memory, then releases the X slot; once the
-//             first stage of the next tile is quantized (the MMAs of the
-//             previous one have drained meanwhile) the workers read the
-//             previous tile's accumulator (warp w: lane quarter w % 4,
-//             64 columns) and store it. The CTAs of the first column tile
-//             can also write the codes and scales to global memory in the
-//             ROWS layout of mxfp4_quantize.
-// X is re-read (from L2 when neighbouring CTAs share it) and re-quantized
-// once per column tile, so the fusion pays where N is small. RT is the
-// number of X rows a tile covers: 128, or 64 when 128-row tiles would leave
-// SMs idle (a small N); then the MMA still spans 128 rows, of which the last
-// 64 are left over in shared memory and never stored, and an X slot holds a
-// whole K = 256 stage of the 64 rows.
+//   warps 3-18 (workers): during a tile's main loop the threads quantize
+//             the row groups of every X slot (one or a part of a group
+//             each) with the rows quantizer's arithmetic (bf16 absmax, OCP
+//             scale byte, the product with 2^-e formed as one exact
+//             mixed-precision multiply of the bf16 input, nearest-even
+//             E2M1: bit-identical codes), write the code bytes into the
+//             operand stage at their place in the 128-byte-swizzled K-major
+//             layout of the MMA and the scale byte into the blocked tile
+//             that tcgen05.cp copies to tensor memory, then release the X
+//             slot; once the first stage of the next tile is quantized (the
+//             MMAs of the previous one have drained meanwhile) the workers
+//             read the previous tile's accumulator (warp w: lane quarter
+//             w % 4, 64 columns) and store it. The CTAs of the first column
+//             tile can also write the codes and scales to global memory in
+//             the ROWS layout of mxfp4_quantize.
+// RT is the number of X rows a tile covers: 128, or 64 when 128-row tiles
+// would leave SMs idle; then the MMA still spans 128 rows, of which the
+// last 64 are left over in shared memory and never stored.
+//
+// Clusters (CS = 2 or 4 CTAs): every column tile needs the whole quantized
+// A of its rows, so without sharing X is re-read and re-quantized once per
+// column tile. The CS CTAs of a cluster take the same rows and CS adjacent
+// column tiles; each loads and quantizes RT / CS of the rows of every
+// K = 256 stage and sends the codes and scale words to the operand stage of
+// every CTA of the cluster with asynchronous distributed-shared-memory
+// stores, whose bytes complete that CTA's stage barrier (armed by its MMA
+// thread with the stage's byte count): no fence or arrival on the workers'
+// path. A stage is written once every CTA's MMAs have finished reading it:
+// each MMA thread's commit arrives on that barrier in every CTA of the
+// cluster. Work per CTA and X traffic drop by CS.
 // ---------------------------------------------------------------------------
 
 constexpr int kQWorkers = 16;
 constexpr int kQFirstWorker = 3;   // warps 0-2: X loads, MMA, B loads
 constexpr int kQThreads = 32 * (kQFirstWorker + kQWorkers);
 
-// Shared memory of k_gemm_qa<RT> (byte offsets from a 1024-aligned base):
-// the X ring (kQX slots of 32 KB), the A ring (kQA stages of RT rows x 128
-// code bytes), the B ring (kQB stages of 256 rows x 128 bytes), the blocked
-// scale tiles of A and B per stage, the mbarriers. With RT = 64 the MMA
-// still reads 128 rows of A: a stage's last 64 rows are the next 8 KB of
-// shared memory (the next A stage, or the first B stage), whose products
-// land in accumulator rows that are never stored; the 8 KB saved per stage
-// buy a third B stage.
-template <int RT>
+// How a K = 256 stage (8 groups of 32 per row) is shared out for tiles of
+// RT rows in clusters of CS CTAs: each CTA quantizes kRows = RT / CS of the
+// rows; an X slot holds kSlotG of the 8 groups of those rows (kRows x 64
+// kSlotG bytes, boxes of 64 columns), so a stage takes kSlots slots; kTpg
+// adjacent worker threads share one group, each with kChunks of its four
+// 16-byte chunks (8 elements each). Without a cluster the 512 workers take
+// one group each (the slot holds 4 groups of 128 rows, or all 8 of 64);
+// in a cluster a slot holds the whole stage of a CTA's rows.
+template <int RT, int CS>
+struct QaSplit {
+  static constexpr int kRows = RT / CS;
+  static constexpr int kSlotG = CS > 1 ? 8 : (512 / RT < 8 ? 512 / RT : 8);
+  static constexpr int kSlots = 8 / kSlotG;
+  static constexpr int kTpg = 32 * kQWorkers / (kRows * kSlotG);
+  static constexpr int kChunks = 4 / kTpg;
+  static_assert(kRows % 16 == 0 && kSlotG % 2 == 0 && kTpg >= 1 && kTpg <= 4 &&
+                    kRows * kSlotG * kTpg == 32 * kQWorkers,
+                "work split");
+};
+
+// Shared memory of k_gemm_qa<RT, CS> (byte offsets from a 1024-aligned
+// base): the X ring (kQX slots, 96 KB in all), the A ring (kQA stages of RT
+// rows x 128 code bytes), the B ring (kQB stages of 256 rows x 128 bytes),
+// the blocked scale tiles of A and B per stage, the mbarriers. With RT = 64
+// the MMA still reads 128 rows of A: a stage's last 64 rows are the next
+// 8 KB of shared memory (the next A stage, or the first B stage), whose
+// products land in accumulator rows that are never stored; the 8 KB saved
+// per stage buy a third B stage.
+template <int RT, int CS>
 struct QaLayout {
-  static constexpr int kQX = 3, kQA = 2, kQB = RT == 64 ? 3 : 2;
-  static constexpr uint32_t kXSlot = 2 * kGM * 128;
+  static constexpr uint32_t kXSlot = QaSplit<RT, CS>::kRows * QaSplit<RT, CS>::kSlotG * 64;
   static constexpr uint32_t kAStage = RT * 128;
+  // ring depths: without a cluster 96 KB of X slots, two A stages and two B
+  // stages (three with 64-row tiles); in a cluster the X slots shrink with
+  // the CTA's share of the rows and the space goes to deeper A and B rings,
+  // which hide the longer trip of a stage through the cluster
+  static constexpr int kQX = CS > 1 ? (49152 / kXSlot > 2 ? 49152 / kXSlot : 2) : 98304 / kXSlot;
+  static constexpr int kQB = CS > 1 ? (RT == 64 ? 4 : 3) : (RT == 64 ? 3 : 2);
+  static constexpr uint32_t kFixed = kQX * kXSlot + kQB * (kPN * 128 + 2048) + 2048;
+  static constexpr int kQA =
+      CS > 1 ? (kFixed + 4 * (kAStage + 1024) <= 226 * 1024 ? 4 : 3) : 2;
   static constexpr uint32_t kBStage = kPN * 128;
   static constexpr uint32_t kX = 0;
   static constexpr uint32_t kA = kX + kQX * kXSlot;
@@ -641,66 +784,77 @@ struct QaLayout {
   static constexpr uint32_t kDrain = kAccEmpty + 8, kTmemBase = kDrain + 8;
   static constexpr uint32_t kFailed = kTmemBase + 4;
   static constexpr uint32_t kBytes = kFailed + 4;
-  static_assert(kA % 1024 == 0 && kB % 1024 == 0 && kAStage % 1024 == 0, "swizzle atoms");
+  static_assert(kXSlot % 1024 == 0 && kA % 1024 == 0 && kB % 1024 == 0 &&
+                    kAStage % 1024 == 0,
+                "swizzle atoms");
   static_assert(kA + (kQA - 1) * kAStage + kGM * 128 <= kSfa, "A padding rows in bounds");
 };
 
-// One 32-element group of X from its four 16-byte chunks (bf16, in order),
-// quantized as the rows quantizer does: the code chunk (element j in nibble
-// j % 8 of word j / 8) and the scale byte. Nearest rounding: the scaled
-// values v = x 2^-e come from one mixed-precision product of the bf16 input
-// with 2^-e (a normal bf16 power of two for every byte the OCP rule gives),
-// rounded once, the fp32 product the rows quantizer forms after widening.
-// Stochastic rounding (SR): bf16x8_sr_word, the rows quantizer's pair form,
-// with the group's counter base kh (its first pair index, keyed).
-template <bool SR>
-__device__ __forceinline__ uint4 qa_quantize_group(const uint4 (&w)[4], uint32_t& sb,
-                                                   uint32_t kh) {
-  uint32_t mx[8];
+// The part `part` (of TPG) of one 32-element group of X: its 4 / TPG
+// 16-byte chunks of bf16 (chunk 4 part / TPG + j in w[j]), quantized as the
+// rows quantizer does: code words out[j] (element i of the chunk in nibble
+// i) and the group's scale byte sb; the TPG threads of a group are adjacent
+// lanes and combine their maxima with shuffles. Nearest rounding: the
+// scaled values v = x 2^-e come from one mixed-precision product of the
+// bf16 input with 2^-e (a normal bf16 power of two for every byte the OCP
+// rule gives), rounded once, the fp32 product the rows quantizer forms
+// after widening. Stochastic rounding (SR): bf16x8_sr_word, the rows
+// quantizer's pair form, with the group's counter base kh (its first pair
+// index, keyed) and the chunk's index in the group.
+template <bool SR, int TPG>
+__device__ __forceinline__ void qa_quantize_part(const uint4 (&w)[4 / TPG], int part,
+                                                 uint32_t kh, uint32_t& sb,
+                                                 uint32_t (&out)[4 / TPG]) {
+  constexpr int NC = 4 / TPG;
+  uint32_t mx[2 * NC];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    mx[2 * k] = bf16x2_absmax_nan(w[k].x, w[k].y);
-    mx[2 * k + 1] = bf16x2_absmax_nan(w[k].z, w[k].w);
+  for (int j = 0; j < NC; ++j) {
+    mx[2 * j] = bf16x2_absmax_nan(w[j].x, w[j].y);
+    mx[2 * j + 1] = bf16x2_absmax_nan(w[j].z, w[j].w);
   }
 #pragma unroll
-  for (int n = 4; n >= 1; n /= 2)
+  for (int h = NC; h >= 1; h /= 2)
 #pragma unroll
-    for (int i = 0; i < n; ++i) mx[i] = bf16x2_absmax_nan(mx[i], mx[i + n]);
+    for (int i = 0; i < h; ++i) mx[i] = bf16x2_absmax_nan(mx[i], mx[i + h]);
+#pragma unroll
+  for (int o = 1; o < TPG; o *= 2)
+    mx[0] = bf16x2_absmax_nan(mx[0], __shfl_xor_sync(0xFFFFFFFFu, mx[0], o));
   const uint32_t mm = mx[0] & 0x7FFF7FFFu;
   sb = scale_byte(max(mm << 16, mm & 0xFFFF0000u));
   const unsigned short s16 = bf16_inv_scale(sb);
-  uint32_t out[4];
   if (SR) {
     const uint32_t sat2 = bf16x2_six_scale(sb);
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      out[k] = bf16x8_sr_word<false>(reinterpret_cast<const uint32_t*>(&w[k]), s16, sat2, kh,
-                                     uint32_t(k));
+    for (int j = 0; j < NC; ++j)
+      out[j] = bf16x8_sr_word<false>(reinterpret_cast<const uint32_t*>(&w[j]), s16, sat2, kh,
+                                     uint32_t(NC * part + j));
   } else {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t* q = reinterpret_cast<const uint32_t*>(&w[k]);
+    for (int j = 0; j < NC; ++j) {
+      const uint32_t* q = reinterpret_cast<const uint32_t*>(&w[j]);
       float v[8];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         v[2 * t] = bf16lo_mul(q[t], s16);
         v[2 * t + 1] = bf16hi_mul(q[t], s16);
       }
-      out[k] = e2m1x8_rn(v);
+      out[j] = e2m1x8_rn(v);
     }
   }
-  if (sb == 0xFFu) return make_uint4(0, 0, 0, 0);
-  return make_uint4(out[0], out[1], out[2], out[3]);
+  if (sb == 0xFFu)
+#pragma unroll
+    for (int j = 0; j < NC; ++j) out[j] = 0;
 }
 
-template <int RT, bool SR>
+template <int RT, int CS, bool SR>
 __global__ void __launch_bounds__(kQThreads, 1)
     k_gemm_qa(const __grid_constant__ CUtensorMap tm_x,
               const __grid_constant__ CUtensorMap tm_b,
               const uint8_t* __restrict__ sfb, int64_t m, int64_t n, int64_t k, RngKey key,
               float* __restrict__ c, uint8_t* __restrict__ a_codes,
               uint8_t* __restrict__ a_scales, int* __restrict__ status) {
-  using L = QaLayout<RT>;
+  using L = QaLayout<RT, CS>;
+  using P = QaSplit<RT, CS>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* const sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   auto bar = [&](uint32_t off, int i) {
@@ -708,17 +862,32 @@ __global__ void __launch_bounds__(kQThreads, 1)
   };
   int* const failed = reinterpret_cast<int*>(sm + L::kFailed);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this CTA's place: cluster `cid` of `ncl` works on tiles cid, cid + ncl, ..
+  const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
+  const int64_t cid = CS > 1 ? int64_t(cluster_index()) : int64_t(blockIdx.x);
+  const int64_t ncl = CS > 1 ? int64_t(cluster_count()) : int64_t(gridDim.x);
   const int64_t k_tiles = k / 128;
   const int64_t n_kb = k / 256;
   const int64_t n_row_tiles = (n + 127) / 128;
   const int64_t m_tiles = (m + RT - 1) / RT;
-  const int64_t n_col_tiles = (n + kPN - 1) / kPN;
-  const int64_t n_tiles = m_tiles * n_col_tiles;
-  // X slots per K = 256 stage, 64-column boxes per slot, K-elements per slot
-  constexpr int kSlots = RT == 128 ? 2 : 1;
-  constexpr int kBoxes = 4 / kSlots;
-  constexpr int kSlotK = 256 / kSlots;
-  static_assert(RT * 128 * kBoxes == L::kXSlot, "X slot size");
+  const int64_t n_col_groups = ((n + kPN - 1) / kPN + CS - 1) / CS;
+  const int64_t n_tiles = m_tiles * n_col_groups;
+  // tile t of the cluster: X rows from m0, this CTA's C columns from n0;
+  // first: the cluster's columns start at 0
+  auto coords = [&](int64_t t, int64_t& m0, int64_t& n0, bool& first) {
+    int64_t q0;
+    tile_coords(t, m_tiles, n_col_groups, m0, q0, RT);
+    first = q0 == 0;
+    n0 = q0 * CS + int64_t(rank) * kPN;
+  };
+  // a wait ran out: stop this CTA and, through their flags, the others of
+  // the cluster (which would wait for its stages)
+  auto fail = [&]() {
+    atomicExch(failed, 1);
+    if (CS > 1)
+      for (uint32_t d = 0; d < uint32_t(CS); ++d)
+        if (d != rank) st_cluster(cluster_addr(smem_u32(failed), d), 1u);
+  };
 
   if (tid == 0) {
     auto init = [&](uint32_t off, int i, uint32_t count) {
@@ -726,7 +895,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
                    "r"(count));
     };
     for (int i = 0; i < L::kQB; ++i) init(L::kFullB, i, 1), init(L::kEmptyB, i, 1);
-    for (int i = 0; i < L::kQA; ++i) init(L::kFullA, i, kQWorkers), init(L::kEmptyA, i, 1);
+    // a stage is full once every worker warp of the CTA has stored its
+    // share (in a cluster also: once its MMA thread has armed it with the
+    // other CTAs' bytes and those have come in), and free once every CTA's
+    // MMAs have read it
+    for (int i = 0; i < L::kQA; ++i)
+      init(L::kFullA, i, kQWorkers + (CS > 1 ? 1 : 0)), init(L::kEmptyA, i, CS);
     for (int i = 0; i < L::kQX; ++i) init(L::kXFull, i, 1), init(L::kXEmpty, i, kQWorkers);
     init(L::kAccFull, 0, 1);
     init(L::kAccEmpty, 0, kQWorkers);
@@ -742,6 +916,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;");
+  // every CTA's barriers are initialised before any other CTA arrives on them
+  if (CS > 1) cluster_sync_all();
   const uint32_t tmem = *reinterpret_cast<const uint32_t*>(sm + L::kTmemBase);
 
   if (warp == 0 || warp == 2) {
@@ -755,16 +931,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
       // load: every load lands before the CTA ends
       uint32_t issued = 0, last = 0;
       bool stop = false;
-      for (int64_t tile = blockIdx.x; tile < n_tiles && !stop; tile += gridDim.x) {
+      for (int64_t tile = cid; tile < n_tiles && !stop; tile += ncl) {
         int64_t m0, n0;
-        tile_coords(tile, m_tiles, n_col_tiles, m0, n0, RT);
+        bool first;
+        coords(tile, m0, n0, first);
+        // B's rows from n0; none when this column tile of the cluster lies
+        // past n (then the stage is marked full without a load: the MMAs
+        // read whatever the stage holds into accumulator columns that are
+        // never stored)
         const int64_t rb = n0 / 128;
-        const bool half1 = rb + 1 < n_row_tiles;
+        const bool half0 = rb < n_row_tiles, half1 = rb + 1 < n_row_tiles;
         const uint32_t bbytes = L::kBStage + (half1 ? 2048 : 1024);
-        const uint8_t* pb0 = sfb + rb * k_tiles * 512;
-        const uint8_t* pb1 = pb0 + k_tiles * 512;
         for (int64_t kb = 0; kb < n_kb && !stop; ++kb) {
-          for (int h = 0; h < (loads_x ? kSlots : 1); ++h) {
+          for (int h = 0; h < (loads_x ? P::kSlots : 1); ++h) {
             if (!wait_parity_or_failed<false>(bar(loads_x ? L::kXEmpty : L::kEmptyB, s),
                                               ph ^ 1u, failed)) {
               stop = true;
@@ -775,17 +954,27 @@ __global__ void __launch_bounds__(kQThreads, 1)
             if (loads_x) {
               unsigned long long* full = bar(L::kXFull, s);
               expect_tx(full, L::kXSlot);
+              // this CTA's rows (from m0 + rank kRows), the slot's kSlotG
+              // groups in boxes of 64 columns
+              const int64_t e0 = kb * 256 + 32 * P::kSlotG * h;
 #pragma unroll
-              for (int j = 0; j < kBoxes; ++j)
-                tma_load_2d(sm + L::kX + s * L::kXSlot + j * RT * 128, &tm_x,
-                            int((kb * 256 + kSlotK * h + 64 * j) * 2), int(m0), full);
+              for (int j = 0; j < P::kSlotG / 2; ++j)
+                tma_load_2d(sm + L::kX + s * L::kXSlot + j * P::kRows * 128, &tm_x,
+                            int((e0 + 64 * j) * 2), int(m0 + rank * P::kRows), full);
             } else {
               unsigned long long* full = bar(L::kFullB, s);
               uint8_t* sfb_s = sm + L::kSfb + s * 2048;
-              expect_tx(full, bbytes);
-              tma_load_2d(sm + L::kB + s * L::kBStage, &tm_b, int(kb) * 128, int(n0), full);
-              bulk_load(sfb_s, pb0 + kb * 1024, 1024, full);
-              if (half1) bulk_load(sfb_s + 1024, pb1 + kb * 1024, 1024, full);
+              if (half0) {
+                expect_tx(full, bbytes);
+                tma_load_2d(sm + L::kB + s * L::kBStage, &tm_b, int(kb) * 128, int(n0), full);
+                bulk_load(sfb_s, sfb + (rb * k_tiles + 2 * kb) * 512, 1024, full);
+                if (half1)
+                  bulk_load(sfb_s + 1024, sfb + ((rb + 1) * k_tiles + 2 * kb) * 512, 1024,
+                            full);
+              } else {
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(full))
+                             : "memory");
+              }
             }
             if (++s == uint32_t(ring)) {
               s = 0;
@@ -795,7 +984,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         if (failed_flag(failed)) stop = true;
       }
-      if (stop) atomicExch(failed, 1);
+      if (stop) fail();
       // drain (immediate unless a wait ran out)
       for (int st = 0; st < ring; ++st)
         if ((issued >> st) & 1u)
@@ -814,7 +1003,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
       uint32_t sa = 0, pha = 0, sb = 0, phb = 0;
       int64_t ti = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
+      // in a cluster, every A stage expects from the other CTAs their rows
+      // (RT / CS each) of 128 code bytes and two 4-byte scale words
+      constexpr uint32_t kStageBytes = (CS - 1) * P::kRows * (128 + 8);
+      if (CS > 1)
+        for (int i = 0; i < L::kQA; ++i) expect_tx(bar(L::kFullA, i), kStageBytes);
+      for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl, ++ti) {
         if (!wait_parity_or_failed<false>(bar(L::kAccEmpty, 0), uint32_t(ti & 1) ^ 1u,
                                           failed) ||
             failed_flag(failed)) {
@@ -824,9 +1018,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
         asm volatile("tcgen05.fence::after_thread_sync;");
         for (int64_t kb = 0; kb < n_kb; ++kb) {
           if (!wait_parity_or_failed<false>(bar(L::kFullB, sb), phb, failed) ||
-              !wait_parity_or_failed<false>(bar(L::kFullA, sa), pha, failed)) {
+              !(CS > 1 ? wait_cluster_or_failed(bar(L::kFullA, sa), pha, failed)
+                      : wait_parity_or_failed<false>(bar(L::kFullA, sa), pha, failed))) {
             ok = false;
             break;
+          }
+          if (CS > 1) {
+            // arm the stage's next use; the other CTAs' asynchronous stores
+            // that filled this one are ordered before the tensor cores' reads
+            expect_tx(bar(L::kFullA, sa), kStageBytes);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           }
           asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll
@@ -844,7 +1045,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
             mma_mxf4(tmem, a_d0 + (sa * kAStep + 2 * t), b_d0 + (sb * kBStep + 2 * t), idesc,
                      (kb == 0 && t == 0) ? 0u : 1u, tsfa, tsfb);
           }
-          commit_to(bar(L::kEmptyA, sa));
+          // the A stage is shared: free it in every CTA of the cluster
+          if (CS > 1)
+            commit_to_cluster(bar(L::kEmptyA, sa), uint16_t((1u << CS) - 1u));
+          else
+            commit_to(bar(L::kEmptyA, sa));
           commit_to(bar(L::kEmptyB, sb));
           if (++sa == uint32_t(L::kQA)) {
             sa = 0;
@@ -855,24 +1060,30 @@ __global__ void __launch_bounds__(kQThreads, 1)
             phb ^= 1u;
           }
         }
-        if (!ok) atomicExch(failed, 1);
+        if (!ok) fail();
         commit_to(bar(L::kAccFull, 0));
       }
-      if (!ok) atomicExch(failed, 1);
+      if (!ok) fail();
       // drain: every MMA and scale copy issued has completed
       commit_to(bar(L::kDrain, 0));
-      if (!wait_parity(bar(L::kDrain, 0), 0)) atomicExch(failed, 1);
+      if (!wait_parity(bar(L::kDrain, 0), 0)) fail();
     }
     __syncwarp();
   } else {
-    // workers: thread qt quantizes row qt % RT, group qt / RT of every X
-    // slot; warp w stores lane quarter w % 4, columns 64 ((w - 3) / 4) of
-    // every accumulator
+    // workers: thread qt works on part qt % kTpg of group g of row rl of
+    // every X slot (item qt / kTpg: g kRows + rl alone, rl 8 + g in a
+    // cluster, where the four groups of a scale word sit in adjacent
+    // lanes); rl is row r of the tile (row rank kRows + rl in a cluster);
+    // warp w stores lane quarter w % 4, columns 64 ((w - 3) / 4) of every
+    // accumulator
     const int qt = tid - 32 * kQFirstWorker;
-    const int r = qt % RT;
-    const int g = qt / RT;             // group of the slot: box g / 2, group g % 2 of it
-    const uint32_t sw = uint32_t(r & 7);
-    const uint8_t* xrow = sm + L::kX + (g >> 1) * RT * 128 + r * 128;
+    const int part = qt % P::kTpg;
+    const int item = qt / P::kTpg;
+    const int rl = CS > 1 ? item / 8 : item % P::kRows;
+    const int g = CS > 1 ? item % 8 : item / P::kRows;  // box g / 2, half g % 2 of it
+    const int r = int(rank) * P::kRows + rl;
+    const uint32_t sw = uint32_t(rl & 7);              // = r & 7
+    const uint8_t* xrow = sm + L::kX + (g >> 1) * P::kRows * 128 + rl * 128;
     const int q = warp & 3;
     const int cblk = (warp - kQFirstWorker) >> 2;
     uint32_t s = 0, ph = 0, xs = 0, xph = 0;
@@ -886,7 +1097,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                                                    wait_parity(bar(L::kAccFull, 0),
                                                                uint32_t(ti & 1),
                                                                kAccWaitLimit));
-      if (!got) atomicExch(failed, 1);
+      if (!got) fail();
       uint32_t v[64];
       if (got) {
         asm volatile("tcgen05.fence::after_thread_sync;");
@@ -936,44 +1147,79 @@ __global__ void __launch_bounds__(kQThreads, 1)
     };
 
     int64_t ti = 0;
-    for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++ti) {
+    for (int64_t tile = cid; tile < n_tiles && ok; tile += ncl, ++ti) {
       int64_t m0, n0;
-      tile_coords(tile, m_tiles, n_col_tiles, m0, n0, RT);
+      bool first;
+      coords(tile, m0, n0, first);
       const int64_t row = m0 + r;
-      const bool to_global = n0 == 0 && a_codes != nullptr && row < m;
+      const bool to_global = first && a_codes != nullptr && row < m;
       for (int64_t kb = 0; kb < n_kb; ++kb) {
-        // the A stage is free once the MMAs of its last use completed
+        // the A stage is free once the MMAs of its last use completed (in
+        // every CTA of the cluster)
         if (!__all_sync(0xFFFFFFFFu,
-                        wait_parity_or_failed<false>(bar(L::kEmptyA, s), ph ^ 1u, failed))) {
+                        CS > 1 ? wait_cluster_or_failed(bar(L::kEmptyA, s), ph ^ 1u, failed)
+                               : wait_parity_or_failed<false>(bar(L::kEmptyA, s), ph ^ 1u,
+                                                             failed))) {
           ok = false;
           break;
         }
-        uint8_t* const a_s = sm + L::kA + s * L::kAStage;
-        uint8_t* const sfa_s = sm + L::kSfa + s * 1024;
-        for (int h = 0; h < kSlots; ++h) {
+        const uint32_t a_s = smem_u32(sm + L::kA + s * L::kAStage);
+        const uint32_t sfa_s = smem_u32(sm + L::kSfa + s * 1024);
+        for (int h = 0; h < P::kSlots; ++h) {
           if (!__all_sync(0xFFFFFFFFu,
                           wait_parity_or_failed<false>(bar(L::kXFull, xs), xph, failed))) {
             ok = false;
             break;
           }
           const uint8_t* xr = xrow + xs * L::kXSlot;
-          uint4 w[4];
+          uint4 w[P::kChunks];
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            w[j] = *reinterpret_cast<const uint4*>(xr + (((4 * (g & 1) + j) ^ sw) << 4));
-          const int G = (8 / kSlots) * h + g;  // group within the stage's 256
+          for (int j = 0; j < P::kChunks; ++j)
+            w[j] = *reinterpret_cast<const uint4*>(
+                xr + (((4 * (g & 1) + P::kChunks * part + j) ^ sw) << 4));
+          // the group within the stage's 8
+          const int G = P::kSlotG * h + g;
           uint32_t kh = 0;
           if (SR) {  // the group's first pair index, row-major over X
             const uint64_t p0 = uint64_t(row * (k / 32) + kb * 8 + G) * 16u;
             kh = inner_key(key, uint32_t(p0 >> 32)) + uint32_t(p0);
           }
-          uint32_t scb;
-          const uint4 code = qa_quantize_group<SR>(w, scb, kh);
-          *reinterpret_cast<uint4*>(a_s + r * 128 + ((uint32_t(G) ^ sw) << 4)) = code;
-          sfa_s[512 * (G >> 2) + 16 * (r & 31) + 4 * (r >> 5) + (G & 3)] = uint8_t(scb);
+          uint32_t scb, code[P::kChunks];
+          qa_quantize_part<SR, P::kTpg>(w, part, kh, scb, code);
+          const uint32_t code_off = r * 128 + ((uint32_t(G) ^ sw) << 4) + 4 * P::kChunks * part;
+          const uint32_t sc_off = 512 * (G >> 2) + 16 * (r & 31) + 4 * (r >> 5);
+          if constexpr (CS > 1) {
+            // the scale word of groups 4t .. 4t+3 (t = G / 4) of row r,
+            // gathered in the lane of group 4t, part 0
+            uint32_t word = scb << (8 * (G & 3));
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, P::kTpg);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2 * P::kTpg);
+            const bool word_lane = (G & 3) == 0 && part == 0;
+            // into this CTA's operand stage, and asynchronously into every
+            // other CTA's, whose stage barrier counts the bytes
+            st_smem(a_s + code_off, code);
+            if (word_lane) st_smem(sfa_s + sc_off, word);
+            const uint32_t fa = smem_u32(bar(L::kFullA, s));
+#pragma unroll
+            for (int j = 1; j < CS; ++j) {
+              const uint32_t d = (rank + uint32_t(j)) % uint32_t(CS);
+              const uint32_t bd = cluster_addr(fa, d);
+              st_async(cluster_addr(a_s + code_off, d), code, bd);
+              if (word_lane) st_async(cluster_addr(sfa_s + sc_off, d), word, bd);
+            }
+          } else {
+            st_smem(a_s + code_off, code);
+            if (part == 0) st_smem_u8(sfa_s + sc_off + (G & 3), scb);
+          }
           if (to_global) {
-            *reinterpret_cast<uint4*>(a_codes + row * (k / 2) + kb * 128 + 16 * G) = code;
-            a_scales[row * (k / 32) + kb * 8 + G] = uint8_t(scb);
+            uint8_t* gc = a_codes + row * (k / 2) + kb * 128 + 16 * G + 4 * P::kChunks * part;
+            if constexpr (P::kChunks == 4)
+              *reinterpret_cast<uint4*>(gc) = make_uint4(code[0], code[1], code[2], code[3]);
+            else if constexpr (P::kChunks == 2)
+              *reinterpret_cast<uint2*>(gc) = make_uint2(code[0], code[1]);
+            else
+              *reinterpret_cast<uint32_t*>(gc) = code[0];
+            if (part == 0) a_scales[row * (k / 32) + kb * 8 + G] = uint8_t(scb);
           }
           // release the X slot after the stores that depend on every value
           // loaded from it: a thread's arrival does not wait for its shared
@@ -990,8 +1236,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
           }
         }
         if (!ok) break;
-        // the stage's codes and scales were written through the generic
-        // proxy; the tensor cores read them through the async proxy
+        // this CTA's share of the stage was written through the generic
+        // proxy; the tensor cores read it through the async proxy
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0)
@@ -1012,11 +1258,19 @@ __global__ void __launch_bounds__(kQThreads, 1)
       if (!ok) break;
       pend_ti = ti, pend_m0 = m0, pend_n0 = n0;
     }
-    if (!ok) atomicExch(failed, 1);
+    if (!ok) fail();
     if (pend_ti >= 0) drain_tile(pend_ti, pend_m0, pend_n0);
   }
+  // after a timeout, asynchronous stores of this cluster may still be on
+  // their way to a CTA that stopped waiting for them: let them land before
+  // any CTA of the cluster can leave (they take microseconds)
+  if (CS > 1 && failed_flag(failed))
+    for (int i = 0; i < 100; ++i) __nanosleep(1000);
   asm volatile("tcgen05.fence::before_thread_sync;");
   __syncthreads();
+  // no CTA leaves while another of the cluster may still store into its
+  // shared memory or arrive on its barriers
+  if (CS > 1) cluster_sync_all();
   report_failure(status, failed);
   if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
@@ -1089,25 +1343,63 @@ cudaError_t launch_gemm_mxf4(const uint8_t* a, const uint8_t* a_scales,
 
 namespace {
 
-template <int RT, bool SR>
+template <int RT, int CS, bool SR>
 cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, RngKey key,
                          const uint8_t* b, const uint8_t* b_scales, float* c, uint8_t* a_codes,
                          uint8_t* a_scales, int* status, cudaStream_t s) {
   // X as a byte array [m][2k] for the TMA: 128-byte boxes of 64 bf16
   CUtensorMap mx, mb;
-  if (!encode_rows_sw128(&mx, x, m, 2 * k, RT) || !encode_codes_map(&mb, b, n, k, kPN))
+  if (!encode_rows_sw128(&mx, x, m, 2 * k, QaSplit<RT, CS>::kRows) ||
+      !encode_codes_map(&mb, b, n, k, kPN))
     return cudaErrorInvalidValue;
-  constexpr size_t smem = QaLayout<RT>::kBytes + 1024;
+  constexpr size_t smem = QaLayout<RT, CS>::kBytes + 1024;
   static_assert(smem <= 227 * 1024, "fused GEMM shared memory");
-  auto kern = k_gemm_qa<RT, SR>;
+  auto kern = k_gemm_qa<RT, CS, SR>;
   cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  const int64_t tiles = ((m + RT - 1) / RT) * ((n + kPN - 1) / kPN);
-  const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kQThreads, smem, tiles);
-  kern<<<grid, kQThreads, smem, s>>>(mx, mb, b_scales, m, n, k, key, c, a_codes, a_scales,
-                                     status);
-  return cudaGetLastError();
+  // tiles of a cluster: RT rows x CS column tiles
+  const int64_t tiles = ((m + RT - 1) / RT) * (((n + kPN - 1) / kPN + CS - 1) / CS);
+  if (CS == 1) {
+    const int grid = persistent_grid(reinterpret_cast<const void*>(kern), kQThreads, smem, tiles);
+    kern<<<grid, kQThreads, smem, s>>>(mx, mb, b_scales, m, n, k, key, c, a_codes, a_scales,
+                                       status);
+    return cudaGetLastError();
+  }
+  // persistent clusters: as many as can be resident at once
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cfg.gridDim = dim3(unsigned(sms / CS * CS));
+  int clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  cfg.gridDim = dim3(unsigned((tiles < clusters ? tiles : clusters) * CS));
+  return cudaLaunchKernelEx(&cfg, kern, mx, mb, b_scales, m, n, k, key, c, a_codes, a_scales,
+                            status);
+}
+
+template <int RT, bool SR>
+cudaError_t gemm_qa_cluster(int cs, const void* x, int64_t m, int64_t n, int64_t k, RngKey key,
+                            const uint8_t* b, const uint8_t* b_scales, float* c,
+                            uint8_t* a_codes, uint8_t* a_scales, int* status, cudaStream_t s) {
+  if (cs == 4)
+    return gemm_qa_impl<RT, 4, SR>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales, status, s);
+  if (cs == 2)
+    return gemm_qa_impl<RT, 2, SR>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales, status, s);
+  return gemm_qa_impl<RT, 1, SR>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales, status, s);
 }
 
 }  // namespace
@@ -1118,20 +1410,25 @@ cudaError_t launch_gemm_qa(const void* x, int64_t m, int64_t n, int64_t k, bool 
                            cudaStream_t s) {
   if (k % 256) return cudaErrorInvalidValue;
   const RngKey key = make_key(seed, 0);
-  // 64-row tiles where 128-row ones would not give every SM a tile
+  // clusters of up to 4 CTAs share the quantization of their rows over as
+  // many column tiles; 64-row tiles where they all run at once (a 64-row
+  // tile takes about 0.8 of a 128-row one, so 128-row tiles win as soon as
+  // the 64-row ones would need a second wave)
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles128 = ((m + 127) / 128) * ((n + kPN - 1) / kPN);
-  if (tiles128 < sms)
-    return sr ? gemm_qa_impl<64, true>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
-                                       status, s)
-              : gemm_qa_impl<64, false>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
-                                        status, s);
-  return sr ? gemm_qa_impl<128, true>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
-                                      status, s)
-            : gemm_qa_impl<128, false>(x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
-                                       status, s);
+  const int64_t col_tiles = (n + kPN - 1) / kPN;
+  const int cs = col_tiles >= 4 ? 4 : (col_tiles >= 2 ? 2 : 1);
+  const int64_t ctas64 = ((m + 63) / 64) * ((col_tiles + cs - 1) / cs) * cs;
+  if (ctas64 <= sms)
+    return sr ? gemm_qa_cluster<64, true>(cs, x, m, n, k, key, b, b_scales, c, a_codes,
+                                          a_scales, status, s)
+              : gemm_qa_cluster<64, false>(cs, x, m, n, k, key, b, b_scales, c, a_codes,
+                                           a_scales, status, s);
+  return sr ? gemm_qa_cluster<128, true>(cs, x, m, n, k, key, b, b_scales, c, a_codes, a_scales,
+                                         status, s)
+            : gemm_qa_cluster<128, false>(cs, x, m, n, k, key, b, b_scales, c, a_codes,
+                                          a_scales, status, s);
 }
 
 }  // namespace mxfp4

@@ -7,6 +7,10 @@ the two-step path it replaces and against the oracle.
 - C equals mxfp4_gemm on those codes bit for bit (same tiles, same MMA
   sequence) and lies within the fp32 accumulation bound of the oracle's
   exact product: (k - 1) 2^-24 sum_j |a_j b_j|.
+
+The shapes reach every tile form of the kernel: 64- and 128-row tiles, alone
+or in clusters of 2 or 4 CTAs that share the quantization of their rows
+(more than one column tile of 256), with column tiles of a cluster past n.
 """
 import numpy as np
 import pytest
@@ -51,7 +55,16 @@ def check_against_oracle(c, xc, xs, wc, ws, k, rows=None):
                                  (9000, 512, 256), (20000, 520, 256),
                                  # one row; two weight rows; n not a multiple of 4
                                  # (scalar stores of C)
-                                 (1, 256, 256), (65, 2, 512), (100, 130, 256)])
+                                 (1, 256, 256), (65, 2, 512), (100, 130, 256),
+                                 # 128-row tiles without clusters (149 row tiles)
+                                 (19000, 200, 256),
+                                 # clusters of 4 CTAs sharing the quantization of
+                                 # their rows: 64-row tiles; 128-row tiles with the
+                                 # second cluster's last three column tiles past n
+                                 (300, 1024, 512), (5000, 1100, 512),
+                                 # clusters of 2 over 3 column tiles (one CTA of the
+                                 # last cluster past n), rows not a multiple of 64
+                                 (4100, 700, 768)])
 def test_fused_equals_quantize_then_gemm(mnk):
     mm, nn, k = mnk
     x = W.normal_bf16(mm, k, 21, 0.005, 50.0)
@@ -116,7 +129,7 @@ def test_fused_on_the_sweep_activation(n):
 
 
 @pytest.mark.parametrize("mnk", [(200, 136, 512), (9000, 512, 256), (20000, 520, 256),
-                                 (384, 1024, 2560)])
+                                 (384, 1024, 2560), (5000, 1100, 512), (19000, 200, 256)])
 def test_fused_stochastic_rounding(mnk):
     """Q_S(X) in the load stage (a gradient for a backward GEMM): the codes of
     mxfp4_quantize with the same seed, and the two-step C."""
