@@ -376,10 +376,12 @@ mxfp4_status mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
  *   status    device int or NULL, as in mxfp4_gemm; when it is set, the
  *             tiles of C that were not completed hold NaN or were left
  *             unwritten
- * k must be a multiple of 256; m, n > 0 within the size limit. X is read
- * and quantized once per 256 columns of C (tiles that run together share
- * it through L2), so the fusion pays where n is small; for large n the
- * separate quantize + mxfp4_gemm is faster.
+ * k must be a multiple of 256; m, n > 0 within the size limit. With more
+ * than 256 columns of C, clusters of 2 or 4 CTAs (up to 1024 columns) share
+ * the quantization of their rows, so X is read and quantized once per 1024
+ * columns; the fusion pays where n is small (up to a few hundred to about
+ * a thousand columns on B200); for large n the separate quantize +
+ * mxfp4_gemm is faster.
  */
 mxfp4_status mxfp4_gemm_quantize_a(const void* x, int64_t m, int64_t n, int64_t k,
                                    int rounding, uint64_t seed, const uint8_t* b_codes,

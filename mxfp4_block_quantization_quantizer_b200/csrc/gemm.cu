@@ -622,22 +622,15 @@ __device__ __forceinline__ bool wait_cluster_or_failed(unsigned long long* bar,
   }
   return false;
 }
-// Stores to this CTA's shared memory (a shared::cta address).
-__device__ __forceinline__ void st_smem_u8(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u8 [%0], %1;" ::"r"(a), "h"(static_cast<unsigned short>(v))
-               : "memory");
+// The code words v (4, 8 or 16 bytes) to p, in one store.
+__device__ __forceinline__ void put_words(uint8_t* p, const uint32_t (&v)[1]) {
+  *reinterpret_cast<uint32_t*>(p) = v[0];
 }
-__device__ __forceinline__ void st_smem(uint32_t a, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+__device__ __forceinline__ void put_words(uint8_t* p, const uint32_t (&v)[2]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(v[0], v[1]);
 }
-__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[1]) { st_smem(a, v[0]); }
-__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[2]) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(v[0]), "r"(v[1]) : "memory");
-}
-__device__ __forceinline__ void st_smem(uint32_t a, const uint32_t (&v)[4]) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[0]), "r"(v[1]),
-               "r"(v[2]), "r"(v[3])
-               : "memory");
+__device__ __forceinline__ void put_words(uint8_t* p, const uint32_t (&v)[4]) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 // A plain store to another CTA's shared memory (a from cluster_addr).
 __device__ __forceinline__ void st_cluster(uint32_t a, uint32_t v) {
@@ -1163,8 +1156,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t a_s = smem_u32(sm + L::kA + s * L::kAStage);
-        const uint32_t sfa_s = smem_u32(sm + L::kSfa + s * 1024);
+        uint8_t* const a_s = sm + L::kA + s * L::kAStage;
+        uint8_t* const sfa_s = sm + L::kSfa + s * 1024;
         for (int h = 0; h < P::kSlots; ++h) {
           if (!__all_sync(0xFFFFFFFFu,
                           wait_parity_or_failed<false>(bar(L::kXFull, xs), xph, failed))) {
@@ -1197,28 +1190,23 @@ __global__ void __launch_bounds__(kQThreads, 1)
             const bool word_lane = (G & 3) == 0 && part == 0;
             // into this CTA's operand stage, and asynchronously into every
             // other CTA's, whose stage barrier counts the bytes
-            st_smem(a_s + code_off, code);
-            if (word_lane) st_smem(sfa_s + sc_off, word);
+            put_words(a_s + code_off, code);
+            if (word_lane) *reinterpret_cast<uint32_t*>(sfa_s + sc_off) = word;
             const uint32_t fa = smem_u32(bar(L::kFullA, s));
+            const uint32_t ca = smem_u32(a_s + code_off), wa = smem_u32(sfa_s + sc_off);
 #pragma unroll
             for (int j = 1; j < CS; ++j) {
               const uint32_t d = (rank + uint32_t(j)) % uint32_t(CS);
               const uint32_t bd = cluster_addr(fa, d);
-              st_async(cluster_addr(a_s + code_off, d), code, bd);
-              if (word_lane) st_async(cluster_addr(sfa_s + sc_off, d), word, bd);
+              st_async(cluster_addr(ca, d), code, bd);
+              if (word_lane) st_async(cluster_addr(wa, d), word, bd);
             }
           } else {
-            st_smem(a_s + code_off, code);
-            if (part == 0) st_smem_u8(sfa_s + sc_off + (G & 3), scb);
+            put_words(a_s + code_off, code);
+            if (part == 0) sfa_s[sc_off + (G & 3)] = uint8_t(scb);
           }
           if (to_global) {
-            uint8_t* gc = a_codes + row * (k / 2) + kb * 128 + 16 * G + 4 * P::kChunks * part;
-            if constexpr (P::kChunks == 4)
-              *reinterpret_cast<uint4*>(gc) = make_uint4(code[0], code[1], code[2], code[3]);
-            else if constexpr (P::kChunks == 2)
-              *reinterpret_cast<uint2*>(gc) = make_uint2(code[0], code[1]);
-            else
-              *reinterpret_cast<uint32_t*>(gc) = code[0];
+            put_words(a_codes + row * (k / 2) + kb * 128 + 16 * G + 4 * P::kChunks * part, code);
             if (part == 0) a_scales[row * (k / 32) + kb * 8 + G] = uint8_t(scb);
           }
           // release the X slot after the stores that depend on every value
