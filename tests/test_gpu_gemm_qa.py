@@ -46,13 +46,16 @@ def check_against_oracle(c, xc, xs, wc, ws, k, rows=None):
 
 @pytest.mark.parametrize("mnk", [(128, 256, 256),    # one tile, one stage
                                  (200, 136, 512),    # ragged rows and columns
-                                 (384, 520, 768),    # 3 x 3 tiles, a 8-column edge tile
+                                 # 3 x 3 tiles, a 8-column edge tile (64-row
+                                 # tiles in clusters of 2)
+                                 (384, 520, 768),
                                  (1000, 64, 1024),   # narrow output, many row tiles
                                  (256, 768, 2560),   # 10 stages: the rings wrap
-                                 # several tiles per CTA with one stage each (the
-                                 # accumulator drained after the next tile's only
-                                 # stage): 64-row tiles, then 128-row tiles
-                                 (9000, 512, 256), (20000, 520, 256),
+                                 # several tiles per CTA (or cluster) with one stage
+                                 # each (the accumulator drained after the next
+                                 # tile's only stage): one CTA per tile, clusters of 2;
+                                 # one tile per cluster of 2
+                                 (40000, 200, 256), (20000, 520, 256), (9000, 512, 256),
                                  # one row; two weight rows; n not a multiple of 4
                                  # (scalar stores of C)
                                  (1, 256, 256), (65, 2, 512), (100, 130, 256),
