@@ -741,13 +741,13 @@ struct QaSplit {
 };
 
 // Shared memory of k_gemm_qa<RT, CS> (byte offsets from a 1024-aligned
-// base): the X ring (kQX slots, 96 KB in all), the A ring (kQA stages of RT
-// rows x 128 code bytes), the B ring (kQB stages of 256 rows x 128 bytes),
-// the blocked scale tiles of A and B per stage, the mbarriers. With RT = 64
-// the MMA still reads 128 rows of A: a stage's last 64 rows are the next
-// 8 KB of shared memory (the next A stage, or the first B stage), whose
-// products land in accumulator rows that are never stored; the 8 KB saved
-// per stage buy a third B stage.
+// base): the X ring (kQX slots), the A ring (kQA stages of RT rows x 128
+// code bytes), the B ring (kQB stages of 256 rows x 128 bytes), the blocked
+// scale tiles of A and B per stage, the mbarriers. With RT = 64 the MMA
+// still reads 128 rows of A: a stage's last 64 rows are the next 8 KB of
+// shared memory (the next A stage, or the first B stage), whose products
+// land in accumulator rows that are never stored; the 8 KB saved per stage
+// buy a deeper B ring.
 template <int RT, int CS>
 struct QaLayout {
   static constexpr uint32_t kXSlot = QaSplit<RT, CS>::kRows * QaSplit<RT, CS>::kSlotG * 64;
