@@ -112,6 +112,31 @@ def test_fuzz_fused_gemm(case):
         assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
 
 
+@pytest.mark.parametrize("i", range(16), ids=lambda i: "case%d" % i)
+def test_fuzz_fused_gemm_clusters(i):
+    """More than one column tile of C (clusters of 2 or 4 CTAs sharing the
+    quantization of their rows), 64- or 128-row tiles, ragged m and n."""
+    g = np.random.Generator(np.random.PCG64(4500 + i))
+    mm = int(g.integers(1, 12000))
+    n = int(g.integers(257, 2100))
+    k = 256 * int(g.integers(1, 5))
+    seed = int(g.integers(0, 2**32))
+    x = g.standard_normal((mm, k)) * np.exp2(g.integers(-8, 8, size=(mm, k)))
+    xd = to_dev(x.astype(np.float32).astype(BF16))
+    wc, ws = m.quantize(to_dev(g.standard_normal((n, k)).astype(np.float32).astype(BF16)),
+                        m.ROWS, m.RNE)
+    wb = m.scales_to_blocked(ws)
+    for rnd in (m.RNE, m.SR):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        c, ac, as_ = m.gemm_quantize_a(xd, wc, wb, rounding=rnd, seed=seed, want_a=True,
+                                       status=st)
+        assert int(st.item()) == 0
+        qc, qs = m.quantize(xd, m.ROWS, rnd, seed)
+        assert torch.equal(ac, qc) and torch.equal(as_, qs)
+        ref = m.gemm(qc, m.scales_to_blocked(qs), wc, wb, k)
+        assert torch.equal(c.view(torch.int32), ref.view(torch.int32))
+
+
 def tracker_weights(g, rows, cols):
     """fp32 weights with one group maximum per group (a fixed scale) and many
     values near a rounding edge, like the tracker workload."""
