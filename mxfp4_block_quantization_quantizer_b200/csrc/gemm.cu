@@ -1369,11 +1369,17 @@ cudaError_t gemm_qa_impl(const void* x, int64_t m, int64_t n, int64_t k, RngKey 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cfg.gridDim = dim3(unsigned(sms / CS * CS));
-  int clusters = 0;
-  e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-  if (e != cudaSuccess) return e;
-  if (clusters < 1) return cudaErrorInvalidConfiguration;
+  // the number of resident clusters, asked once per device (the query
+  // costs more host time than the launch)
+  static int resident[64] = {};
+  int clusters = dev >= 0 && dev < 64 ? resident[dev] : 0;
+  if (clusters < 1) {
+    cfg.gridDim = dim3(unsigned(sms / CS * CS));
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) resident[dev] = clusters;
+  }
   cfg.gridDim = dim3(unsigned((tiles < clusters ? tiles : clusters) * CS));
   return cudaLaunchKernelEx(&cfg, kern, mx, mb, b_scales, m, n, k, key, c, a_codes, a_scales,
                             status);
