@@ -171,3 +171,35 @@ def test_fused_stochastic_rounding_on_the_sweep():
         oc, os_ = O.quantize(x[r:r + 1], O.ROWS, O.SR, 5, row0=r)
         assert np.array_equal(acn[r:r + 1], oc) and np.array_equal(asn[r:r + 1], os_)
         check_against_oracle(cn[r:r + 1], oc, os_, to_np(wc), to_np(ws), K)
+
+
+@pytest.mark.parametrize("mnk", [(200, 136, 512),     # one CTA per tile
+                                 (384, 520, 768),     # clusters of 2, a CTA past n
+                                 (300, 1100, 512),    # clusters of 4, three CTAs past n
+                                 (5000, 1100, 256)])  # the same with 128-row tiles
+def test_fused_outputs_stay_inside_their_buffers(mnk):
+    """C and the optional Q(X) outputs written into guarded buffers: the
+    canary bytes around each are untouched (rows past m, column tiles of a
+    cluster past n) and the results equal an unguarded call."""
+    mm, nn, k = mnk
+    xd = to_dev(W.normal_bf16(mm, k, 27, 0.005, 50.0))
+    wc, ws = weight(nn, k, 28)
+    wb = m.scales_to_blocked(ws)
+    pad, canary = 4096, 0xA5
+
+    def guarded(nbytes):
+        buf = torch.full((nbytes + 2 * pad,), canary, dtype=torch.uint8, device="cuda")
+        return buf, buf[pad:pad + nbytes]
+
+    cbuf, cv = guarded(4 * mm * nn)
+    abuf, av = guarded(mm * k // 2)
+    sbuf, sv = guarded(mm * k // 32)
+    out = (cv.view(torch.float32).view(mm, nn), av.view(mm, k // 2), sv.view(mm, k // 32))
+    for rnd in (m.RNE, m.SR):
+        m.gemm_quantize_a(xd, wc, wb, rounding=rnd, seed=3, out=out, want_a=True)
+        ref_c, ref_a, ref_s = m.gemm_quantize_a(xd, wc, wb, rounding=rnd, seed=3, want_a=True)
+        for b in (cbuf, abuf, sbuf):
+            h = to_np(b)
+            assert np.all(h[:pad] == canary) and np.all(h[-pad:] == canary)
+        assert torch.equal(out[0].view(torch.int32), ref_c.view(torch.int32))
+        assert torch.equal(out[1], ref_a) and torch.equal(out[2], ref_s)
